@@ -1,0 +1,118 @@
+"""Seeded synthetic inputs shared by the tests, the benchmark and the oracle checks.
+
+This module draws random numbers and shapes them into the workloads; it holds
+none of the loss or log-probability arithmetic.  Every tensor is produced on the
+CPU by a seeded ``torch.Generator`` (fp32 master values, then rounded to
+nearest-even into the working dtype), so the GPU path and the oracle always see
+the same bits.
+
+Recipes (N(mu, sigma): sigma is the standard deviation; "uniform in [a, b]" on
+integers includes both ends):
+
+* loss-only: policy = -2|N(0,1)|, old = policy + N(0,0.1), ref = policy + N(0,0.05),
+  advantages N(0,1) per sequence (fp32), int8 prefix mask with lengths uniform in
+  the given range;
+* fused linear: X ~ N(0,1) [N,H], W ~ N(0,0.02) [V,H], Xref = X + N(0,0.01),
+  Wref = W + N(0,0.002), optional bias ~ N(0,0.01), targets uniform in [0,V),
+  advantages N(0,1) per sequence, prefix mask, and the N(0,0.1) noise that is
+  added to the policy log-prob to make the behaviour log-probs (old_lp).
+
+Seeds are ``0x5EED0000 + 16*workload + variant``.
+"""
+from __future__ import annotations
+
+import torch
+
+SEED_BASE = 0x5EED0000
+
+
+def seed_for(workload: int, variant: int = 0) -> int:
+    return SEED_BASE + 16 * workload + variant
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def normal(shape, seed: int, std: float = 1.0, mean: float = 0.0) -> torch.Tensor:
+    x = torch.randn(tuple(shape), generator=_gen(seed), dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    if mean != 0.0:
+        x.add_(mean)
+    return x
+
+
+def randint(shape, lo: int, hi_inclusive: int, seed: int) -> torch.Tensor:
+    return torch.randint(lo, hi_inclusive + 1, tuple(shape), generator=_gen(seed),
+                         dtype=torch.int64)
+
+
+def prefix_mask(lengths: torch.Tensor, T: int) -> torch.Tensor:
+    """int8 [bs, T] mask whose row b has its first lengths[b] entries set."""
+    pos = torch.arange(T, dtype=torch.int64).unsqueeze(0)
+    return (pos < lengths.to(torch.int64).unsqueeze(1)).to(torch.int8)
+
+
+def loss_inputs(bs: int, seq: int, dtype: torch.dtype, seed: int,
+                len_lo: int = 64, len_hi: int = 1024) -> dict:
+    """Log-prob inputs for the loss-only kernel (all on CPU)."""
+    s = int(seed)
+    pol = normal((bs, seq), s + 1).abs_().mul_(-2.0)
+    old = pol + normal((bs, seq), s + 2, std=0.1)
+    ref = pol + normal((bs, seq), s + 3, std=0.05)
+    adv = normal((bs,), s + 4)
+    lens = randint((bs,), min(len_lo, seq), min(len_hi, seq), s + 5)
+    return {
+        "policy_lp": pol.to(dtype), "old_lp": old.to(dtype), "ref_lp": ref.to(dtype),
+        "adv": adv, "mask": prefix_mask(lens, seq), "lengths": lens,
+    }
+
+
+def fused_inputs(bs: int, T: int, H: int, V: int, dtype: torch.dtype, seed: int, *,
+                 bias: bool = False, len_lo: int = 1, len_hi: int | None = None,
+                 fully_masked_last: bool = False, need_ref: bool = True) -> dict:
+    """Inputs of the fused linear path (all on CPU).  ``old_noise`` is the
+    N(0,0.1) term the caller adds to the policy log-prob to form old_lp."""
+    s = int(seed)
+    N = bs * T
+    len_hi = T if len_hi is None else len_hi
+    X32 = normal((N, H), s + 1)
+    W32 = normal((V, H), s + 2, std=0.02)
+    out = {"X": X32.to(dtype), "W": W32.to(dtype)}
+    if need_ref:
+        out["Xref"] = (X32 + normal((N, H), s + 3, std=0.01)).to(dtype)
+        out["Wref"] = (W32 + normal((V, H), s + 4, std=0.002)).to(dtype)
+    else:
+        out["Xref"] = None
+        out["Wref"] = None
+    del X32, W32
+    out["bias"] = normal((V,), s + 5, std=0.01).to(dtype) if bias else None
+    out["targets"] = randint((N,), 0, V - 1, s + 6)
+    out["adv"] = normal((bs,), s + 7)
+    lens = randint((bs,), min(len_lo, T), min(len_hi, T), s + 8)
+    if fully_masked_last and bs > 0:
+        lens[bs - 1] = 0
+    out["lengths"] = lens
+    out["mask"] = prefix_mask(lens, T)
+    out["old_noise"] = normal((N,), s + 9, std=0.1)
+    return out
+
+
+# The workloads, by number, as (kind, shape) records.
+WORKLOADS = {
+    0: dict(kind="fused", bs=2, T=16, H=64, V=512, dtype=torch.bfloat16, len_lo=1, len_hi=16,
+            eps_lo=0.2, eps_hi=0.28, beta=0.04),
+    1: dict(kind="loss", bs=16, seq=1024, len_lo=64, len_hi=1024, eps_lo=0.2, eps_hi=0.28,
+            beta=0.04),
+    2: dict(kind="fused", bs=1, T=1024, H=4096, V=128256, dtype=torch.bfloat16, len_lo=256,
+            len_hi=1024, eps_lo=0.2, eps_hi=0.28, beta=0.04),
+    3: dict(kind="fused", bs=4, T=1024, H=4096, V=128256, dtype=torch.float16, bias=True,
+            len_lo=256, len_hi=1024, eps_lo=0.2, eps_hi=0.28, beta=0.04),
+    4: dict(kind="fused", bs=8, T=1024, H=4096, V=128256, dtype=torch.bfloat16, len_lo=1,
+            len_hi=1024, fully_masked_last=True, eps_lo=0.2, eps_hi=0.28, beta=0.04),
+    5: dict(kind="fused", bs=8, T=1024, H=4000, V=152064, dtype=torch.bfloat16, len_lo=1,
+            len_hi=1024, fully_masked_last=True, eps_lo=0.2, eps_hi=0.28, beta=0.04),
+}
