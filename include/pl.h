@@ -1,0 +1,195 @@
+/*
+ * pl.h -- C ABI of the B200 (sm_100a) fused GRPO/BNPO policy-loss library (libpl.so).
+ *
+ * Two forms of one hot path, both defined by the pages this library restates:
+ *
+ *   pl_loss / pl_loss_ex -- the loss-only kernel on precomputed log-probs:
+ *       ratio     = exp(policy_lp - old_lp)
+ *       clipped   = clip(ratio, 1 - eps_lo, 1 + eps_hi)
+ *       per_token = -adv[b] * min(ratio, clipped)
+ *       kl        = exp(ref_lp - policy_lp) - (ref_lp - policy_lp) - 1
+ *       BNPO: loss = sum(mask * (per_token + beta*kl)) / max(sum(mask), 1)
+ *       GRPO: loss = mean_b( sum_t(mask * (per_token + beta*kl)) / max(sum_t mask, 1) )
+ *     ("Geometric-AI Kernels" model card, sections "BNPO Loss" and "GRPO Loss";
+ *      the fused forward+backward returning (loss, grad_logprobs) and the
+ *      forward-only variant are the card's "Entry points" section).
+ *
+ *   pl_fused_linear_grpo -- the fused linear path: hidden states x lm_head weight ->
+ *     per-token log-prob of the sampled token (logsumexp over the whole vocabulary,
+ *     temperature 1.0) for the policy and the reference model -> the loss above ->
+ *     grad_logits = g * (onehot - softmax) -> dX, dW, dbias, in row chunks of at
+ *     most 1024 with fp32 weight-gradient accumulation across chunks
+ *     ("Add SM100 CuTe DSL GRPO fast path", Liger-Kernel PR #1363, sections
+ *      "Summary", "Why it is faster and uses less memory" and "Native scope").
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers to contiguous row-major arrays on the
+ *     current CUDA device; the caller owns every buffer.  Nothing is freed or
+ *     retained by the library except the per-(device, stream) scratch of pl_loss.
+ *   - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default stream) and
+ *     the calls return without synchronising the host.
+ *   - Host-detectable problems (NULL required pointer, negative size, unsupported
+ *     dtype, workspace too small, a device that is not compute capability 10.0)
+ *     return an error code before any launch and before any output is written.
+ *   - Problems only the device can see (a bounded wait that ran out, a target id
+ *     outside [0, V)) set a sticky flag in the workspace; outputs are then
+ *     undefined.  Read and clear it with pl_device_status().
+ *   - No exception crosses this boundary.
+ */
+#ifndef PL_H_
+#define PL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so this header needs no CUDA header. */
+typedef struct CUstream_st* pl_stream_t;
+
+typedef enum {
+  PL_OK = 0,
+  PL_ERR_ARG = 1,            /* NULL required pointer, negative size, bad eps/beta/mode bits */
+  PL_ERR_DTYPE = 2,          /* dtype field not supported by this entry point */
+  PL_ERR_ALIGN = 3,          /* a pitch the tensor-memory-access unit cannot address */
+  PL_ERR_WORKSPACE = 4,      /* workspace NULL or smaller than the *_workspace_bytes() size */
+  PL_ERR_ARCH = 5,           /* current device is not compute capability 10.0 (B200) */
+  PL_ERR_CUDA = 6,           /* a CUDA runtime call or kernel launch failed */
+  PL_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait ran out (reported by pl_device_status) */
+  PL_ERR_BAD_TARGET = 8      /* a target id outside [0, V) (reported by pl_device_status) */
+} pl_status;
+
+/* ---- mode bit-field ----------------------------------------------------------
+ * bits 0-1  reduction: PL_BNPO (global token mean) or PL_GRPO (per-sequence mean,
+ *           then mean over the bs sequences, fully masked sequences counted).
+ * bits 4-7  dtype of the log-probs (pl_loss) or of X/W/Xref/Wref/bias/dX/dW/dbias
+ *           (pl_fused_linear_grpo): PL_F32, PL_F16 or PL_BF16.
+ * bit 8     PL_ADV_LP_DTYPE: adv is in that dtype instead of fp32.
+ * bit 9     PL_CLIP_TWO_SIDED: use -min(A*ratio, A*clipped) instead of the literal
+ *           -A*min(ratio, clipped).  (The literal form makes eps_lo inert; the
+ *           two-sided form is the standard PPO objective.)
+ * bits 16-23 pl_fused_linear_grpo only: rows per chunk / 128; 0 selects 1024.
+ */
+#define PL_BNPO 0u
+#define PL_GRPO 1u
+#define PL_REDUCTION_MASK 0x3u
+#define PL_F32 (0u << 4)
+#define PL_F16 (1u << 4)
+#define PL_BF16 (2u << 4)
+#define PL_DTYPE_MASK (0xFu << 4)
+#define PL_ADV_LP_DTYPE (1u << 8)
+#define PL_CLIP_TWO_SIDED (1u << 9)
+#define PL_CHUNK_SHIFT 16
+#define PL_CHUNK_ROWS(n) ((uint32_t)(((n) / 128) & 0xFF) << PL_CHUNK_SHIFT)
+
+/* ---- loss-only kernel ---------------------------------------------------------
+ * pl_loss: fused forward + backward (grad_out != NULL) or forward-only
+ * (grad_out == NULL) of the BNPO/GRPO loss above, as ONE kernel launch: the
+ * valid-token counts (global for BNPO, per sequence for GRPO) are taken on the
+ * device in a first phase, a bounded grid barrier orders them before the
+ * scaling phase, and the last block to finish reduces the per-block partial sums
+ * in a fixed order (deterministic).  No host synchronisation.
+ *
+ *   policy_lp, old_lp, ref_lp : [bs, seq] in the mode's dtype.  ref_lp may be NULL
+ *                               only when beta == 0 (the KL branch is then compiled
+ *                               out and ref_lp is never read).
+ *   adv                       : [bs], fp32 (or the log-prob dtype with PL_ADV_LP_DTYPE).
+ *   mask                      : [bs, seq] bytes (bool or int8); nonzero = valid.
+ *   eps_lo, eps_hi, beta      : clip band [1-eps_lo, 1+eps_hi] (both >= 0), KL weight (>= 0).
+ *   loss_out                  : device fp32 scalar.
+ *   grad_out                  : [bs, seq] in the log-prob dtype = dLoss/dpolicy_lp, or NULL.
+ * bs*seq == 0 writes loss 0.  Pointers that are not 16-byte aligned take a scalar
+ * path; they never fail.
+ * Scratch: pl_loss keeps one small zero-initialised buffer per (device, stream),
+ * allocated on the first call on that pair (make that first call outside any
+ * stream capture).  Calls on one stream are ordered; calls on different streams
+ * use different scratch.
+ */
+pl_status pl_loss(const void* policy_lp, const void* old_lp, const void* ref_lp,
+                  const void* adv, const uint8_t* mask, int64_t bs, int64_t seq,
+                  float eps_lo, float eps_hi, float beta, uint32_t mode,
+                  float* loss_out, void* grad_out, pl_stream_t stream);
+
+/* pl_loss with caller-owned scratch and optional count outputs.
+ *   n_valid_out   : device int64 scalar, the global valid-token count, or NULL.
+ *   row_valid_out : device int64 [bs], the per-sequence counts, or NULL.
+ *   workspace     : device buffer of at least pl_loss_workspace_bytes(bs, seq) bytes,
+ *                   zero-filled by the caller ONCE after allocation; the kernel
+ *                   returns its counters to zero, so it stays reusable.  Calls that
+ *                   share a workspace must be ordered on one stream.
+ */
+pl_status pl_loss_ex(const void* policy_lp, const void* old_lp, const void* ref_lp,
+                     const void* adv, const uint8_t* mask, int64_t bs, int64_t seq,
+                     float eps_lo, float eps_hi, float beta, uint32_t mode,
+                     float* loss_out, void* grad_out, int64_t* n_valid_out,
+                     int64_t* row_valid_out, void* workspace, size_t ws_bytes,
+                     pl_stream_t stream);
+
+size_t pl_loss_workspace_bytes(int64_t bs, int64_t seq);
+
+/* ---- fused linear path ----------------------------------------------------------
+ * pl_fused_linear_grpo: for the N = bs*T rows (sequence-major),
+ *   z      = X W^T (+ bias),  logp = z[target] - logsumexp(z)        (policy)
+ *   z_ref  = Xref Wref^T,     ref_logp likewise                        (reference, no bias)
+ *   loss   = the BNPO/GRPO loss of pl_loss on (logp, old_lp, ref_logp)
+ *   g      = dLoss/dlogp,  dz = g * (onehot(target) - softmax(z))
+ *   dX = dz W,  dW = dz^T X,  dbias = sum over rows of dz.
+ * Rows are processed in chunks (1024 by default, see the mode bits).  Per chunk a
+ * persistent tcgen05 GEMM computes the reference and policy logits tile by tile;
+ * its epilogue keeps a per-(row, 256-column tile) running max / sum of exponentials
+ * and the target logit, and stores the policy logits into a bounded workspace of
+ * chunk x V elements (full-batch logits are never materialised).  The logits are
+ * then turned into dz in place and a second persistent GEMM computes dX and dW;
+ * dW and dbias are accumulated in fp32 across chunks (the first chunk stores, later
+ * chunks add, the last converts to the model dtype).
+ *
+ *   X [N,H], W [V,H], bias [V] or NULL : model dtype (PL_F16 or PL_BF16).
+ *   targets [N] int64                  : sampled token ids; a row whose id is outside
+ *                                        [0, V) is treated as masked and raises
+ *                                        PL_ERR_BAD_TARGET in pl_device_status.
+ *   Xref [N,H], Wref [V,H]             : reference model inputs, model dtype; NULL
+ *                                        allowed only when beta == 0 (the reference
+ *                                        GEMM is then skipped).
+ *   old_lp [N] fp32, adv [bs], mask [bs,T] bytes : as for pl_loss.
+ *   H must be a multiple of 8 (16-byte row pitch); any V >= 1.
+ *   loss                               : device fp32 scalar (required).
+ *   dX [N,H], dW [V,H], dbias [V]      : model dtype, each NULL if not needed (its
+ *                                        GEMM or reduction is skipped).
+ *   logp_out, ref_logp_out [N] fp32    : optional per-token log-probs (the latter is
+ *                                        written only when beta != 0).
+ *   n_valid_out                        : optional device int64 scalar.
+ *   workspace                          : at least pl_fused_linear_grpo_workspace_bytes()
+ *                                        bytes, zero-filled once after allocation.
+ */
+pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias,
+                               const int64_t* targets, const void* Xref, const void* Wref,
+                               const float* old_lp, const void* adv, const uint8_t* mask,
+                               int64_t bs, int64_t T, int64_t H, int64_t V,
+                               float eps_lo, float eps_hi, float beta, uint32_t mode,
+                               float* loss, void* dX, void* dW, void* dbias,
+                               float* logp_out, float* ref_logp_out, int64_t* n_valid_out,
+                               void* workspace, size_t ws_bytes, pl_stream_t stream);
+
+size_t pl_fused_linear_grpo_workspace_bytes(int64_t bs, int64_t T, int64_t H, int64_t V,
+                                            uint32_t mode, int need_dW, int need_dbias);
+
+/* ---- status ---------------------------------------------------------------------
+ * pl_device_status: synchronises `stream`, reads the sticky device error flag of
+ * `workspace` (NULL = pl_loss's own scratch for the current device and `stream`),
+ * clears it and returns PL_OK, PL_ERR_DEVICE_TIMEOUT or PL_ERR_BAD_TARGET.
+ */
+pl_status pl_device_status(const void* workspace, pl_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* pl_status_string(pl_status status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int pl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PL_H_ */

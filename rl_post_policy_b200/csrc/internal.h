@@ -1,0 +1,71 @@
+// Internal declarations shared by the host-side sources of libpl.so.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/pl.h"
+
+namespace pl {
+
+// Element type of log-probs / model tensors (the mode's dtype field).
+enum class DType : int { F32 = 0, F16 = 1, BF16 = 2 };
+
+inline size_t dtype_size(DType d) { return d == DType::F32 ? 4 : 2; }
+
+// Sticky device error bits, stored in the first word of every workspace.
+constexpr unsigned kDevErrTimeout = 1u;
+constexpr unsigned kDevErrTarget = 2u;
+
+// Every workspace starts with this 256-byte header:
+//   +0  u32 error flag (sticky, cleared by pl_device_status)
+//   +4  u32 grid-barrier arrival counter
+//   +8  u32 finished-block counter
+//   +16 u64 global valid-token count
+constexpr size_t kWsHeader = 256;
+
+// Bound on every device-side wait, in nanoseconds of %globaltimer.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// Loss-kernel workspace: header, u64 row counts [bs], f64 block partials.
+constexpr int kLossMaxBlocks = 4096;
+inline size_t loss_partial_offset(int64_t bs) {
+  size_t off = kWsHeader + (size_t)(bs > 0 ? bs : 0) * 8;
+  return (off + 255) & ~(size_t)255;
+}
+inline size_t loss_ws_bytes(int64_t bs) { return loss_partial_offset(bs) + (size_t)kLossMaxBlocks * 8; }
+
+struct LossArgs {
+  const void* lp;
+  const void* old;
+  const void* ref;
+  const void* adv;
+  const uint8_t* mask;
+  void* grad;
+  float* loss_out;
+  int64_t* n_valid_out;
+  int64_t* row_valid_out;
+  unsigned char* ws;
+  int64_t bs, seq, n;
+  int64_t chunk;        // tokens per block, multiple of 64
+  float lo, hi, beta;
+  int grpo;
+  int adv_lp_dtype;
+  int need_rows;
+  int64_t partial_offset;  // byte offset of the f64 block partials inside ws
+};
+
+// Launches the single-pass loss kernel; returns a CUDA error code.
+cudaError_t launch_loss(const LossArgs& a, DType dt, bool has_kl, bool has_grad, bool two_sided,
+                        bool vec, cudaStream_t stream);
+
+// Device properties cached per device.
+struct DevInfo {
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+  size_t smem_optin = 0;
+};
+cudaError_t dev_info(DevInfo* out);
+
+}  // namespace pl

@@ -1,0 +1,343 @@
+// Single-launch BNPO/GRPO loss kernel (forward + optional backward).
+//
+// Per token ("Geometric-AI Kernels" model card, "BNPO Loss"):
+//   ratio = exp(lp - old), clipped = clip(ratio, lo, hi), per_token = -A*min(ratio, clipped),
+//   kl = exp(ref - lp) - (ref - lp) - 1   (here expm1(e) - e, e = ref - lp)
+// Reductions: BNPO divides by the global valid-token count ("BNPO Loss"), GRPO by
+// each sequence's count and then by bs ("GRPO Loss").  The counts are taken on the
+// device with integer atomics (no host mask.sum()), as the card's "BNPO Loss"
+// section describes; the KL branch is compiled out when beta == 0.
+//
+// One cooperative launch, three phases:
+//   A. every block counts the mask over its contiguous token range (global and
+//      per-sequence counts, exact u64 atomics);
+//   -- bounded grid barrier (gives up after kWaitLimitNs and raises the error flag);
+//   B. 16-byte vector loads of the log-probs, per-token math in fp32, the scaled
+//      gradient written in the log-prob dtype, and a per-block partial loss;
+//   C. the last block to finish sums the partials in block order (fp64, so the
+//      result is deterministic), writes the loss and counts, and returns the
+//      workspace counters to zero.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "internal.h"
+#include "policy_math.cuh"
+
+namespace pl {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kSmemRows = 64;
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __half from_f<__half>(float x) { return __float2half_rn(x); }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// 16-byte vector <-> VW floats.
+template <typename T, int VW>
+__device__ __forceinline__ void load16(const T* p, float (&v)[VW]) {
+  static_assert(VW * sizeof(T) == 16, "16-byte vectors");
+  uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+  for (int j = 0; j < VW; ++j) v[j] = to_f(e[j]);
+}
+
+template <typename T, int VW>
+__device__ __forceinline__ void store16(T* p, const float (&v)[VW]) {
+  uint4 u;
+  T* e = reinterpret_cast<T*>(&u);
+#pragma unroll
+  for (int j = 0; j < VW; ++j) e[j] = from_f<T>(v[j]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+template <typename T>
+__device__ __forceinline__ float load_adv(const LossArgs& a, int64_t r) {
+  if (a.adv_lp_dtype) return to_f(reinterpret_cast<const T*>(a.adv)[r]);
+  return reinterpret_cast<const float*>(a.adv)[r];
+}
+
+template <typename T, bool HAS_KL, bool HAS_GRAD, bool TWO_SIDED, bool VEC>
+__global__ void __launch_bounds__(kThreads) loss_kernel(LossArgs a) {
+  constexpr int VW = VEC ? (int)(16 / sizeof(T)) : 1;
+  __shared__ unsigned long long s_rows[kSmemRows];
+  __shared__ double s_red[kThreads / 32];
+  __shared__ unsigned long long s_cnt[kThreads / 32];
+  __shared__ int s_flag;
+
+  unsigned* err = reinterpret_cast<unsigned*>(a.ws);
+  unsigned* arrive = reinterpret_cast<unsigned*>(a.ws + 4);
+  unsigned* done = reinterpret_cast<unsigned*>(a.ws + 8);
+  unsigned long long* nvalid = reinterpret_cast<unsigned long long*>(a.ws + 16);
+  unsigned long long* rowcnt = reinterpret_cast<unsigned long long*>(a.ws + kWsHeader);
+  double* partial = reinterpret_cast<double*>(a.ws + a.partial_offset);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t n = a.n, seq = a.seq;
+  const int64_t t0 = min(n, (int64_t)blockIdx.x * a.chunk);
+  const int64_t t1 = min(n, t0 + a.chunk);
+  const bool any = t1 > t0;
+  const int64_t r0 = any ? t0 / seq : 0;
+  const int64_t r1 = any ? (t1 - 1) / seq : -1;
+  const bool rows_in_smem = a.need_rows && any && (r1 - r0 + 1) <= kSmemRows;
+
+  if (tid < kSmemRows) s_rows[tid] = 0;
+  if (tid == 0) s_flag = 0;
+  __syncthreads();
+
+  // ---------------- phase A: valid-token counts ----------------
+  unsigned long long my_total = 0;
+  const uint8_t* mk = a.mask;
+  for (int64_t t = t0 + (int64_t)tid * 16; t < t1; t += (int64_t)kThreads * 16) {
+    uint8_t b[16];
+    const int cnt = (int)min((int64_t)16, t1 - t);
+    if (VEC && cnt == 16) {
+      *reinterpret_cast<uint4*>(b) = __ldg(reinterpret_cast<const uint4*>(mk + t));
+    } else {
+      for (int j = 0; j < 16; ++j) b[j] = j < cnt ? mk[t + j] : 0;
+    }
+    int64_t r = t / seq;
+    int64_t boundary = (r + 1) * seq;
+    unsigned c = 0;
+    for (int j = 0; j < cnt; ++j) {
+      if (t + j == boundary) {
+        if (a.need_rows && c) {
+          if (rows_in_smem) atomicAdd(&s_rows[r - r0], (unsigned long long)c);
+          else atomicAdd(&rowcnt[r], (unsigned long long)c);
+        }
+        my_total += c;
+        c = 0;
+        ++r;
+        boundary += seq;
+      }
+      c += b[j] != 0;
+    }
+    if (a.need_rows && c) {
+      if (rows_in_smem) atomicAdd(&s_rows[r - r0], (unsigned long long)c);
+      else atomicAdd(&rowcnt[r], (unsigned long long)c);
+    }
+    my_total += c;
+  }
+  // block total of valid tokens -> one global atomic
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) my_total += __shfl_xor_sync(0xffffffffu, my_total, o);
+  if (lane == 0) s_cnt[warp] = my_total;
+  __syncthreads();
+  if (tid == 0) {
+    unsigned long long s = 0;
+    for (int w = 0; w < kThreads / 32; ++w) s += s_cnt[w];
+    if (s) atomicAdd(nvalid, s);
+  }
+  if (rows_in_smem && tid < (int)(r1 - r0 + 1) && s_rows[tid]) atomicAdd(&rowcnt[r0 + tid], s_rows[tid]);
+
+  // ---------------- bounded grid barrier ----------------
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    atomicAdd(arrive, 1u);
+    const unsigned long long start = globaltimer_ns();
+    while (ld_acquire_u32(arrive) < gridDim.x) {
+      if (globaltimer_ns() - start > kWaitLimitNs) {
+        atomicOr(err, kDevErrTimeout);
+        s_flag = 1;
+        break;
+      }
+      __nanosleep(100);
+    }
+    __threadfence();
+  }
+  __syncthreads();
+
+  // ---------------- phase B: per-token loss and gradient ----------------
+  float acc = 0.0f;
+  if (!s_flag && any) {
+    const unsigned long long total = __ldcg(nvalid);
+    const float inv_total = (float)(1.0 / (double)(total > 0 ? total : 1));
+    const T* lp = reinterpret_cast<const T*>(a.lp);
+    const T* od = reinterpret_cast<const T*>(a.old);
+    const T* rf = reinterpret_cast<const T*>(a.ref);
+    T* gr = reinterpret_cast<T*>(a.grad);
+    const float lo = a.lo, hi = a.hi, beta = a.beta;
+    int64_t cur_row = -1;
+    float A = 0.0f, scale = 0.0f;
+    auto row_state = [&](int64_t r) {
+      if (r != cur_row) {
+        cur_row = r;
+        A = load_adv<T>(a, r);
+        if (a.grpo) {
+          const unsigned long long c = __ldcg(&rowcnt[r]);
+          scale = (float)(1.0 / ((double)a.bs * (double)(c > 0 ? c : 1)));
+        } else {
+          scale = inv_total;
+        }
+      }
+    };
+    auto scalar_span = [&](int64_t t, int64_t te) {
+      // unaligned operands, or the ragged tail of the last block
+      for (int64_t u = t; u < te; ++u) {
+        row_state(u / seq);
+        float term, dterm;
+        token_math<HAS_KL, TWO_SIDED>(to_f(lp[u]), to_f(od[u]), HAS_KL ? to_f(rf[u]) : 0.0f, A, lo,
+                                      hi, beta, term, dterm);
+        const bool valid = a.mask[u] != 0;
+        acc += valid ? term * scale : 0.0f;
+        if (HAS_GRAD) gr[u] = from_f<T>(valid ? dterm * scale : 0.0f);
+      }
+    };
+    for (int64_t t = t0 + (int64_t)tid * VW; t < t1; t += (int64_t)kThreads * VW) {
+      if constexpr (VEC) {
+        if (t + VW > t1) {
+          scalar_span(t, t1);
+          continue;
+        }
+        float vl[VW], vo[VW], vr[VW], vg[VW];
+        load16<T, VW>(lp + t, vl);
+        load16<T, VW>(od + t, vo);
+        if (HAS_KL) load16<T, VW>(rf + t, vr);
+        uint8_t m[VW];
+        if constexpr (VW == 8) {
+          *reinterpret_cast<uint2*>(m) = __ldg(reinterpret_cast<const uint2*>(a.mask + t));
+        } else {
+          *reinterpret_cast<unsigned*>(m) = __ldg(reinterpret_cast<const unsigned*>(a.mask + t));
+        }
+        int64_t r = t / seq;
+        int64_t boundary = (r + 1) * seq;
+#pragma unroll
+        for (int j = 0; j < VW; ++j) {
+          if (t + j == boundary) { ++r; boundary += seq; }
+          row_state(r);
+          float term, dterm;
+          token_math<HAS_KL, TWO_SIDED>(vl[j], vo[j], HAS_KL ? vr[j] : 0.0f, A, lo, hi, beta, term,
+                                        dterm);
+          const bool valid = m[j] != 0;
+          acc += valid ? term * scale : 0.0f;
+          vg[j] = valid ? dterm * scale : 0.0f;
+        }
+        if (HAS_GRAD) store16<T, VW>(gr + t, vg);
+      } else {
+        scalar_span(t, t + 1);
+      }
+    }
+  }
+
+  // block partial (warp shuffle in fp32, then fp64 across warps)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) s_red[warp] = (double)acc;
+  __syncthreads();
+
+  // ---------------- phase C: last-block finalize ----------------
+  if (tid == 0) {
+    double s = 0.0;
+    for (int w = 0; w < kThreads / 32; ++w) s += s_red[w];
+    partial[blockIdx.x] = s;
+    __threadfence();
+    const unsigned prev = atomicAdd(done, 1u);
+    s_flag = (prev == gridDim.x - 1) ? 2 : 0;
+  }
+  __syncthreads();
+  if (s_flag == 2) {
+    __threadfence();
+    if (tid == 0) {
+      double s = 0.0;
+      for (unsigned b = 0; b < gridDim.x; ++b) s += __ldcg(&partial[b]);
+      *a.loss_out = (float)s;
+      if (a.n_valid_out) *a.n_valid_out = (int64_t)__ldcg(nvalid);
+      *nvalid = 0ull;
+      *arrive = 0u;
+      *done = 0u;
+    }
+    for (int64_t r = tid; r < a.bs; r += kThreads) {
+      if (a.row_valid_out) a.row_valid_out[r] = (int64_t)__ldcg(&rowcnt[r]);
+      rowcnt[r] = 0ull;
+    }
+  }
+}
+
+template <typename T, bool HAS_KL, bool HAS_GRAD, bool TWO_SIDED, bool VEC>
+cudaError_t launch_t(const LossArgs& a0, cudaStream_t stream) {
+  auto kern = loss_kernel<T, HAS_KL, HAS_GRAD, TWO_SIDED, VEC>;
+  static int per_sm = -1;
+  if (per_sm < 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0);
+    if (e != cudaSuccess) { per_sm = -1; return e; }
+    if (per_sm < 1) per_sm = 1;
+  }
+  DevInfo di;
+  cudaError_t e = dev_info(&di);
+  if (e != cudaSuccess) return e;
+  LossArgs a = a0;
+  // Enough blocks to cover the tokens with a few vector iterations per thread,
+  // never more than can be co-resident (the grid barrier needs all of them).
+  constexpr int64_t kMinTokensPerBlock = 4096;
+  int64_t want = (a.n + kMinTokensPerBlock - 1) / kMinTokensPerBlock;
+  int64_t cap = (int64_t)per_sm * di.sm_count;
+  if (cap > kLossMaxBlocks) cap = kLossMaxBlocks;
+  int64_t grid = want < 1 ? 1 : (want > cap ? cap : want);
+  int64_t chunk = (a.n + grid - 1) / grid;
+  chunk = (chunk + 63) / 64 * 64;
+  if (chunk < 64) chunk = 64;
+  grid = a.n > 0 ? (a.n + chunk - 1) / chunk : 1;
+  a.chunk = chunk;
+  void* args[] = {&a};
+  return cudaLaunchCooperativeKernel((const void*)kern, dim3((unsigned)grid), dim3(kThreads), args, 0,
+                                     stream);
+}
+
+template <typename T>
+cudaError_t dispatch_t(const LossArgs& a, bool kl, bool g, bool two, bool vec, cudaStream_t s) {
+#define PL_LOSS_CASE(KL, G, TW, VE) \
+  if (kl == KL && g == G && two == TW && vec == VE) return launch_t<T, KL, G, TW, VE>(a, s);
+  PL_LOSS_CASE(true, true, false, true)
+  PL_LOSS_CASE(true, true, false, false)
+  PL_LOSS_CASE(true, true, true, true)
+  PL_LOSS_CASE(true, true, true, false)
+  PL_LOSS_CASE(true, false, false, true)
+  PL_LOSS_CASE(true, false, false, false)
+  PL_LOSS_CASE(true, false, true, true)
+  PL_LOSS_CASE(true, false, true, false)
+  PL_LOSS_CASE(false, true, false, true)
+  PL_LOSS_CASE(false, true, false, false)
+  PL_LOSS_CASE(false, true, true, true)
+  PL_LOSS_CASE(false, true, true, false)
+  PL_LOSS_CASE(false, false, false, true)
+  PL_LOSS_CASE(false, false, false, false)
+  PL_LOSS_CASE(false, false, true, true)
+  PL_LOSS_CASE(false, false, true, false)
+#undef PL_LOSS_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_loss(const LossArgs& a, DType dt, bool has_kl, bool has_grad, bool two_sided,
+                        bool vec, cudaStream_t stream) {
+  switch (dt) {
+    case DType::F32: return dispatch_t<float>(a, has_kl, has_grad, two_sided, vec, stream);
+    case DType::F16: return dispatch_t<__half>(a, has_kl, has_grad, two_sided, vec, stream);
+    case DType::BF16: return dispatch_t<__nv_bfloat16>(a, has_kl, has_grad, two_sided, vec, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace pl
