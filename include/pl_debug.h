@@ -1,0 +1,47 @@
+/*
+ * pl_debug.h -- test hooks of libpl.so (not part of the loss path).
+ *
+ * pl_debug_gemm runs one plain GEMM through the same persistent tcgen05 kernel
+ * the fused path uses, so the tensor-core mainloop can be checked in isolation:
+ *
+ *   D[m, n] = sum_k A(m, k) * B(n, k)            (fp32, row-major [M, N])
+ *   A(m, k) = a_mn ? A[k*lda + m] : A[m*lda + k]   (K-major or MN-major)
+ *   B(n, k) = b_mn ? B[k*ldb + n] : B[n*ldb + k]
+ *
+ * A, B: device, 16-bit (mode PL_F16 or PL_BF16), 16-byte aligned, lda/ldb
+ * multiples of 8.  D: device fp32.  Enqueued on `stream`; a bounded wait that
+ * runs out is reported by pl_device_status(NULL, stream).
+ * Returns PL_ERR_ARG / PL_ERR_DTYPE / PL_ERR_ALIGN before any launch on bad input.
+ */
+#ifndef PL_DEBUG_H_
+#define PL_DEBUG_H_
+
+#include "pl.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+pl_status pl_debug_gemm(const void* A, int a_mn, int64_t lda, const void* B, int b_mn, int64_t ldb,
+                        float* D, int64_t M, int64_t N, int64_t K, uint32_t mode, pl_stream_t stream);
+
+/*
+ * Kernel timing for the benchmark.  While enabled, every kernel the library
+ * launches is bracketed by a pair of CUDA events recorded on the launching
+ * stream.  pl_debug_timing_read() waits for the recorded events, returns per
+ * kind the summed device milliseconds and launch counts, and clears them.
+ * Kinds: 0 = GEMM (tcgen05 kernel), 1 = loss-only kernel, 2 = other kernels of
+ * the fused path (counts, combine, dlogits, finalize).  Arrays have 3 entries.
+ * Not thread-safe; meant for one benchmarking thread.
+ */
+void pl_debug_timing(int enable);
+pl_status pl_debug_timing_read(double* ms, int64_t* launches);
+
+/* Number of kernels this library has launched in this process. */
+int64_t pl_debug_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PL_DEBUG_H_ */

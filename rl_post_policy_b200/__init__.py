@@ -56,10 +56,19 @@ _lib.pl_status_string.argtypes = [_I]
 _lib.pl_status_string.restype = ctypes.c_char_p
 _lib.pl_version.argtypes = []
 _lib.pl_version.restype = _I
+_lib.pl_debug_gemm.argtypes = [_P, _I, _I64, _P, _I, _I64, _P, _I64, _I64, _I64, _U32, _P]
+_lib.pl_debug_gemm.restype = _I
+_lib.pl_debug_timing.argtypes = [_I]
+_lib.pl_debug_timing.restype = None
+_lib.pl_debug_timing_read.argtypes = [_P, _P]
+_lib.pl_debug_timing_read.restype = _I
+_lib.pl_debug_launch_count.argtypes = []
+_lib.pl_debug_launch_count.restype = _I64
 
 EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
-            "pl_version")
+            "pl_version", "pl_debug_gemm", "pl_debug_timing", "pl_debug_timing_read",
+            "pl_debug_launch_count")
 
 
 class PLError(RuntimeError):
@@ -140,3 +149,25 @@ def pl_status_string(status: int) -> str:
 
 def pl_version() -> int:
     return int(_lib.pl_version())
+
+
+def pl_debug_gemm(A, a_mn, lda, B, b_mn, ldb, D, M, N, K, mode, stream=None) -> int:
+    """Test hook (include/pl_debug.h): plain GEMM through the tcgen05 kernel."""
+    return _lib.pl_debug_gemm(_ptr(A), int(a_mn), lda, _ptr(B), int(b_mn), ldb, _ptr(D), M, N, K,
+                              mode, _stream(stream))
+
+
+def pl_debug_timing(enable: bool) -> None:
+    _lib.pl_debug_timing(int(bool(enable)))
+
+
+def pl_debug_timing_read():
+    """((gemm_ms, loss_ms, other_ms), (gemm_launches, loss_launches, other_launches))."""
+    ms = (ctypes.c_double * 3)()
+    n = (ctypes.c_int64 * 3)()
+    check(_lib.pl_debug_timing_read(ms, n), "pl_debug_timing_read")
+    return tuple(ms), tuple(n)
+
+
+def pl_debug_launch_count() -> int:
+    return int(_lib.pl_debug_launch_count())

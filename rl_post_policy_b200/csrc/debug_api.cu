@@ -1,0 +1,96 @@
+// pl_debug_gemm: a plain GEMM through the persistent tcgen05 kernel (test hook).
+#include "../../include/pl_debug.h"
+#include "gemm.h"
+
+using namespace pl;
+
+extern "C" pl_status pl_debug_gemm(const void* A, int a_mn, int64_t lda, const void* B, int b_mn,
+                                   int64_t ldb, float* D, int64_t M, int64_t N, int64_t K, uint32_t mode,
+                                   pl_stream_t stream) {
+  if (!A || !B || !D || M < 1 || N < 1 || K < 1) return PL_ERR_ARG;
+  if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return PL_ERR_ARG;
+  const uint32_t dcode = (mode & PL_DTYPE_MASK) >> 4;
+  if (dcode != 1 && dcode != 2) return PL_ERR_DTYPE;
+  if (mode & ~PL_DTYPE_MASK) return PL_ERR_ARG;
+  if ((lda % 8) || (ldb % 8) || (((uintptr_t)A) & 15) || (((uintptr_t)B) & 15)) return PL_ERR_ALIGN;
+  if (lda < (a_mn ? M : K) || ldb < (b_mn ? N : K)) return PL_ERR_ARG;
+  pl_status st = check_arch();
+  if (st != PL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  if ((st = own_workspace(s, loss_ws_bytes(0), &scratch, true)) != PL_OK) return st;
+  const DType dt = (DType)dcode;
+  GemmParams p{};
+  p.err = static_cast<unsigned*>(scratch);
+  p.wait_ns = kWaitLimitNs;
+  bool ok = a_mn ? make_tmap_2d(&p.maps[0], A, dt, M, K, lda * 2, 64, kBK)
+                 : make_tmap_2d(&p.maps[0], A, dt, K, M, lda * 2, kBK, kBM);
+  ok = ok && (b_mn ? make_tmap_2d(&p.maps[1], B, dt, N, K, ldb * 2, 64, kBK)
+                   : make_tmap_2d(&p.maps[1], B, dt, K, N, ldb * 2, kBK, kBN));
+  if (!ok) return PL_ERR_CUDA;
+  GemmJob& j = p.jobs[0];
+  j.a_map = 0; j.b_map = 1; j.a_mn = a_mn ? 1 : 0; j.b_mn = b_mn ? 1 : 0;
+  j.M = (int)M; j.N = (int)N; j.K = (int)K; j.n_inner = 0; j.epi = kEpiStore;
+  j.out = D; j.out_f32 = 1; j.acc_in = nullptr; j.out_ld = N; j.scale = nullptr;
+  p.njobs = 1;
+  gemm_finalize_jobs(&p);
+  return launch_gemm(p, dt, s) == cudaSuccess ? PL_OK : PL_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- launch bookkeeping
+#include <atomic>
+#include <vector>
+
+namespace {
+std::atomic<int64_t> g_launches{0};
+bool g_timing = false;
+struct EvPair {
+  cudaEvent_t a = nullptr, b = nullptr;
+  int kind = 0;
+};
+std::vector<EvPair> g_pool;
+size_t g_used = 0;
+}  // namespace
+
+namespace pl {
+void launch_begin(int kind, cudaStream_t stream) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (!g_timing) return;
+  if (g_used == g_pool.size()) {
+    EvPair e;
+    if (cudaEventCreate(&e.a) != cudaSuccess || cudaEventCreate(&e.b) != cudaSuccess) return;
+    g_pool.push_back(e);
+  }
+  g_pool[g_used].kind = kind;
+  cudaEventRecord(g_pool[g_used].a, stream);
+}
+void launch_end(int kind, cudaStream_t stream) {
+  (void)kind;
+  if (!g_timing || g_used >= g_pool.size()) return;
+  cudaEventRecord(g_pool[g_used].b, stream);
+  ++g_used;
+}
+}  // namespace pl
+
+extern "C" void pl_debug_timing(int enable) { g_timing = enable != 0; }
+
+extern "C" pl_status pl_debug_timing_read(double* ms, int64_t* launches) {
+  for (int k = 0; k < 3; ++k) {
+    if (ms) ms[k] = 0.0;
+    if (launches) launches[k] = 0;
+  }
+  for (size_t i = 0; i < g_used; ++i) {
+    float t = 0.0f;
+    if (cudaEventSynchronize(g_pool[i].b) != cudaSuccess) return PL_ERR_CUDA;
+    if (cudaEventElapsedTime(&t, g_pool[i].a, g_pool[i].b) != cudaSuccess) return PL_ERR_CUDA;
+    const int k = g_pool[i].kind;
+    if (k >= 0 && k < 3) {
+      if (ms) ms[k] += t;
+      if (launches) launches[k] += 1;
+    }
+  }
+  g_used = 0;
+  return PL_OK;
+}
+
+extern "C" int64_t pl_debug_launch_count(void) { return g_launches.load(); }

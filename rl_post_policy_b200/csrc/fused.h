@@ -1,0 +1,74 @@
+// Workspace layout and kernel arguments of the fused linear path.
+#pragma once
+
+#include <cstdint>
+
+#include "internal.h"
+
+namespace pl {
+
+// Byte offsets of the regions of a fused-path workspace (after the common
+// 256-byte header).  Every region starts on a 1024-byte boundary.
+struct FusedOffsets {
+  int64_t row_cnt;    // u64 [bs]           valid tokens per sequence
+  int64_t loss_part;  // f64 [nchunks, part_stride]  per-block loss partials
+  int64_t gmax;       // u32 [nchunks]       max |g| of the chunk (float bits)
+  int64_t inv_scale;  // f32 [nchunks]       2^-e undoing the dlogits scale
+  int64_t lse;        // f32 [C]             policy logsumexp of the chunk's rows
+  int64_t g;          // f32 [C]             dLoss/dlogp of the chunk's rows
+  int64_t zt;         // f32 [C]             policy target logit
+  int64_t zt_ref;     // f32 [C]             reference target logit
+  int64_t part;       // float2 [C, ntv]     policy (max, sum exp) per vocab tile
+  int64_t part_ref;   // float2 [C, ntv]     reference ditto
+  int64_t logits;     // T [C, ld]           logits, then dlogits (if a gradient is wanted)
+  int64_t dw_acc;     // f32 [V, H]          dW accumulator (multi-chunk only)
+  int64_t db_acc;     // f32 [V]             dbias accumulator (multi-chunk only)
+  int64_t total;
+};
+
+// How a chunk's weight/bias gradient contribution is written.
+enum AccMode : int {
+  kAccNone = 0,
+  kAccStoreModel = 1,  // only chunk: store in the model dtype
+  kAccStoreF32 = 2,    // first of several: store fp32 (the accumulator is born here)
+  kAccAddF32 = 3,      // middle: fp32 read-modify-write
+  kAccAddConvert = 4,  // last: fp32 accumulator + this chunk -> model dtype
+};
+
+struct CombineArgs {
+  unsigned char* ws;
+  FusedOffsets off;
+  const int64_t* targets;
+  const float* old_lp;
+  const void* adv;
+  const uint8_t* mask;
+  float* logp_out;
+  float* ref_logp_out;
+  int64_t row0, rows, bs, T, V;
+  int ntv;            // vocabulary tiles (partials per row)
+  int chunk, part_stride;
+  float lo, hi, beta;
+  int grpo, adv_lp_dtype, bf16;
+};
+
+struct DlogitsArgs {
+  unsigned char* ws;
+  FusedOffsets off;
+  const int64_t* targets;
+  void* logits;
+  int64_t ld;
+  int64_t row0, rows, V;
+  int chunk;
+  int dbias_mode;
+  float* dbias_acc;
+  void* dbias;
+};
+
+cudaError_t launch_count(const uint8_t* mask, int64_t bs, int64_t T, unsigned char* ws, int nchunks,
+                         const FusedOffsets& off, cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs& a, bool has_kl, bool two_sided, cudaStream_t s);
+cudaError_t launch_dlogits(const DlogitsArgs& a, DType dt, cudaStream_t s);
+cudaError_t launch_finalize(const unsigned char* ws, const FusedOffsets& off, int nchunks, int part_stride,
+                            int nblocks_last, float* loss, int64_t* n_valid_out, cudaStream_t s);
+
+}  // namespace pl

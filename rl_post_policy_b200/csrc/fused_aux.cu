@@ -1,0 +1,306 @@
+// Memory-bound kernels of the fused linear path (everything except the GEMMs).
+//
+//   count_kernel    -- exact per-sequence and global valid-token counts (mask != 0),
+//                      needed before any gradient can be scaled ("Geometric-AI
+//                      Kernels" model card: the denominators are computed on the GPU).
+//   combine_kernel  -- per row: logsumexp from the per-tile (max, sum exp) partials
+//                      of the GEMM epilogue, logp = z[target] - lse for the policy
+//                      and the reference model, then the clipped-ratio loss with
+//                      the KL term, g = dLoss/dlogp and the chunk's loss partials.
+//   dlogits_kernel  -- in place over the chunk's logits workspace:
+//                      dz = g * (onehot(target) - exp(z - lse)) * 2^e, stored in the
+//                      model dtype, and the column sums of dz (the bias gradient),
+//                      stored / accumulated in fp32 / converted like dW.
+//   finalize_kernel -- fixed-order sum of every chunk's loss partials.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "fused.h"
+#include "policy_math.cuh"
+
+namespace pl {
+namespace {
+
+__device__ __forceinline__ float cvt(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float cvt(__half x) { return __half2float(x); }
+template <typename T> __device__ __forceinline__ T to_t(float x);
+template <> __device__ __forceinline__ __nv_bfloat16 to_t<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+template <> __device__ __forceinline__ __half to_t<__half>(float x) { return __float2half_rn(x); }
+
+// ---------------------------------------------------------------- counts
+__global__ void count_kernel(const uint8_t* __restrict__ mask, int64_t bs, int64_t T,
+                             unsigned char* ws, int nchunks, const FusedOffsets off) {
+  unsigned* done = reinterpret_cast<unsigned*>(ws + 8);
+  unsigned long long* nvalid = reinterpret_cast<unsigned long long*>(ws + 16);
+  unsigned long long* rowcnt = reinterpret_cast<unsigned long long*>(ws + off.row_cnt);
+  unsigned* gmax = reinterpret_cast<unsigned*>(ws + off.gmax);
+  __shared__ unsigned long long s_cnt[8];
+  __shared__ int s_last;
+  const int64_t b = blockIdx.x;
+  if (b == 0)
+    for (int c = threadIdx.x; c < nchunks; c += blockDim.x) gmax[c] = 0u;
+  unsigned long long c = 0;
+  const uint8_t* m = mask + b * T;
+  for (int64_t t = threadIdx.x; t < T; t += blockDim.x) c += m[t] != 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) s_cnt[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long s = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += s_cnt[w];
+    rowcnt[b] = s;
+    __threadfence();
+    s_last = atomicAdd(done, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (s_last && threadIdx.x == 0) {
+    __threadfence();
+    unsigned long long s = 0;
+    for (int64_t r = 0; r < bs; ++r) s += __ldcg(&rowcnt[r]);
+    *nvalid = s;
+    *done = 0u;
+  }
+}
+
+// ---------------------------------------------------------------- combine
+template <bool HAS_KL, bool TWO_SIDED>
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  __shared__ double s_part[8];
+  __shared__ float s_gmax[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t i = (int64_t)blockIdx.x * 8 + warp;  // row within the chunk
+  float contrib = 0.0f, gabs = 0.0f;
+  if (i < a.rows) {
+    const int64_t g = a.row0 + i;
+    const unsigned char* ws = a.ws;
+    const float2* part = reinterpret_cast<const float2*>(ws + a.off.part) + i * a.ntv;
+    const float* zt = reinterpret_cast<const float*>(ws + a.off.zt);
+    // logsumexp over the vocabulary tiles: lse = M + log(sum_j s_j exp(m_j - M))
+    float M = -INFINITY;
+    for (int j = lane; j < a.ntv; j += 32) M = fmaxf(M, part[j].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float S = 0.0f;
+    for (int j = lane; j < a.ntv; j += 32) S += part[j].y * expf(part[j].x - M);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+    const float lse = M + logf(S);
+    float ref_lp = 0.0f;
+    if (HAS_KL) {
+      const float2* pr = reinterpret_cast<const float2*>(ws + a.off.part_ref) + i * a.ntv;
+      float Mr = -INFINITY;
+      for (int j = lane; j < a.ntv; j += 32) Mr = fmaxf(Mr, pr[j].x);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
+      float Sr = 0.0f;
+      for (int j = lane; j < a.ntv; j += 32) Sr += pr[j].y * expf(pr[j].x - Mr);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) Sr += __shfl_xor_sync(0xffffffffu, Sr, o);
+      const float* ztr = reinterpret_cast<const float*>(ws + a.off.zt_ref);
+      ref_lp = ztr[i] - (Mr + logf(Sr));
+    }
+    if (lane == 0) {
+      const int64_t tgt = a.targets[g];
+      const bool tvalid = tgt >= 0 && tgt < a.V;
+      if (!tvalid) atomicOr(reinterpret_cast<unsigned*>(a.ws), kDevErrTarget);
+      const float logp = tvalid ? zt[i] - lse : __int_as_float(0x7fc00000);
+      const int64_t b = g / a.T;
+      const bool valid = tvalid && a.mask[g] != 0;
+      const float A = a.adv_lp_dtype ? (a.bf16 ? cvt(reinterpret_cast<const __nv_bfloat16*>(a.adv)[b])
+                                               : cvt(reinterpret_cast<const __half*>(a.adv)[b]))
+                                     : reinterpret_cast<const float*>(a.adv)[b];
+      float scale;
+      if (a.grpo) {
+        const unsigned long long c = reinterpret_cast<const unsigned long long*>(ws + a.off.row_cnt)[b];
+        scale = (float)(1.0 / ((double)a.bs * (double)(c > 0 ? c : 1)));
+      } else {
+        const unsigned long long c = *reinterpret_cast<const unsigned long long*>(ws + 16);
+        scale = (float)(1.0 / (double)(c > 0 ? c : 1));
+      }
+      float term = 0.0f, dterm = 0.0f;
+      if (valid)
+        token_math<HAS_KL, TWO_SIDED>(logp, a.old_lp[g], ref_lp, A, a.lo, a.hi, a.beta, term, dterm);
+      const float gv = valid ? dterm * scale : 0.0f;
+      contrib = valid ? term * scale : 0.0f;
+      gabs = fabsf(gv);
+      reinterpret_cast<float*>(a.ws + a.off.g)[i] = gv;
+      reinterpret_cast<float*>(a.ws + a.off.lse)[i] = lse;
+      if (a.logp_out) a.logp_out[g] = logp;
+      if (HAS_KL && a.ref_logp_out) a.ref_logp_out[g] = tvalid ? ref_lp : __int_as_float(0x7fc00000);
+    }
+  }
+  if (lane == 0) {
+    s_part[warp] = (double)contrib;
+    s_gmax[warp] = gabs;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    float gm = 0.0f;
+    for (int w = 0; w < 8; ++w) {
+      s += s_part[w];
+      gm = fmaxf(gm, s_gmax[w]);
+    }
+    reinterpret_cast<double*>(a.ws + a.off.loss_part)[(int64_t)a.chunk * a.part_stride + blockIdx.x] = s;
+    if (gm > 0.0f) atomicMax(reinterpret_cast<unsigned*>(a.ws + a.off.gmax) + a.chunk, __float_as_uint(gm));
+  }
+}
+
+// ---------------------------------------------------------------- dlogits
+// Block = 256 threads = 8 warps over a 256-column strip of the chunk's logits;
+// lane l owns columns [8l, 8l+8) of the strip, warp w rows w, w+8, ...
+template <typename T>
+__global__ void __launch_bounds__(256) dlogits_kernel(DlogitsArgs a) {
+  extern __shared__ float s_dyn[];
+  float* s_lse = s_dyn;                                    // [rows]
+  float* s_g = s_lse + a.rows;                             // [rows]
+  int* s_t = reinterpret_cast<int*>(s_g + a.rows);         // [rows]
+  __shared__ float s_col[8][256];
+  const unsigned char* ws = a.ws;
+  for (int64_t i = threadIdx.x; i < a.rows; i += 256) {
+    s_lse[i] = reinterpret_cast<const float*>(ws + a.off.lse)[i];
+    s_g[i] = reinterpret_cast<const float*>(ws + a.off.g)[i];
+    const int64_t tg = a.targets[a.row0 + i];
+    s_t[i] = (tg >= 0 && tg < a.V) ? (int)tg : -1;
+  }
+  // power-of-two scale 2^e keeping max|dz| * 2^e <= 2^14 (fp16 range), exact to undo
+  const float gm = __uint_as_float(reinterpret_cast<const unsigned*>(ws + a.off.gmax)[a.chunk]);
+  int e = 0;
+  if (gm > 0.0f) {
+    e = 14 - (int)ceilf(log2f(gm));
+    e = max(-100, min(100, e));
+  }
+  const float sc = ldexpf(1.0f, e);
+  if (blockIdx.x == 0 && threadIdx.x == 0)
+    reinterpret_cast<float*>(a.ws + a.off.inv_scale)[a.chunk] = ldexpf(1.0f, -e);
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t col = (int64_t)blockIdx.x * 256 + lane * 8;
+  const bool full8 = col + 8 <= a.V;
+  float csum[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) csum[q] = 0.0f;
+  T* L = reinterpret_cast<T*>(a.logits);
+  constexpr float kLog2e = 1.4426950408889634f;
+  if (col < a.V) {
+#pragma unroll 4
+    for (int64_t i = warp; i < a.rows; i += 8) {
+      T* p = L + i * a.ld + col;
+      const float gi = s_g[i];
+      const float lsei = s_lse[i] * kLog2e;
+      const int ti = s_t[i];
+      float z[8];
+      if (full8) {
+        uint4 u = *reinterpret_cast<const uint4*>(p);
+        const T* e8 = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) z[q] = cvt(e8[q]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) z[q] = (col + q < a.V) ? cvt(p[q]) : 0.0f;
+      }
+      float d[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float pr = exp2f(fmaf(z[q], kLog2e, -lsei));
+        const float oh = (col + q == ti) ? 1.0f : 0.0f;
+        d[q] = gi * (oh - pr);
+        csum[q] += d[q];
+      }
+      if (full8) {
+        uint4 u;
+        T* e8 = reinterpret_cast<T*>(&u);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) e8[q] = to_t<T>(d[q] * sc);
+        *reinterpret_cast<uint4*>(p) = u;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (col + q < a.V) p[q] = to_t<T>(d[q] * sc);
+      }
+    }
+  }
+  if (a.dbias_mode == kAccNone) return;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) s_col[warp][lane * 8 + q] = csum[q];
+  __syncthreads();
+  const int64_t v = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (v < a.V) {
+    float s = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += s_col[w][threadIdx.x];
+    float* acc = a.dbias_acc;
+    T* out = reinterpret_cast<T*>(a.dbias);
+    switch (a.dbias_mode) {
+      case kAccStoreModel: out[v] = to_t<T>(s); break;
+      case kAccStoreF32: acc[v] = s; break;
+      case kAccAddF32: acc[v] += s; break;
+      case kAccAddConvert: out[v] = to_t<T>(acc[v] + s); break;
+      default: break;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- finalize
+__global__ void finalize_kernel(const unsigned char* ws, FusedOffsets off, int nchunks, int part_stride,
+                                int nblocks_last, float* loss, int64_t* n_valid_out) {
+  if (threadIdx.x != 0) return;
+  const double* part = reinterpret_cast<const double*>(ws + off.loss_part);
+  double s = 0.0;
+  for (int c = 0; c < nchunks; ++c) {
+    const int nb = c == nchunks - 1 ? nblocks_last : part_stride;
+    for (int b = 0; b < nb; ++b) s += part[(int64_t)c * part_stride + b];
+  }
+  *loss = (float)s;
+  if (n_valid_out) *n_valid_out = (int64_t) * reinterpret_cast<const unsigned long long*>(ws + 16);
+}
+
+}  // namespace
+
+cudaError_t launch_count(const uint8_t* mask, int64_t bs, int64_t T, unsigned char* ws, int nchunks,
+                         const FusedOffsets& off, cudaStream_t s) {
+  if (bs <= 0) return cudaSuccess;
+  { launch_begin(2, s); count_kernel<<<(unsigned)bs, 256, 0, s>>>(mask, bs, T, ws, nchunks, off); launch_end(2, s); }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CombineArgs& a, bool has_kl, bool two_sided, cudaStream_t s) {
+  const unsigned grid = (unsigned)((a.rows + 7) / 8);
+  if (grid == 0) return cudaSuccess;
+  if (has_kl) {
+    if (two_sided) { launch_begin(2, s); combine_kernel<true, true><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
+    else { launch_begin(2, s); combine_kernel<true, false><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
+  } else {
+    if (two_sided) { launch_begin(2, s); combine_kernel<false, true><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
+    else { launch_begin(2, s); combine_kernel<false, false><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dlogits(const DlogitsArgs& a, DType dt, cudaStream_t s) {
+  const unsigned grid = (unsigned)((a.V + 255) / 256);
+  const size_t smem = (size_t)a.rows * 12;
+  if (dt == DType::BF16) {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(dlogits_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+    { launch_begin(2, s); dlogits_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(a); launch_end(2, s); }
+  } else {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(dlogits_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    { launch_begin(2, s); dlogits_kernel<__half><<<grid, 256, smem, s>>>(a); launch_end(2, s); }
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const unsigned char* ws, const FusedOffsets& off, int nchunks, int part_stride,
+                            int nblocks_last, float* loss, int64_t* n_valid_out, cudaStream_t s) {
+  { launch_begin(2, s); finalize_kernel<<<1, 32, 0, s>>>(ws, off, nchunks, part_stride, nblocks_last, loss, n_valid_out); launch_end(2, s); }
+  return cudaGetLastError();
+}
+
+}  // namespace pl

@@ -1,0 +1,449 @@
+// Persistent tcgen05 GEMM for sm_100a with the epilogues of the fused path.
+//
+// Each CTA owns one SM (grid = min(tiles, SMs)) and walks the concatenated tile
+// list of up to two GEMM problems in a static round-robin.  Roles:
+//   warp 0    one elected lane issues TMA tile loads (128-byte swizzle) into a
+//             4-stage shared-memory ring (48 KB per stage);
+//   warp 1    allocates 512 tensor-memory columns (two 128x256 fp32
+//             accumulators) and one elected lane issues tcgen05.mma
+//             (M=128, N=256, K=16, bf16/fp16 -> fp32), committing each stage
+//             back to the producer and each finished tile to the epilogue;
+//   warps 2-5 the epilogue: one accumulator row per thread (tcgen05.ld
+//             32x32b), 32 columns at a time, overlapping the next tile's
+//             mainloop thanks to the second accumulator.
+// Operands may be K-major or MN-major (the backward GEMMs read the logits
+// workspace and the weights transposed without copying them).
+//
+// Epilogues ("Add SM100 CuTe DSL GRPO fast path", Liger-Kernel PR #1363,
+// "Summary": full logits are never materialised beyond a bounded workspace):
+//   kEpiLse   -- per (row, 256-column vocabulary tile): running max and sum of
+//                exp(z - max) over the valid columns, the target logit when the
+//                row's target falls in the tile, optional bias add and optional
+//                store of the logits in the model dtype;
+//   kEpiStore -- acc * scale (+ an fp32 accumulator) stored in the model dtype
+//                or in fp32 (dX; dW / dbias with fp32 accumulation across chunks).
+//
+// Every wait is bounded (GemmParams::wait_ns); when one runs out the CTA sets a
+// shared abort flag, every role drains out, tensor memory is released and the
+// sticky device error flag is raised.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "gemm.h"
+#include "sm100.cuh"
+
+namespace pl {
+namespace {
+
+using namespace sm100;
+
+constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB
+constexpr uint32_t kBBytes = kBN * kBK * 2;             // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 48 KB
+constexpr uint32_t kTmemCols = 512;
+constexpr size_t kGemmSmem = 1024 + kStages * kStageBytes + 256;
+
+__device__ __forceinline__ float cvt_in(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float cvt_in(__half x) { return __half2float(x); }
+
+template <typename T> __device__ __forceinline__ uint32_t pack2(float a, float b);
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+template <typename T> __device__ __forceinline__ T cvt_out(float x);
+template <> __device__ __forceinline__ __nv_bfloat16 cvt_out<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+template <> __device__ __forceinline__ __half cvt_out<__half>(float x) { return __float2half_rn(x); }
+
+template <typename T> struct AbFormat;
+template <> struct AbFormat<__half> { static constexpr uint32_t v = 0; };
+template <> struct AbFormat<__nv_bfloat16> { static constexpr uint32_t v = 1; };
+
+struct TileCoord {
+  int job, mb, nb;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const GemmParams& p, int tile) {
+  TileCoord c;
+  c.job = (p.njobs > 1 && tile >= p.jobs[1].tile_begin) ? 1 : 0;
+  const GemmJob& j = p.jobs[c.job];
+  const int local = tile - j.tile_begin;
+  if (j.n_inner) {
+    c.mb = local / j.tiles_n;
+    c.nb = local - c.mb * j.tiles_n;
+  } else {
+    c.nb = local / j.tiles_m;
+    c.mb = local - c.nb * j.tiles_m;
+  }
+  return c;
+}
+
+// Stores 32 consecutive values (or the first `nvalid`) of one row.
+template <typename T>
+__device__ __forceinline__ void store_row32(T* dst, const float (&v)[32], int nvalid) {
+  if (nvalid >= 32 && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 u;
+      u.x = pack2<T>(v[8 * q + 0], v[8 * q + 1]);
+      u.y = pack2<T>(v[8 * q + 2], v[8 * q + 3]);
+      u.z = pack2<T>(v[8 * q + 4], v[8 * q + 5]);
+      u.w = pack2<T>(v[8 * q + 6], v[8 * q + 7]);
+      d4[q] = u;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nvalid) dst[j] = cvt_out<T>(v[j]);
+  }
+}
+
+__device__ __forceinline__ void store_row32_f32(float* dst, const float (&v)[32], int nvalid) {
+  if (nvalid >= 32 && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nvalid) dst[j] = v[j];
+  }
+}
+
+__device__ __forceinline__ void add_row32_f32(const float* src, float (&v)[32], int nvalid) {
+  if (nvalid >= 32 && ((reinterpret_cast<uintptr_t>(src) & 15) == 0)) {
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 a = s4[q];
+      v[4 * q] += a.x;
+      v[4 * q + 1] += a.y;
+      v[4 * q + 2] += a.z;
+      v[4 * q + 3] += a.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nvalid) v[j] += src[j];
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void add_bias32(const T* bias, float (&v)[32], int nvalid) {
+  if (nvalid >= 32 && ((reinterpret_cast<uintptr_t>(bias) & 15) == 0)) {
+    const uint4* b4 = reinterpret_cast<const uint4*>(bias);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 u = __ldg(b4 + q);
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[8 * q + j] += cvt_in(e[j]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nvalid) v[j] += cvt_in(bias[j]);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    for (int q = 0; q < p.njobs; ++q) {
+      prefetch_tmap(&p.maps[p.jobs[q].a_map]);
+      prefetch_tmap(&p.maps[p.jobs[q].b_map]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const unsigned long long lim = p.wait_ns;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < p.total_tiles && !*abort_flag; tile += gridDim.x) {
+        const TileCoord tc = tile_coord(p, tile);
+        const GemmJob& j = p.jobs[tc.job];
+        const int m0 = tc.mb * kBM, n0 = tc.nb * kBN;
+        const CUtensorMap* amap = &p.maps[j.a_map];
+        const CUtensorMap* bmap = &p.maps[j.b_map];
+        for (int k = 0; k < j.k_steps; ++k) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, lim)) break;
+          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          uint8_t* a_dst = ring + stage * kStageBytes;
+          uint8_t* b_dst = a_dst + kABytes;
+          const int k0 = k * kBK;
+          if (!j.a_mn) {
+            tma_load_2d(a_dst, amap, &full[stage], k0, m0);
+          } else {
+            tma_load_2d(a_dst, amap, &full[stage], m0, k0);
+            tma_load_2d(a_dst + 8192, amap, &full[stage], m0 + 64, k0);
+          }
+          if (!j.b_mn) {
+            tma_load_2d(b_dst, bmap, &full[stage], k0, n0);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tma_load_2d(b_dst + q * 8192, bmap, &full[stage], n0 + 64 * q, k0);
+          }
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      const uint32_t ring_addr = smem_u32(ring);
+      for (int tile = blockIdx.x; tile < p.total_tiles && !*abort_flag; tile += gridDim.x) {
+        const TileCoord tc = tile_coord(p, tile);
+        const GemmJob& j = p.jobs[tc.job];
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, lim)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kBN;
+        const uint32_t idesc = instr_desc_f16(AbFormat<T>::v, j.a_mn, j.b_mn, kBM, kBN);
+        bool ok = true;
+        for (int k = 0; k < j.k_steps; ++k) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, lim)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = ring_addr + stage * kStageBytes;
+          const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = j.a_mn ? smem_desc(a_addr + kk * 2048, 8192, 1024)
+                                       : smem_desc(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = j.b_mn ? smem_desc(b_addr + kk * 2048, 8192, 1024)
+                                       : smem_desc(b_addr + kk * 32, 16, 1024);
+            mma_f16_ss(d_tmem, ad, bd, idesc, (k | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quarter = warp & 3;  // tensor-memory lanes [32*quarter, 32*quarter+32)
+    const int r_local = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    constexpr float kLog2e = 1.4426950408889634f;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, lim)) break;
+      tc_fence_after();
+      const TileCoord tc = tile_coord(p, tile);
+      const GemmJob& j = p.jobs[tc.job];
+      const int m0 = tc.mb * kBM, n0 = tc.nb * kBN;
+      const int row = m0 + r_local;
+      const bool row_ok = row < j.M;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kBN;
+      if (j.epi == kEpiLse) {
+        const T* bias = reinterpret_cast<const T*>(j.bias);
+        T* logits = reinterpret_cast<T*>(j.logits);
+        const int64_t tgt_rel = row_ok ? (j.targets[row] - (int64_t)n0) : (int64_t)-1;
+        float m_run = -INFINITY, s_run = 0.0f, ztv = 0.0f;
+        bool got = false;
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          float v[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, v);
+          const int col0 = n0 + c * 32;
+          const int nvalid = min(32, j.N - col0);
+          if (nvalid <= 0) continue;
+          if (bias) add_bias32<T>(bias + col0, v, nvalid);
+          float cmax = -INFINITY;
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            if (q < nvalid) cmax = fmaxf(cmax, v[q]);
+          const float m_new = fmaxf(m_run, cmax);
+          const float mb = m_new * kLog2e;
+          float s = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            if (q < nvalid) s += exp2f(fmaf(v[q], kLog2e, -mb));
+          s_run = s_run * exp2f(fmaf(m_run, kLog2e, -mb)) + s;
+          m_run = m_new;
+          const int64_t rel = tgt_rel - c * 32;
+          if (rel >= 0 && rel < 32) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (q == (int)rel) ztv = v[q];
+            got = true;
+          }
+          if (logits && row_ok) store_row32<T>(logits + (int64_t)row * j.logits_ld + col0, v, nvalid);
+        }
+        if (row_ok) {
+          j.part[(int64_t)row * j.part_ld + tc.nb] = make_float2(m_run, s_run);
+          if (got) j.zt[row] = ztv;
+        }
+      } else {
+        const float sc = j.scale ? __ldg(j.scale) : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          float v[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, v);
+          const int col0 = n0 + c * 32;
+          const int nvalid = min(32, j.N - col0);
+          if (!row_ok || nvalid <= 0) continue;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] *= sc;
+          const int64_t off = (int64_t)row * j.out_ld + col0;
+          if (j.acc_in) add_row32_f32(j.acc_in + off, v, nvalid);
+          if (j.out_f32) store_row32_f32(reinterpret_cast<float*>(j.out) + off, v, nvalid);
+          else store_row32<T>(reinterpret_cast<T*>(j.out) + off, v, nvalid);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kDevErrTimeout);
+}
+
+}  // namespace
+
+void gemm_finalize_jobs(GemmParams* p) {
+  int begin = 0;
+  for (int i = 0; i < p->njobs; ++i) {
+    GemmJob& j = p->jobs[i];
+    j.tiles_m = (j.M + kBM - 1) / kBM;
+    j.tiles_n = (j.N + kBN - 1) / kBN;
+    j.k_steps = (j.K + kBK - 1) / kBK;
+    j.tile_begin = begin;
+    begin += j.tiles_m * j.tiles_n;
+  }
+  p->total_tiles = begin;
+}
+
+cudaError_t launch_gemm(const GemmParams& p, DType dt, cudaStream_t stream) {
+  if (p.total_tiles <= 0) return cudaSuccess;
+  DevInfo di;
+  cudaError_t e = dev_info(&di);
+  if (e != cudaSuccess) return e;
+  const int grid = p.total_tiles < di.sm_count ? p.total_tiles : di.sm_count;
+  if (dt == DType::BF16) {
+    static bool attr = false;
+    if (!attr) {
+      e = cudaFuncSetAttribute(gemm_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kGemmSmem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    launch_begin(0, stream);
+    gemm_kernel<__nv_bfloat16><<<grid, kGemmThreads, kGemmSmem, stream>>>(p);
+    launch_end(0, stream);
+  } else if (dt == DType::F16) {
+    static bool attr = false;
+    if (!attr) {
+      e = cudaFuncSetAttribute(gemm_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kGemmSmem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    launch_begin(0, stream);
+    gemm_kernel<__half><<<grid, kGemmThreads, kGemmSmem, stream>>>(p);
+    launch_end(0, stream);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- tensor maps
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+}  // namespace
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, uint64_t outer,
+                  uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (pitch_bytes & 15)) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType t =
+      dt == DType::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = fn(map, t, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace pl

@@ -60,6 +60,12 @@ struct LossArgs {
 cudaError_t launch_loss(const LossArgs& a, DType dt, bool has_kl, bool has_grad, bool two_sided,
                         bool vec, cudaStream_t stream);
 
+// Launch bookkeeping: every kernel launch of the library is bracketed by
+// launch_begin/launch_end (kind: 0 GEMM, 1 loss kernel, 2 other).  Counts
+// launches; records CUDA events on `stream` while timing is enabled.
+void launch_begin(int kind, cudaStream_t stream);
+void launch_end(int kind, cudaStream_t stream);
+
 // Device properties cached per device.
 struct DevInfo {
   int sm_count = 0;
@@ -67,5 +73,13 @@ struct DevInfo {
   size_t smem_optin = 0;
 };
 cudaError_t dev_info(DevInfo* out);
+
+// PL_OK when the current device is compute capability 10.0.
+pl_status check_arch();
+
+// Library-owned, zero-initialised scratch of at least `need` bytes for the
+// current device and `stream` (created or grown when `create`; growing
+// synchronises the stream).  *out is NULL when none exists and !create.
+pl_status own_workspace(cudaStream_t stream, size_t need, void** out, bool create);
 
 }  // namespace pl

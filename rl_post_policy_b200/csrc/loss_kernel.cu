@@ -300,8 +300,10 @@ cudaError_t launch_t(const LossArgs& a0, cudaStream_t stream) {
   grid = a.n > 0 ? (a.n + chunk - 1) / chunk : 1;
   a.chunk = chunk;
   void* args[] = {&a};
-  return cudaLaunchCooperativeKernel((const void*)kern, dim3((unsigned)grid), dim3(kThreads), args, 0,
-                                     stream);
+  launch_begin(1, stream);
+  e = cudaLaunchCooperativeKernel((const void*)kern, dim3((unsigned)grid), dim3(kThreads), args, 0, stream);
+  launch_end(1, stream);
+  return e;
 }
 
 template <typename T>

@@ -42,18 +42,14 @@ pl_status check_arch() {
 }
 
 namespace {
-
-bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
-
-bool finite_nonneg(float x) { return std::isfinite(x) && x >= 0.0f; }
-
-// Library-owned scratch of pl_loss, one per (device, stream).
+// Library-owned scratch, one per (device, stream).
 struct OwnWs {
   void* ptr = nullptr;
   size_t bytes = 0;
 };
 std::mutex g_ws_mu;
 std::map<std::pair<int, cudaStream_t>, OwnWs> g_ws;
+}  // namespace
 
 pl_status own_workspace(cudaStream_t stream, size_t need, void** out, bool create) {
   int dev = -1;
@@ -78,6 +74,12 @@ pl_status own_workspace(cudaStream_t stream, size_t need, void** out, bool creat
   *out = p;
   return PL_OK;
 }
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+bool finite_nonneg(float x) { return std::isfinite(x) && x >= 0.0f; }
 
 constexpr uint32_t kLossModeBits = PL_REDUCTION_MASK | PL_DTYPE_MASK | PL_ADV_LP_DTYPE | PL_CLIP_TWO_SIDED;
 

@@ -1,10 +1,11 @@
 """Seeded synthetic inputs shared by the tests, the benchmark and the oracle checks.
 
 This module draws random numbers and shapes them into the workloads; it holds
-none of the loss or log-probability arithmetic.  Every tensor is produced on the
-CPU by a seeded ``torch.Generator`` (fp32 master values, then rounded to
-nearest-even into the working dtype), so the GPU path and the oracle always see
-the same bits.
+none of the loss or log-probability arithmetic.  Every tensor is produced by a
+seeded ``torch.Generator`` (fp32 master values, then rounded to nearest-even
+into the working dtype).  Parity tests generate on the CPU, so the GPU path and
+the oracle see the same bits; the benchmark may generate the same recipes
+directly on the GPU (``device="cuda"``), which is faster for the 1 GB weights.
 
 Recipes (N(mu, sigma): sigma is the standard deviation; "uniform in [a, b]" on
 integers includes both ends):
@@ -30,14 +31,14 @@ def seed_for(workload: int, variant: int = 0) -> int:
     return SEED_BASE + 16 * workload + variant
 
 
-def _gen(seed: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def _gen(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(int(seed))
     return g
 
 
-def normal(shape, seed: int, std: float = 1.0, mean: float = 0.0) -> torch.Tensor:
-    x = torch.randn(tuple(shape), generator=_gen(seed), dtype=torch.float32)
+def normal(shape, seed: int, std: float = 1.0, mean: float = 0.0, device="cpu") -> torch.Tensor:
+    x = torch.randn(tuple(shape), generator=_gen(seed, device), dtype=torch.float32, device=device)
     if std != 1.0:
         x.mul_(std)
     if mean != 0.0:
@@ -45,26 +46,26 @@ def normal(shape, seed: int, std: float = 1.0, mean: float = 0.0) -> torch.Tenso
     return x
 
 
-def randint(shape, lo: int, hi_inclusive: int, seed: int) -> torch.Tensor:
-    return torch.randint(lo, hi_inclusive + 1, tuple(shape), generator=_gen(seed),
-                         dtype=torch.int64)
+def randint(shape, lo: int, hi_inclusive: int, seed: int, device="cpu") -> torch.Tensor:
+    return torch.randint(lo, hi_inclusive + 1, tuple(shape), generator=_gen(seed, device),
+                         dtype=torch.int64, device=device)
 
 
 def prefix_mask(lengths: torch.Tensor, T: int) -> torch.Tensor:
     """int8 [bs, T] mask whose row b has its first lengths[b] entries set."""
-    pos = torch.arange(T, dtype=torch.int64).unsqueeze(0)
+    pos = torch.arange(T, dtype=torch.int64, device=lengths.device).unsqueeze(0)
     return (pos < lengths.to(torch.int64).unsqueeze(1)).to(torch.int8)
 
 
 def loss_inputs(bs: int, seq: int, dtype: torch.dtype, seed: int,
-                len_lo: int = 64, len_hi: int = 1024) -> dict:
-    """Log-prob inputs for the loss-only kernel (all on CPU)."""
+                len_lo: int = 64, len_hi: int = 1024, device="cpu") -> dict:
+    """Log-prob inputs for the loss-only kernel."""
     s = int(seed)
-    pol = normal((bs, seq), s + 1).abs_().mul_(-2.0)
-    old = pol + normal((bs, seq), s + 2, std=0.1)
-    ref = pol + normal((bs, seq), s + 3, std=0.05)
-    adv = normal((bs,), s + 4)
-    lens = randint((bs,), min(len_lo, seq), min(len_hi, seq), s + 5)
+    pol = normal((bs, seq), s + 1, device=device).abs_().mul_(-2.0)
+    old = pol + normal((bs, seq), s + 2, std=0.1, device=device)
+    ref = pol + normal((bs, seq), s + 3, std=0.05, device=device)
+    adv = normal((bs,), s + 4, device=device)
+    lens = randint((bs,), min(len_lo, seq), min(len_hi, seq), s + 5, device=device)
     return {
         "policy_lp": pol.to(dtype), "old_lp": old.to(dtype), "ref_lp": ref.to(dtype),
         "adv": adv, "mask": prefix_mask(lens, seq), "lengths": lens,
@@ -73,31 +74,35 @@ def loss_inputs(bs: int, seq: int, dtype: torch.dtype, seed: int,
 
 def fused_inputs(bs: int, T: int, H: int, V: int, dtype: torch.dtype, seed: int, *,
                  bias: bool = False, len_lo: int = 1, len_hi: int | None = None,
-                 fully_masked_last: bool = False, need_ref: bool = True) -> dict:
-    """Inputs of the fused linear path (all on CPU).  ``old_noise`` is the
-    N(0,0.1) term the caller adds to the policy log-prob to form old_lp."""
+                 fully_masked_last: bool = False, need_ref: bool = True, device="cpu") -> dict:
+    """Inputs of the fused linear path.  ``old_noise`` is the N(0,0.1) term the
+    caller adds to the policy log-prob to form old_lp."""
     s = int(seed)
     N = bs * T
     len_hi = T if len_hi is None else len_hi
-    X32 = normal((N, H), s + 1)
-    W32 = normal((V, H), s + 2, std=0.02)
-    out = {"X": X32.to(dtype), "W": W32.to(dtype)}
+    X32 = normal((N, H), s + 1, device=device)
+    out = {"X": X32.to(dtype)}
     if need_ref:
-        out["Xref"] = (X32 + normal((N, H), s + 3, std=0.01)).to(dtype)
-        out["Wref"] = (W32 + normal((V, H), s + 4, std=0.002)).to(dtype)
+        out["Xref"] = (X32 + normal((N, H), s + 3, std=0.01, device=device)).to(dtype)
+    del X32
+    W32 = normal((V, H), s + 2, std=0.02, device=device)
+    out["W"] = W32.to(dtype)
+    if need_ref:
+        W32.add_(normal((V, H), s + 4, std=0.002, device=device))
+        out["Wref"] = W32.to(dtype)
     else:
         out["Xref"] = None
         out["Wref"] = None
-    del X32, W32
-    out["bias"] = normal((V,), s + 5, std=0.01).to(dtype) if bias else None
-    out["targets"] = randint((N,), 0, V - 1, s + 6)
-    out["adv"] = normal((bs,), s + 7)
-    lens = randint((bs,), min(len_lo, T), min(len_hi, T), s + 8)
+    del W32
+    out["bias"] = normal((V,), s + 5, std=0.01, device=device).to(dtype) if bias else None
+    out["targets"] = randint((N,), 0, V - 1, s + 6, device=device)
+    out["adv"] = normal((bs,), s + 7, device=device)
+    lens = randint((bs,), min(len_lo, T), min(len_hi, T), s + 8, device=device)
     if fully_masked_last and bs > 0:
         lens[bs - 1] = 0
     out["lengths"] = lens
     out["mask"] = prefix_mask(lens, T)
-    out["old_noise"] = normal((N,), s + 9, std=0.1)
+    out["old_noise"] = normal((N,), s + 9, std=0.1, device=device)
     return out
 
 

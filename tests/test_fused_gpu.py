@@ -1,0 +1,156 @@
+"""Parity of the fused linear path (pl_fused_linear_grpo) with the CPU oracle.
+
+Tolerances: selected log-probs abs <= 2e-3; loss relative <= 1e-3; dX, dW and
+dbias relative Frobenius <= 1e-2; the valid-token count bit-exact.  Inputs are
+seeded; a test asserts that no token sits within 1e-4 (in log space) of the clip
+bound, where fp32 and fp64 may legitimately choose different sides of the min().
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+EPS_LO, EPS_HI = 0.2, 0.28
+
+
+def pl():
+    import rl_post_policy_b200 as m
+    return m
+
+
+def build_inputs(bs, T, H, V, dtype, seed, bias=False, beta=0.04, len_lo=1, len_hi=None,
+                 fully_masked_last=False):
+    inp = synth.fused_inputs(bs, T, H, V, dtype, seed, bias=bias, len_lo=len_lo, len_hi=len_hi,
+                             fully_masked_last=fully_masked_last, need_ref=True)
+    _, logp, _ = oracle.lm_head_logprob(inp["X"], inp["W"], inp["bias"], inp["targets"])
+    inp["old_lp"] = (torch.from_numpy(logp) + inp["old_noise"].double()).float()
+    return inp
+
+
+def run_fused(inp, dtype, red, beta, chunk=None, want=("dX", "dW", "dbias"), two_sided=False,
+              targets=None):
+    m = pl()
+    dev = "cuda"
+    bs, T = inp["mask"].shape
+    N, H = inp["X"].shape
+    V = inp["W"].shape[0]
+    X, W = inp["X"].to(dev), inp["W"].to(dev)
+    b = inp["bias"].to(dev) if inp["bias"] is not None else None
+    Xr = inp["Xref"].to(dev) if beta != 0 else None
+    Wr = inp["Wref"].to(dev) if beta != 0 else None
+    tg = (targets if targets is not None else inp["targets"]).to(dev)
+    old = inp["old_lp"].to(dev)
+    adv = inp["adv"].float().to(dev)
+    mask = inp["mask"].to(dev)
+    loss = torch.full((1,), float("nan"), device=dev)
+    dX = torch.full((N, H), float("nan"), dtype=dtype, device=dev) if "dX" in want else None
+    dW = torch.full((V, H), float("nan"), dtype=dtype, device=dev) if "dW" in want else None
+    db = (torch.full((V,), float("nan"), dtype=dtype, device=dev)
+          if ("dbias" in want and b is not None) else None)
+    lp = torch.full((N,), float("nan"), device=dev)
+    rlp = torch.full((N,), float("nan"), device=dev)
+    nv = torch.full((1,), -1, dtype=torch.int64, device=dev)
+    mode = m.dtype_mode(dtype) | red | (m.PL_CLIP_TWO_SIDED if two_sided else 0)
+    if chunk:
+        mode |= m.PL_CHUNK_ROWS(chunk)
+    wsb = m.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, dW is not None, db is not None)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    rc = m.pl_fused_linear_grpo(X, W, b, tg, Xr, Wr, old, adv, mask, bs, T, H, V, EPS_LO, EPS_HI,
+                                beta, mode, loss, dX, dW, db, lp, rlp, nv, ws, wsb)
+    m.check(rc, "pl_fused_linear_grpo")
+    torch.cuda.synchronize()
+    status = m.pl_device_status(ws)
+    out = {"loss": loss.item(), "logp": lp.cpu().double().numpy(), "ref_logp": rlp.cpu().double().numpy(),
+           "n_valid": int(nv.item()), "status": status}
+    for k, t in (("dX", dX), ("dW", dW), ("dbias", db)):
+        out[k] = None if t is None else t.cpu().double().numpy()
+    return out
+
+
+def rel_fro(a, b):
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+def check(inp, got, red, beta, two_sided=False, check_grads=True):
+    want = oracle.fused_grpo(inp["X"], inp["W"], inp["bias"], inp["targets"], inp["Xref"],
+                             inp["Wref"], inp["old_lp"].reshape(inp["mask"].shape), inp["adv"],
+                             inp["mask"], eps_lo=EPS_LO, eps_hi=EPS_HI, beta=beta, reduction=red,
+                             two_sided=two_sided)
+    old = inp["old_lp"].double().numpy()
+    d = want["logp"] - old
+    assert np.all(np.abs(d - np.log(float(np.float32(1) + np.float32(EPS_HI)))) > 1e-4)
+    assert got["status"] == 0
+    assert got["n_valid"] == want["n_valid"]
+    assert np.max(np.abs(got["logp"] - want["logp"])) <= 2e-3
+    if beta != 0:
+        assert np.max(np.abs(got["ref_logp"] - want["ref_logp"])) <= 2e-3
+    assert abs(got["loss"] - want["loss"]) <= 1e-3 * abs(want["loss"]), (got["loss"], want["loss"])
+    if check_grads:
+        for k in ("dX", "dW", "dbias"):
+            if got.get(k) is not None:
+                e = rel_fro(got[k], want[k])
+                assert e <= 1e-2, (k, e)
+    return want
+
+
+@pytest.mark.parametrize("red", [0, 1], ids=["bnpo", "grpo"])
+def test_tiny_workload(red):
+    w = synth.WORKLOADS[0]
+    inp = build_inputs(w["bs"], w["T"], w["H"], w["V"], w["dtype"], synth.seed_for(0),
+                       len_lo=w["len_lo"], len_hi=w["len_hi"])
+    got = run_fused(inp, w["dtype"], red, w["beta"])
+    check(inp, got, red, w["beta"])
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16], ids=["bf16", "fp16"])
+@pytest.mark.parametrize("chunk", [None, 128], ids=["one_chunk", "chunks128"])
+@pytest.mark.parametrize("beta", [0.04, 0.0], ids=["beta0.04", "beta0"])
+def test_ragged_multi_tile(dtype, chunk, beta):
+    # N=300 rows (3 row tiles, ragged), H=200 (K tail), V=1000 (4 vocab tiles, ragged), bias
+    inp = build_inputs(3, 100, 200, 1000, dtype, 4242, bias=True, len_lo=0, len_hi=100,
+                       fully_masked_last=True)
+    for red in (0, 1):
+        got = run_fused(inp, dtype, red, beta, chunk=chunk)
+        check(inp, got, red, beta)
+
+
+def test_two_sided_clip():
+    inp = build_inputs(2, 64, 128, 640, torch.bfloat16, 99, bias=False)
+    got = run_fused(inp, torch.bfloat16, 1, 0.04, two_sided=True)
+    check(inp, got, 1, 0.04, two_sided=True)
+
+
+@pytest.mark.parametrize("want", [("dX",), ("dW",), ("dbias",), ()])
+def test_partial_gradients(want):
+    inp = build_inputs(2, 96, 128, 700, torch.bfloat16, 7, bias=True)
+    got = run_fused(inp, torch.bfloat16, 1, 0.04, want=want, chunk=128)
+    check(inp, got, 1, 0.04)
+
+
+def test_bad_target_is_flagged_and_masked():
+    m = pl()
+    inp = build_inputs(2, 32, 64, 512, torch.bfloat16, 11)
+    bad = inp["targets"].clone()
+    bad[0] = 512  # == V: out of range (position 0 is always inside the valid prefix)
+    got = run_fused(inp, torch.bfloat16, 0, 0.04, targets=bad)
+    assert got["status"] == m.PL_ERR_BAD_TARGET
+    assert np.isnan(got["logp"][0])
+    # the row counts as masked: compare against the oracle with that token masked out
+    masked = dict(inp)
+    mk = inp["mask"].clone().reshape(-1)
+    mk[0] = 0
+    masked["mask"] = mk.reshape(inp["mask"].shape)
+    want = oracle.fused_grpo(inp["X"], inp["W"], None, inp["targets"], inp["Xref"], inp["Wref"],
+                             inp["old_lp"].reshape(2, 32), inp["adv"], masked["mask"], eps_lo=EPS_LO,
+                             eps_hi=EPS_HI, beta=0.04, reduction=0)
+    # the token contributes nothing, but the BNPO denominator is the mask's own count
+    n_orig = int(inp["mask"].sum())
+    expect = want["loss"] * (n_orig - 1) / n_orig
+    assert got["n_valid"] == n_orig
+    assert abs(got["loss"] - expect) <= 1e-3 * abs(expect)
+    assert np.all(got["dX"][0] == 0.0)
