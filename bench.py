@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of the fused GRPO policy-loss hot path on B200.
+
+One step = the whole hot path on one synthetic batch: the policy and reference
+lm_head GEMMs with the logsumexp / target-logit epilogue, the clipped-ratio GRPO
+loss with the KL term, the in-place dlogits pass, and the dX / dW GEMMs, all
+through the C ABI (pl_fused_linear_grpo) with inputs resident in HBM.  The default
+workload is batch 1 x T=1024, H=4096, V=128256, bf16 (the shape of the published
+B200 table of "Add SM100 CuTe DSL GRPO fast path", Liger-Kernel PR #1363).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  Under torchrun each rank runs its own batch
+(weak scaling, no data-path collective); the time is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import torch  # noqa: E402
+
+METRIC = "fused GRPO fwd+bwd tokens/s and % of B200 BF16 tensor peak; loss-only GB/s"
+# Published CuTe-DSL latency at batch 1, T=1024, H=4096, V=128256, BF16 on B200
+# ("Add SM100 CuTe DSL GRPO fast path", "B200 results" table).
+PUBLISHED_MS = {1: 6.69, 2: 12.09, 4: 23.07, 8: 43.79}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+EPS_LO, EPS_HI = 0.2, 0.28
+GEMM_SOURCES = ["rl_post_policy_b200/csrc/gemm_tc.cu", "rl_post_policy_b200/csrc/sm100.cuh",
+                "rl_post_policy_b200/csrc/gemm.h"]
+LOSS_SOURCES = ["rl_post_policy_b200/csrc/loss_kernel.cu", "rl_post_policy_b200/csrc/policy_math.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5])
+    ap.add_argument("--no-loss-only", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=64, help="rows in the oracle's timed sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        return json.loads(p.read_text()), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def sources_sha(paths) -> str:
+    h = hashlib.sha256()
+    for rel in paths:
+        h.update((ROOT / rel).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, paths):
+    """Per-launch DRAM bytes from an ncu capture, if taken on the current sources."""
+    f = ROOT / "profiles" / "traffic.json"
+    if not f.exists():
+        return None
+    d = json.loads(f.read_text()).get(kernel)
+    if not d or d.get("sources_sha") != sources_sha(paths):
+        return None
+    return d.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ distributed
+def dist_init(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.sel = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.sel:
+            cmd += ["-i", self.sel]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        load = [x for x in sm if mx and x > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload
+def workload_desc(w: int) -> dict:
+    import synth
+    d = dict(synth.WORKLOADS[w])
+    d["N"] = d["bs"] * d["T"]
+    return d
+
+
+def make_fused_inputs(w: int, rank: int):
+    """Synthetic inputs on the GPU; old_lp = policy log-prob (from a forward-only
+    call of the same entry point) + N(0, 0.1)."""
+    import rl_post_policy_b200 as pl
+    import synth
+    d = workload_desc(w)
+    inp = synth.fused_inputs(d["bs"], d["T"], d["H"], d["V"], d["dtype"], synth.seed_for(w, rank),
+                             bias=d.get("bias", False), len_lo=d["len_lo"], len_hi=d["len_hi"],
+                             fully_masked_last=d.get("fully_masked_last", False), device="cuda")
+    N, V, H, bs, T = d["N"], d["V"], d["H"], d["bs"], d["T"]
+    mode = pl.dtype_mode(d["dtype"]) | pl.PL_GRPO
+    wsb = pl.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, 1, int(inp["bias"] is not None))
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    loss = torch.zeros(1, device="cuda")
+    logp = torch.zeros(N, device="cuda")
+    zeros = torch.zeros(N, device="cuda")
+    pl.check(pl.pl_fused_linear_grpo(inp["X"], inp["W"], inp["bias"], inp["targets"], None, None, zeros,
+                                     inp["adv"], inp["mask"], bs, T, H, V, EPS_LO, EPS_HI, 0.0, mode, loss,
+                                     None, None, None, logp, None, None, ws, wsb), "forward for old_lp")
+    torch.cuda.synchronize()
+    inp["old_lp"] = (logp + inp["old_noise"]).contiguous()
+    return d, inp, ws, wsb, mode
+
+
+class FusedStep:
+    def __init__(self, d, inp, ws, wsb, mode):
+        import rl_post_policy_b200 as pl
+        self.pl, self.d, self.inp, self.ws, self.wsb, self.mode = pl, d, inp, ws, wsb, mode
+        N, H, V = d["N"], d["H"], d["V"]
+        self.loss = torch.zeros(1, device="cuda")
+        self.dX = torch.empty(N, H, dtype=d["dtype"], device="cuda")
+        self.dW = torch.empty(V, H, dtype=d["dtype"], device="cuda")
+        self.db = torch.empty(V, dtype=d["dtype"], device="cuda") if inp["bias"] is not None else None
+
+    def __call__(self, X=None, Xref=None, targets=None, old_lp=None, adv=None, mask=None):
+        i, d = self.inp, self.d
+        rc = self.pl.pl_fused_linear_grpo(
+            i["X"] if X is None else X, i["W"], i["bias"], i["targets"] if targets is None else targets,
+            i["Xref"] if Xref is None else Xref, i["Wref"], i["old_lp"] if old_lp is None else old_lp,
+            i["adv"] if adv is None else adv, i["mask"] if mask is None else mask, d["bs"], d["T"], d["H"],
+            d["V"], EPS_LO, EPS_HI, d["beta"], self.mode, self.loss, self.dX, self.dW, self.db, None, None,
+            None, self.ws, self.wsb)
+        if rc != 0:
+            raise RuntimeError(f"pl_fused_linear_grpo: {self.pl.pl_status_string(rc)}")
+
+
+def time_steps(fn, steps, ws_world):
+    s = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws_world)
+    torch.cuda.synchronize()
+    a.record(s)
+    for _ in range(steps):
+        fn()
+    b.record(s)
+    torch.cuda.synchronize()
+    barrier(ws_world)
+    return a.elapsed_time(b)
+
+
+# ------------------------------------------------------------------ loss-only kernel
+def loss_only(peaks, peak_kind):
+    """Bandwidth of the single-launch loss kernel on a large bf16 batch (bs=16,
+    seq=2^23: inputs ~1.2 GB, far larger than L2) and the latency at bs=16 x 1024."""
+    import rl_post_policy_b200 as pl
+    import synth
+    res = {}
+    for name, (bs, seq, reps) in {"sweep": (16, 1 << 23, 10), "small": (16, 1024, 200)}.items():
+        inp = synth.loss_inputs(bs, seq, torch.bfloat16, synth.seed_for(1, 1), len_lo=min(64, seq),
+                                len_hi=seq, device="cuda")
+        g = torch.empty_like(inp["policy_lp"])
+        loss = torch.zeros(1, device="cuda")
+        wsb = pl.pl_loss_workspace_bytes(bs, seq)
+        ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+        mode = pl.PL_BF16 | pl.PL_BNPO
+
+        def call():
+            pl.pl_loss_ex(inp["policy_lp"], inp["old_lp"], inp["ref_lp"], inp["adv"], inp["mask"], bs, seq,
+                          EPS_LO, EPS_HI, 0.04, mode, loss, g, None, None, ws, wsb)
+
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        pl.pl_debug_timing_read()
+        pl.pl_debug_timing(True)
+        for _ in range(reps):
+            call()
+        torch.cuda.synchronize()
+        pl.pl_debug_timing(False)
+        ms, n = pl.pl_debug_timing_read()
+        per = ms[1] / max(n[1], 1)
+        tokens = bs * seq
+        bytes_ = 9 * tokens  # 3 bf16 reads + bf16 grad write + 1 mask byte
+        gbs = bytes_ / (per * 1e-3) / 1e9
+        res[name] = {"bs": bs, "seq": seq, "us_per_call": per * 1e3, "GB_per_s": gbs,
+                     "tokens_per_s": tokens / (per * 1e-3), "algorithmic_bytes": bytes_}
+        del inp, g, ws
+    peak = float(peaks["hbm_gbs"])
+    sw = res["sweep"]
+    return {
+        "metric": "loss-only GB/s", "value": sw["GB_per_s"], "unit": "GB/s",
+        "workload": "loss-only BNPO fwd+bwd, bf16, beta=0.04, bs=16 x seq=8388608 (inputs > L2)",
+        "roofline": {"bound": "hbm", "achieved": sw["GB_per_s"], "peak": peak, "unit": "GB/s",
+                     "frac": sw["GB_per_s"] / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                     "traffic": recorded_traffic("loss_kernel", LOSS_SOURCES)},
+        "small_workload": {"workload": "bs=16 x seq=1024 (launch-latency bound)",
+                           "us_per_call": res["small"]["us_per_call"],
+                           "tokens_per_s": res["small"]["tokens_per_s"]},
+    }
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(inp, d, rows):
+    """The fp64 oracle on the first `rows` rows of the batch (one sequence of
+    `rows` tokens): policy + reference forward over the full vocabulary, the
+    loss, and dX / dW / dbias for those rows.  Returns (seconds, threads)."""
+    import oracle
+    cpu = {k: (v[:rows].cpu() if k in ("X", "Xref", "targets", "old_lp") else v)
+           for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    W = inp["W"].cpu()
+    Wref = inp["Wref"].cpu() if inp.get("Wref") is not None else None
+    bias = inp["bias"].cpu() if inp.get("bias") is not None else None
+    mask = inp["mask"].reshape(-1)[:rows].reshape(1, rows).cpu()
+    adv = inp["adv"][:1].cpu()
+    t0 = time.perf_counter()
+    oracle.fused_grpo(cpu["X"], W, bias, cpu["targets"], cpu.get("Xref"), Wref,
+                      cpu["old_lp"].reshape(1, rows), adv, mask, eps_lo=EPS_LO, eps_hi=EPS_HI,
+                      beta=d["beta"], reduction=oracle.GRPO)
+    return time.perf_counter() - t0, oracle.threads()
+
+
+# ------------------------------------------------------------------ arms
+def run_reference(args):
+    ws_world, rank = dist_init(args)
+    if rank != 0:
+        return
+    d = workload_desc(args.workload)
+    import oracle  # noqa: F401
+    # Inputs: the same recipe, generated on the CPU (no GPU work on this arm).
+    import synth
+    rows = max(1, min(args.cpu_rows // 4, d["N"]))
+    inp = synth.fused_inputs(1, rows, d["H"], d["V"], d["dtype"], synth.seed_for(args.workload),
+                             bias=d.get("bias", False), len_lo=rows, len_hi=rows)
+    import oracle as orc
+    _, lp, _ = orc.lm_head_logprob(inp["X"], inp["W"], inp["bias"], inp["targets"])
+    inp["old_lp"] = (torch.from_numpy(lp) + inp["old_noise"].double()).float()
+    times = []
+    for i in range(args.warmup + args.steps):
+        t, cores = oracle_sample(inp, d, rows)
+        if i >= args.warmup:
+            times.append(t)
+    per = sum(times) / len(times)
+    val = rows / per
+    sample = (f"{rows} rows (one sequence) of the workload per step: policy+reference forward over "
+              f"V={d['V']}, loss, dX/dW/dbias, fp64")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"fused GRPO fwd+bwd, bs=1 x T={rows} sample of workload {args.workload}",
+                   "H": d["H"], "V": d["V"]},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }), flush=True)
+
+
+def run_ours(args):
+    ws_world, rank = dist_init(args)
+    import rl_post_policy_b200 as pl
+    peaks, peak_kind = load_peaks()
+    d, inp, ws, wsb, mode = make_fused_inputs(args.workload, rank)
+    step = FusedStep(d, inp, ws, wsb, mode)
+    N, H, V = d["N"], d["H"], d["V"]
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    pl.check(pl.pl_device_status(ws), "device status after warm-up")
+
+    # ---- device-resident timed region ----
+    clocks = ClockSampler(torch.cuda.current_device())
+    pl.pl_debug_timing_read()
+    launches0 = pl.pl_debug_launch_count()
+    clocks.start()
+    pl.pl_debug_timing(True)
+    elapsed = time_steps(step, args.steps, ws_world)
+    pl.pl_debug_timing(False)
+    clk = clocks.stop()
+    launches = pl.pl_debug_launch_count() - launches0
+    kms, kn = pl.pl_debug_timing_read()
+    pl.check(pl.pl_device_status(ws), "device status after timing")
+    t_max = max_over_ranks(elapsed, ws_world)
+    ms_per_step = t_max / args.steps
+    total_tokens = sum_over_ranks(float(N * args.steps), ws_world)
+    value = total_tokens / (t_max * 1e-3)
+
+    # ---- roofline of the dominant kernel (the tcgen05 GEMM) ----
+    flops_step = (8 if d["beta"] != 0 else 6) * N * H * V
+    gemm_ms = kms[0] / max(kn[0], 1)
+    gemm_flops_launch = flops_step * args.steps / max(kn[0], 1)
+    achieved = gemm_flops_launch / (gemm_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    if d["dtype"] == torch.float16:
+        peak_note = f"{peak_kind} bf16 sustained x 1.0 (fp16 nominal ratio 1:1)"
+    else:
+        peak_note = f"{peak_kind} bf16 sustained (the GEMMs run back to back for seconds)"
+    step_tflops = flops_step / (ms_per_step * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": recorded_traffic("gemm_kernel", GEMM_SOURCES),
+                "kernel": "gemm_kernel (tcgen05 persistent GEMM)", "peak_source": peak_note,
+                "launch_ms": gemm_ms, "launches": kn[0],
+                "share_of_step": kms[0] / max(sum(kms), 1e-9),
+                "step_tflops": step_tflops, "step_frac_of_peak": step_tflops / peak}
+
+    # ---- end to end through the C ABI from pinned host buffers ----
+    host = {k: inp[k].cpu().pin_memory() for k in ("X", "Xref", "targets", "old_lp", "adv", "mask")}
+    dev = {k: torch.empty_like(inp[k]) for k in host}
+    loss_host = torch.zeros(1).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+
+    def e2e_step():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        step(**dev)
+        loss_host.copy_(step.loss, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_ms = max_over_ranks(time_steps(e2e_step, args.steps, ws_world), ws_world) / args.steps
+    e2e_val = total_tokens / args.steps / (e2e_ms * 1e-3)
+
+    extra = {}
+    if rank == 0 and ws_world == 1 and not args.no_loss_only:
+        extra["loss_only"] = loss_only(peaks, peak_kind)
+    cpu = None
+    if rank == 0 and ws_world == 1 and not args.no_cpu_baseline:
+        rows = max(1, min(args.cpu_rows, N))
+        secs, cores = oracle_sample(inp, d, rows)
+        cpu = {"value": rows / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {rows} rows of the batch as one sequence: policy+reference forward over "
+                         f"V={V}, GRPO loss, dX/dW/dbias, fp64 ({secs:.1f} s)"}
+
+    if rank == 0:
+        bsz = d["bs"]
+        pub = PUBLISHED_MS.get(bsz) if (args.workload in (2, 4) and H == 4096 and V == 128256) else None
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": (value / ws_world) / (N / (pub * 1e-3)) if pub else None,
+            "dtype": "bf16" if d["dtype"] == torch.bfloat16 else "fp16", "data": "synthetic",
+            "config": {"workload": f"fused GRPO fwd+bwd, bs={d['bs']} x T={d['T']} (N={N}), H={H}, V={V}, "
+                                   f"beta={d['beta']}, GRPO, eps=0.2/0.28",
+                       "per_gpu_rows": N, "chunk_rows": 1024,
+                       "l2": "inputs larger than L2 (W and Wref are 1 GB each); no flush",
+                       "parallelism": f"dp{ws_world} (independent batches)"},
+            "clocks": clk, "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                                   "d2h_bytes_per_step": 4, "ms_per_step": e2e_ms},
+            "gpu_launches": launches, "roofline": roofline, "cpu_baseline": cpu,
+            "kernel_ms_per_step": {"gemm": kms[0] / args.steps, "loss_kernel": kms[1] / args.steps,
+                                   "other": kms[2] / args.steps},
+        }
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+    if ws_world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

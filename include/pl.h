@@ -116,7 +116,7 @@ pl_status pl_loss(const void* policy_lp, const void* old_lp, const void* ref_lp,
  *   n_valid_out   : device int64 scalar, the global valid-token count, or NULL.
  *   row_valid_out : device int64 [bs], the per-sequence counts, or NULL.
  *   workspace     : device buffer of at least pl_loss_workspace_bytes(bs, seq) bytes,
- *                   zero-filled by the caller ONCE after allocation; the kernel
+ *                   256-byte aligned, zero-filled by the caller ONCE after allocation; the kernel
  *                   returns its counters to zero, so it stays reusable.  Calls that
  *                   share a workspace must be ordered on one stream.
  */
@@ -161,7 +161,8 @@ size_t pl_loss_workspace_bytes(int64_t bs, int64_t seq);
  *                                        written only when beta != 0).
  *   n_valid_out                        : optional device int64 scalar.
  *   workspace                          : at least pl_fused_linear_grpo_workspace_bytes()
- *                                        bytes, zero-filled once after allocation.
+ *                                        bytes, 256-byte aligned, zero-filled once after
+ *                                        allocation; calls sharing it must be stream-ordered.
  */
 pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias,
                                const int64_t* targets, const void* Xref, const void* Wref,

@@ -37,6 +37,19 @@ pl_status pl_debug_gemm(const void* A, int a_mn, int64_t lda, const void* B, int
 void pl_debug_timing(int enable);
 pl_status pl_debug_timing_read(double* ms, int64_t* launches);
 
+/*
+ * Failure-detection test knobs, applied to later launches on this process.
+ *   wait_ns        : bound on every device-side wait (0 restores the default, 2 s).
+ *   extra_arrivals : the loss kernel's grid barrier waits for this many arrivals
+ *                    beyond the blocks that exist, so it runs out after wait_ns.
+ *   extra_tx       : each GEMM pipeline stage expects this many bytes beyond its
+ *                    TMA loads, so its wait runs out after wait_ns.
+ * A wait that runs out raises PL_ERR_DEVICE_TIMEOUT (pl_device_status); the
+ * kernel then releases tensor memory and returns, and the context stays usable.
+ * Pass (0, 0, 0) to restore normal operation.
+ */
+void pl_debug_set_wait(unsigned long long wait_ns, unsigned extra_arrivals, unsigned extra_tx);
+
 /* Number of kernels this library has launched in this process. */
 int64_t pl_debug_launch_count(void);
 

@@ -1,173 +1,14 @@
-"""Thin Python binding of libpl.so (the C ABI declared in include/pl.h).
+"""B200 (sm_100a) fused GRPO/BNPO policy loss: Python side of libpl.so.
 
-Every function here has the name of the C entry point it calls and does
-argument marshalling only: torch tensors become device pointers, torch streams
-become cudaStream_t handles.  All arithmetic runs in the library's CUDA
-kernels.  If libpl.so has not been built, importing this package raises
-ImportError: there is no fallback path.
+The binding (``rl_post_policy_b200.binding``) is loaded on first attribute
+access, so ``python -m rl_post_policy_b200.build`` can rebuild the library
+without loading an older copy of it.  Accessing any entry point when libpl.so
+has not been built raises ImportError: there is no fallback path.
 """
-from __future__ import annotations
-
-import ctypes
-from pathlib import Path
-
-_PKG = Path(__file__).resolve().parent
-LIB_PATH = _PKG / "libpl.so"
-
-if not LIB_PATH.exists():
-    raise ImportError(
-        f"{LIB_PATH} is missing; build it with `python -m rl_post_policy_b200.build` "
-        "(nvcc, sm_100a). There is no CPU fallback.")
-
-_lib = ctypes.CDLL(str(LIB_PATH))
-
-# ---- constants mirrored from include/pl.h --------------------------------------
-PL_OK, PL_ERR_ARG, PL_ERR_DTYPE, PL_ERR_ALIGN, PL_ERR_WORKSPACE = 0, 1, 2, 3, 4
-PL_ERR_ARCH, PL_ERR_CUDA, PL_ERR_DEVICE_TIMEOUT, PL_ERR_BAD_TARGET = 5, 6, 7, 8
-PL_BNPO, PL_GRPO = 0, 1
-PL_F32, PL_F16, PL_BF16 = 0 << 4, 1 << 4, 2 << 4
-PL_ADV_LP_DTYPE = 1 << 8
-PL_CLIP_TWO_SIDED = 1 << 9
-PL_CHUNK_SHIFT = 16
+import importlib
 
 
-def PL_CHUNK_ROWS(n: int) -> int:
-    return ((n // 128) & 0xFF) << PL_CHUNK_SHIFT
-
-
-_P, _I64, _U32, _F, _SZ, _I = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float,
-                               ctypes.c_size_t, ctypes.c_int)
-
-_lib.pl_loss.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _F, _F, _F, _U32, _P, _P, _P]
-_lib.pl_loss.restype = _I
-_lib.pl_loss_ex.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _F, _F, _F, _U32, _P, _P, _P, _P, _P,
-                            _SZ, _P]
-_lib.pl_loss_ex.restype = _I
-_lib.pl_loss_workspace_bytes.argtypes = [_I64, _I64]
-_lib.pl_loss_workspace_bytes.restype = _SZ
-_lib.pl_fused_linear_grpo.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64,
-                                      _F, _F, _F, _U32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
-_lib.pl_fused_linear_grpo.restype = _I
-_lib.pl_fused_linear_grpo_workspace_bytes.argtypes = [_I64, _I64, _I64, _I64, _U32, _I, _I]
-_lib.pl_fused_linear_grpo_workspace_bytes.restype = _SZ
-_lib.pl_device_status.argtypes = [_P, _P]
-_lib.pl_device_status.restype = _I
-_lib.pl_status_string.argtypes = [_I]
-_lib.pl_status_string.restype = ctypes.c_char_p
-_lib.pl_version.argtypes = []
-_lib.pl_version.restype = _I
-_lib.pl_debug_gemm.argtypes = [_P, _I, _I64, _P, _I, _I64, _P, _I64, _I64, _I64, _U32, _P]
-_lib.pl_debug_gemm.restype = _I
-_lib.pl_debug_timing.argtypes = [_I]
-_lib.pl_debug_timing.restype = None
-_lib.pl_debug_timing_read.argtypes = [_P, _P]
-_lib.pl_debug_timing_read.restype = _I
-_lib.pl_debug_launch_count.argtypes = []
-_lib.pl_debug_launch_count.restype = _I64
-
-EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
-            "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
-            "pl_version", "pl_debug_gemm", "pl_debug_timing", "pl_debug_timing_read",
-            "pl_debug_launch_count")
-
-
-class PLError(RuntimeError):
-    def __init__(self, status: int, where: str):
-        super().__init__(f"{where}: {pl_status_string(status)}")
-        self.status = status
-
-
-def _ptr(x):
-    """Device pointer of a tensor, an int address, or NULL for None."""
-    if x is None:
-        return None
-    if isinstance(x, int):
-        return x
-    return x.data_ptr()
-
-
-def _stream(s):
-    if s is None:
-        import torch
-        return torch.cuda.current_stream().cuda_stream
-    if isinstance(s, int):
-        return s
-    return s.cuda_stream
-
-
-def dtype_mode(dtype) -> int:
-    import torch
-    return {torch.float32: PL_F32, torch.float16: PL_F16, torch.bfloat16: PL_BF16}[dtype]
-
-
-def check(status: int, where: str = "libpl") -> None:
-    if status != PL_OK:
-        raise PLError(status, where)
-
-
-# ---- C entry points ---------------------------------------------------------------
-def pl_loss(policy_lp, old_lp, ref_lp, adv, mask, bs, seq, eps_lo, eps_hi, beta, mode, loss_out,
-            grad_out, stream=None) -> int:
-    return _lib.pl_loss(_ptr(policy_lp), _ptr(old_lp), _ptr(ref_lp), _ptr(adv), _ptr(mask), bs, seq,
-                        eps_lo, eps_hi, beta, mode, _ptr(loss_out), _ptr(grad_out), _stream(stream))
-
-
-def pl_loss_ex(policy_lp, old_lp, ref_lp, adv, mask, bs, seq, eps_lo, eps_hi, beta, mode, loss_out,
-               grad_out, n_valid_out, row_valid_out, workspace, ws_bytes, stream=None) -> int:
-    return _lib.pl_loss_ex(_ptr(policy_lp), _ptr(old_lp), _ptr(ref_lp), _ptr(adv), _ptr(mask), bs,
-                           seq, eps_lo, eps_hi, beta, mode, _ptr(loss_out), _ptr(grad_out),
-                           _ptr(n_valid_out), _ptr(row_valid_out), _ptr(workspace), ws_bytes,
-                           _stream(stream))
-
-
-def pl_loss_workspace_bytes(bs, seq) -> int:
-    return int(_lib.pl_loss_workspace_bytes(bs, seq))
-
-
-def pl_fused_linear_grpo(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, bs, T, H, V, eps_lo,
-                         eps_hi, beta, mode, loss, dX, dW, dbias, logp_out, ref_logp_out,
-                         n_valid_out, workspace, ws_bytes, stream=None) -> int:
-    return _lib.pl_fused_linear_grpo(
-        _ptr(X), _ptr(W), _ptr(bias), _ptr(targets), _ptr(Xref), _ptr(Wref), _ptr(old_lp),
-        _ptr(adv), _ptr(mask), bs, T, H, V, eps_lo, eps_hi, beta, mode, _ptr(loss), _ptr(dX),
-        _ptr(dW), _ptr(dbias), _ptr(logp_out), _ptr(ref_logp_out), _ptr(n_valid_out),
-        _ptr(workspace), ws_bytes, _stream(stream))
-
-
-def pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, need_dW, need_dbias) -> int:
-    return int(_lib.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, int(need_dW),
-                                                         int(need_dbias)))
-
-
-def pl_device_status(workspace=None, stream=None) -> int:
-    return _lib.pl_device_status(_ptr(workspace), _stream(stream))
-
-
-def pl_status_string(status: int) -> str:
-    return _lib.pl_status_string(status).decode()
-
-
-def pl_version() -> int:
-    return int(_lib.pl_version())
-
-
-def pl_debug_gemm(A, a_mn, lda, B, b_mn, ldb, D, M, N, K, mode, stream=None) -> int:
-    """Test hook (include/pl_debug.h): plain GEMM through the tcgen05 kernel."""
-    return _lib.pl_debug_gemm(_ptr(A), int(a_mn), lda, _ptr(B), int(b_mn), ldb, _ptr(D), M, N, K,
-                              mode, _stream(stream))
-
-
-def pl_debug_timing(enable: bool) -> None:
-    _lib.pl_debug_timing(int(bool(enable)))
-
-
-def pl_debug_timing_read():
-    """((gemm_ms, loss_ms, other_ms), (gemm_launches, loss_launches, other_launches))."""
-    ms = (ctypes.c_double * 3)()
-    n = (ctypes.c_int64 * 3)()
-    check(_lib.pl_debug_timing_read(ms, n), "pl_debug_timing_read")
-    return tuple(ms), tuple(n)
-
-
-def pl_debug_launch_count() -> int:
-    return int(_lib.pl_debug_launch_count())
+def __getattr__(name):
+    if name.startswith("__") or name in ("binding", "build"):
+        raise AttributeError(name)
+    return getattr(importlib.import_module(__name__ + ".binding"), name)

@@ -72,6 +72,20 @@ void launch_end(int kind, cudaStream_t stream) {
 }
 }  // namespace pl
 
+namespace pl {
+DebugKnobs& debug_knobs() {
+  static DebugKnobs k;
+  return k;
+}
+}  // namespace pl
+
+extern "C" void pl_debug_set_wait(unsigned long long wait_ns, unsigned extra_arrivals, unsigned extra_tx) {
+  DebugKnobs& k = debug_knobs();
+  k.wait_ns = wait_ns ? wait_ns : kWaitLimitNs;
+  k.extra_arrivals = extra_arrivals;
+  k.extra_tx = extra_tx;
+}
+
 extern "C" void pl_debug_timing(int enable) { g_timing = enable != 0; }
 
 extern "C" pl_status pl_debug_timing_read(double* ms, int64_t* launches) {

@@ -52,6 +52,7 @@ struct __align__(64) GemmParams {
   int total_tiles;
   unsigned* err;
   unsigned long long wait_ns;
+  unsigned extra_tx;       // test-only: extra bytes each stage expects (0 in normal use)
 };
 
 // Encodes a 2-D tensor map over a row-major [outer, inner] array of 16-bit

@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         const CUtensorMap* bmap = &p.maps[j.b_map];
         for (int k = 0; k < j.k_steps; ++k) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, lim)) break;
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          mbar_arrive_expect_tx(&full[stage], kStageBytes + p.extra_tx);
           uint8_t* a_dst = ring + stage * kStageBytes;
           uint8_t* b_dst = a_dst + kABytes;
           const int k0 = k * kBK;
@@ -228,6 +228,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             phase ^= 1;
           }
         }
+      }
+      if (*abort_flag) {
+        // Leave time for copies already issued to land before shared memory is released.
+        const unsigned long long t0 = globaltimer();
+        while (globaltimer() - t0 < 100000ull) __nanosleep(1000);
       }
     }
   } else if (warp == 1) {
@@ -376,8 +381,11 @@ void gemm_finalize_jobs(GemmParams* p) {
   p->total_tiles = begin;
 }
 
-cudaError_t launch_gemm(const GemmParams& p, DType dt, cudaStream_t stream) {
-  if (p.total_tiles <= 0) return cudaSuccess;
+cudaError_t launch_gemm(const GemmParams& p0, DType dt, cudaStream_t stream) {
+  if (p0.total_tiles <= 0) return cudaSuccess;
+  GemmParams p = p0;
+  p.wait_ns = debug_knobs().wait_ns;
+  p.extra_tx = debug_knobs().extra_tx;
   DevInfo di;
   cudaError_t e = dev_info(&di);
   if (e != cudaSuccess) return e;

@@ -54,11 +54,24 @@ struct LossArgs {
   int adv_lp_dtype;
   int need_rows;
   int64_t partial_offset;  // byte offset of the f64 block partials inside ws
+  unsigned long long wait_ns;
+  unsigned extra_arrivals;
 };
 
 // Launches the single-pass loss kernel; returns a CUDA error code.
 cudaError_t launch_loss(const LossArgs& a, DType dt, bool has_kl, bool has_grad, bool two_sided,
                         bool vec, cudaStream_t stream);
+
+// Test-only knobs (set through pl_debug_set_wait): the bound on device waits
+// and two ways to make a bounded wait run out on purpose -- extra grid-barrier
+// arrivals the loss kernel waits for, and extra bytes a GEMM pipeline stage
+// expects from its TMA loads.  Defaults: kWaitLimitNs, 0, 0.
+struct DebugKnobs {
+  unsigned long long wait_ns = kWaitLimitNs;
+  unsigned extra_arrivals = 0;
+  unsigned extra_tx = 0;
+};
+DebugKnobs& debug_knobs();
 
 // Launch bookkeeping: every kernel launch of the library is bracketed by
 // launch_begin/launch_end (kind: 0 GEMM, 1 loss kernel, 2 other).  Counts

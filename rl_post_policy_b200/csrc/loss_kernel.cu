@@ -156,8 +156,8 @@ __global__ void __launch_bounds__(kThreads) loss_kernel(LossArgs a) {
     __threadfence();
     atomicAdd(arrive, 1u);
     const unsigned long long start = globaltimer_ns();
-    while (ld_acquire_u32(arrive) < gridDim.x) {
-      if (globaltimer_ns() - start > kWaitLimitNs) {
+    while (ld_acquire_u32(arrive) < gridDim.x + a.extra_arrivals) {
+      if (globaltimer_ns() - start > a.wait_ns) {
         atomicOr(err, kDevErrTimeout);
         s_flag = 1;
         break;
@@ -299,6 +299,8 @@ cudaError_t launch_t(const LossArgs& a0, cudaStream_t stream) {
   if (chunk < 64) chunk = 64;
   grid = a.n > 0 ? (a.n + chunk - 1) / chunk : 1;
   a.chunk = chunk;
+  a.wait_ns = debug_knobs().wait_ns;
+  a.extra_arrivals = debug_knobs().extra_arrivals;
   void* args[] = {&a};
   launch_begin(1, stream);
   e = cudaLaunchCooperativeKernel((const void*)kern, dim3((unsigned)grid), dim3(kThreads), args, 0, stream);
