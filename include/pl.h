@@ -129,6 +129,32 @@ pl_status pl_loss_ex(const void* policy_lp, const void* old_lp, const void* ref_
 
 size_t pl_loss_workspace_bytes(int64_t bs, int64_t seq);
 
+/* pl_loss_static: pl_loss_ex for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it exists because some
+ * callers must not call cudaMalloc on this path -- for example a process that
+ * reserved all free device memory for its own pool at start-up, or code that
+ * must not risk the device-wide synchronisation an allocation can cause -- and
+ * pl_loss allocates its scratch on first use while pl_loss_ex needs a buffer.
+ *
+ * Here the kernel's scratch is a fixed 64.25 KB array inside libpl.so's device
+ * image (held on every GPU that loads the library until the process exits), so
+ * the call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * routine.  Limits: bs <= 4096; a larger bs returns PL_ERR_WORKSPACE before
+ * any launch.  All other arguments are those of pl_loss_ex.
+ *   status_out : optional device uint32; receives this call's device error bits
+ *                (0 = none, 1 = a bounded wait ran out) and clears them.  With
+ *                NULL, the bits accumulate until a call passes status_out.
+ * The first call on each device looks up the array's device address (with that
+ * device current), so make it before any stream capture.  Every call shares the
+ * one array and resets the counters it needs on `stream` before its kernel:
+ * calls whose work overlaps on the GPU race, so order them on one stream.
+ */
+pl_status pl_loss_static(const void* policy_lp, const void* old_lp, const void* ref_lp,
+                         const void* adv, const uint8_t* mask, int64_t bs, int64_t seq,
+                         float eps_lo, float eps_hi, float beta, uint32_t mode,
+                         float* loss_out, void* grad_out, int64_t* n_valid_out,
+                         int64_t* row_valid_out, uint32_t* status_out, pl_stream_t stream);
+
 /* ---- fused linear path ----------------------------------------------------------
  * pl_fused_linear_grpo: for the N = bs*T rows (sequence-major),
  *   z      = X W^T (+ bias),  logp = z[target] - logsumexp(z)        (policy)

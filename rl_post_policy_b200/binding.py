@@ -43,6 +43,9 @@ _lib.pl_loss.restype = _I
 _lib.pl_loss_ex.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _F, _F, _F, _U32, _P, _P, _P, _P, _P,
                             _SZ, _P]
 _lib.pl_loss_ex.restype = _I
+_lib.pl_loss_static.argtypes = [_P, _P, _P, _P, _P, _I64, _I64, _F, _F, _F, _U32, _P, _P, _P, _P, _P,
+                                _P]
+_lib.pl_loss_static.restype = _I
 _lib.pl_loss_workspace_bytes.argtypes = [_I64, _I64]
 _lib.pl_loss_workspace_bytes.restype = _SZ
 _lib.pl_fused_linear_grpo.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64,
@@ -67,7 +70,7 @@ _lib.pl_debug_set_wait.restype = None
 _lib.pl_debug_launch_count.argtypes = []
 _lib.pl_debug_launch_count.restype = _I64
 
-EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
+EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_static", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
             "pl_version", "pl_debug_gemm", "pl_debug_timing", "pl_debug_timing_read",
             "pl_debug_launch_count", "pl_debug_set_wait")
@@ -120,6 +123,15 @@ def pl_loss_ex(policy_lp, old_lp, ref_lp, adv, mask, bs, seq, eps_lo, eps_hi, be
                            seq, eps_lo, eps_hi, beta, mode, _ptr(loss_out), _ptr(grad_out),
                            _ptr(n_valid_out), _ptr(row_valid_out), _ptr(workspace), ws_bytes,
                            _stream(stream))
+
+
+def pl_loss_static(policy_lp, old_lp, ref_lp, adv, mask, bs, seq, eps_lo, eps_hi, beta, mode,
+                   loss_out, grad_out, n_valid_out, row_valid_out, status_out, stream=None) -> int:
+    """Allocation-free pl_loss_ex: scratch in a fixed array of libpl.so (bs <= 4096)."""
+    return _lib.pl_loss_static(_ptr(policy_lp), _ptr(old_lp), _ptr(ref_lp), _ptr(adv), _ptr(mask), bs,
+                               seq, eps_lo, eps_hi, beta, mode, _ptr(loss_out), _ptr(grad_out),
+                               _ptr(n_valid_out), _ptr(row_valid_out), _ptr(status_out),
+                               _stream(stream))
 
 
 def pl_loss_workspace_bytes(bs, seq) -> int:

@@ -58,6 +58,18 @@ struct LossArgs {
   unsigned extra_arrivals;
 };
 
+// Argument checks shared by the loss entry points (no device call); sets *dt.
+pl_status validate_loss(const void* lp, const void* old, const void* ref, const void* adv,
+                        const uint8_t* mask, int64_t bs, int64_t seq, float eps_lo, float eps_hi,
+                        float beta, uint32_t mode, float* loss_out, DType* dt);
+
+// Fills LossArgs and launches the loss kernel on `ws` (a zero-initialised
+// loss workspace of at least loss_ws_bytes(bs) bytes).
+pl_status run_loss(const void* lp, const void* old, const void* ref, const void* adv,
+                   const uint8_t* mask, int64_t bs, int64_t seq, float eps_lo, float eps_hi,
+                   float beta, uint32_t mode, DType dt, float* loss_out, void* grad_out,
+                   int64_t* n_valid_out, int64_t* row_valid_out, void* ws, cudaStream_t stream);
+
 // Launches the single-pass loss kernel; returns a CUDA error code.
 cudaError_t launch_loss(const LossArgs& a, DType dt, bool has_kl, bool has_grad, bool two_sided,
                         bool vec, cudaStream_t stream);

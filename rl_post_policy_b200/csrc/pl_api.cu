@@ -83,7 +83,9 @@ bool finite_nonneg(float x) { return std::isfinite(x) && x >= 0.0f; }
 
 constexpr uint32_t kLossModeBits = PL_REDUCTION_MASK | PL_DTYPE_MASK | PL_ADV_LP_DTYPE | PL_CLIP_TWO_SIDED;
 
-// Host-side validation shared by pl_loss and pl_loss_ex (no device call).
+}  // namespace
+
+// Host-side validation shared by the loss entry points (no device call).
 pl_status validate_loss(const void* lp, const void* old, const void* ref, const void* adv,
                         const uint8_t* mask, int64_t bs, int64_t seq, float eps_lo, float eps_hi,
                         float beta, uint32_t mode, float* loss_out, DType* dt) {
@@ -135,7 +137,6 @@ pl_status run_loss(const void* lp, const void* old, const void* ref, const void*
   return e == cudaSuccess ? PL_OK : PL_ERR_CUDA;
 }
 
-}  // namespace
 }  // namespace pl
 
 using namespace pl;
