@@ -46,13 +46,14 @@ LOSS_SOURCES = ["rl_post_policy_b200/csrc/loss_kernel.cu", "rl_post_policy_b200/
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5])
     ap.add_argument("--no-loss-only", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=64, help="rows in the oracle's timed sample")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="rows in the oracle's timed sample")
+    ap.add_argument("--ref-rows", type=int, default=4, help="rows per step of the reference (oracle) arm")
     return ap.parse_args()
 
 
@@ -71,14 +72,18 @@ def sources_sha(paths) -> str:
 
 
 def recorded_traffic(kernel: str, paths):
-    """Per-launch DRAM bytes from an ncu capture, if taken on the current sources."""
-    f = ROOT / "profiles" / "traffic.json"
+    """Per-launch DRAM bytes (read + write) from an ncu capture, taken from
+    profiles/traffic.txt lines `<kernel> <sources sha> <bytes per launch>`,
+    and only if the capture was taken on the current sources."""
+    f = ROOT / "profiles" / "traffic.txt"
     if not f.exists():
         return None
-    d = json.loads(f.read_text()).get(kernel)
-    if not d or d.get("sources_sha") != sources_sha(paths):
-        return None
-    return d.get("bytes_per_launch")
+    sha = sources_sha(paths)
+    for line in f.read_text().splitlines():
+        parts = line.split()
+        if len(parts) == 3 and parts[0] == kernel and parts[1] == sha:
+            return float(parts[2])
+    return None
 
 
 # ------------------------------------------------------------------ distributed
@@ -124,7 +129,9 @@ def sum_over_ranks(x: float, ws: int) -> float:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling every 100 ms; stop() keeps the samples whose
+    timestamps fall inside the timed window (mark_start / mark_end)."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -136,8 +143,15 @@ class ClockSampler:
         except Exception:
             self.sel = None
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def start(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        self.t0 = self.t1 = None
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
         if self.sel:
             cmd += ["-i", self.sel]
         try:
@@ -154,11 +168,19 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, mx, reasons = [], None, set()
+        import datetime
+        sm, mx, reasons, total = [], None, set(), 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
+                continue
+            total += 1
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            if self.t0 is not None and ts is not None and not (self.t0 <= ts <= (self.t1 or ts)):
                 continue
             try:
                 sm.append(float(f[1]))
@@ -170,7 +192,7 @@ class ClockSampler:
                     reasons.add(n)
         load = [x for x in sm if mx and x > 0.3 * mx] or sm
         return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "samples_total": total}
 
 
 # ------------------------------------------------------------------ workload
@@ -321,7 +343,7 @@ def run_reference(args):
     import oracle  # noqa: F401
     # Inputs: the same recipe, generated on the CPU (no GPU work on this arm).
     import synth
-    rows = max(1, min(args.cpu_rows // 4, d["N"]))
+    rows = max(1, min(args.ref_rows, d["N"]))
     inp = synth.fused_inputs(1, rows, d["H"], d["V"], d["dtype"], synth.seed_for(args.workload),
                              bias=d.get("bias", False), len_lo=rows, len_hi=rows)
     import oracle as orc
@@ -365,8 +387,13 @@ def run_ours(args):
     pl.pl_debug_timing_read()
     launches0 = pl.pl_debug_launch_count()
     clocks.start()
+    for _ in range(max(1, args.warmup)):  # keep the GPU busy while the sampler starts
+        step()
+    time.sleep(0.3)
     pl.pl_debug_timing(True)
+    clocks.mark_start()
     elapsed = time_steps(step, args.steps, ws_world)
+    clocks.mark_end()
     pl.pl_debug_timing(False)
     clk = clocks.stop()
     launches = pl.pl_debug_launch_count() - launches0

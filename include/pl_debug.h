@@ -50,6 +50,14 @@ pl_status pl_debug_timing_read(double* ms, int64_t* launches);
  */
 void pl_debug_set_wait(unsigned long long wait_ns, unsigned extra_arrivals, unsigned extra_tx);
 
+/*
+ * The persistent GEMM's tile schedule, for a host-side check: two problems of
+ * t0 tiles (c0 k-steps each) and t1 tiles (c1 k-steps each) over `pairs` CTA
+ * pairs.  out_pair[t] (t0 + t1 entries) receives the pair that runs tile t.
+ * Returns 0, or -1 when some tile would run on no pair or on two.
+ */
+int pl_debug_pair_tiles(int t0, int t1, int c0, int c1, int pairs, int32_t* out_pair);
+
 /* Number of kernels this library has launched in this process. */
 int64_t pl_debug_launch_count(void);
 

@@ -23,8 +23,9 @@
 // Everything is fp64.  Low-precision inputs (binary16, bfloat16, binary32) are
 // decoded exactly by the decoders below, written from the IEEE-754 / bfloat16
 // bit-layout definitions.  Contractions are plain sums taken in natural index
-// order; the only concession to speed is that several rows share one pass over
-// a weight row (each sum is still its own accumulator, in the same h order).
+// order; the only concession to speed is that 32 rows share one pass over a
+// weight row, their 32 sums held in vector registers (each sum is still its own
+// accumulator, taken in the same h order).
 //
 // Readings of points the pages leave open (each also listed in the design notes):
 //   * clip bounds mirror fp32 arguments: lo = (double)(1.0f - eps_lo),
@@ -82,6 +83,18 @@ double load(int dt, const void* p, int64_t i) {
   return NAN;
 }
 
+// dst[i] = exact value of element (off + i) for i < n; the dtype switch is
+// taken once per row rather than once per element.
+void load_row(int dt, const void* p, int64_t off, int64_t n, double* dst) {
+  switch (dt) {
+    case DT_F64: for (int64_t i = 0; i < n; ++i) dst[i] = ((const double*)p)[off + i]; break;
+    case DT_F32: for (int64_t i = 0; i < n; ++i) dst[i] = (double)((const float*)p)[off + i]; break;
+    case DT_F16: for (int64_t i = 0; i < n; ++i) dst[i] = decode_f16(((const uint16_t*)p)[off + i]); break;
+    case DT_BF16: for (int64_t i = 0; i < n; ++i) dst[i] = decode_bf16(((const uint16_t*)p)[off + i]); break;
+    default: for (int64_t i = 0; i < n; ++i) dst[i] = NAN;
+  }
+}
+
 int worker_count(int requested) {
   if (requested > 0) return requested;
   cpu_set_t set;
@@ -91,6 +104,40 @@ int worker_count(int requested) {
   }
   unsigned n = std::thread::hardware_concurrency();
   return n ? (int)n : 1;
+}
+
+// acc[r] = sum over h (in order h = 0..H-1) of xT[h*32 + r] * w[h], for the 32
+// rows of a group: the same per-row sums as 32 separate dot products, written
+// with four-wide vector registers so the accumulators stay in registers.
+typedef double v4d __attribute__((vector_size(32), aligned(8)));
+void dot32(const double* xT, const double* w, int64_t H, double* acc) {
+  v4d a0 = {0, 0, 0, 0}, a1 = a0, a2 = a0, a3 = a0, a4 = a0, a5 = a0, a6 = a0, a7 = a0;
+  for (int64_t h = 0; h < H; ++h) {
+    const v4d wv = {w[h], w[h], w[h], w[h]};
+    const v4d* x = reinterpret_cast<const v4d*>(xT + h * 32);
+    a0 += x[0] * wv;
+    a1 += x[1] * wv;
+    a2 += x[2] * wv;
+    a3 += x[3] * wv;
+    a4 += x[4] * wv;
+    a5 += x[5] * wv;
+    a6 += x[6] * wv;
+    a7 += x[7] * wv;
+  }
+  const v4d* all[8] = {&a0, &a1, &a2, &a3, &a4, &a5, &a6, &a7};
+  for (int q = 0; q < 8; ++q)
+    for (int j = 0; j < 4; ++j) acc[4 * q + j] = (*all[q])[j];
+}
+
+// The same for a group of at most 4 rows (xT holds 32 slots per h; only the
+// first 4 are read), so small groups do not pay for 32.
+void dot4(const double* xT, const double* w, int64_t H, double* acc) {
+  v4d a0 = {0, 0, 0, 0};
+  for (int64_t h = 0; h < H; ++h) {
+    const v4d wv = {w[h], w[h], w[h], w[h]};
+    a0 += *reinterpret_cast<const v4d*>(xT + h * 32) * wv;
+  }
+  for (int j = 0; j < 4; ++j) acc[j] = a0[j];
 }
 
 // Runs fn(worker, begin, end) over [0, n) split into contiguous ranges.
@@ -244,13 +291,8 @@ int orc_lm_head_logprob(const void* X, int xdt, const void* W, int wdt,
       std::vector<double> w(H);
       double acc[32];
       for (int64_t v = vb; v < ve; ++v) {
-        for (int64_t h = 0; h < H; ++h) w[h] = load(wdt, W, v * H + h);
-        for (int r = 0; r < R; ++r) acc[r] = 0.0;
-        for (int64_t h = 0; h < H; ++h) {
-          const double wh = w[h];
-          const double* xr = &xT[(size_t)h * R];
-          for (int r = 0; r < R; ++r) acc[r] += xr[r] * wh;
-        }
+        load_row(wdt, W, v * H, H, w.data());
+        if (gr <= 4) dot4(xT.data(), w.data(), H, acc); else dot32(xT.data(), w.data(), H, acc);
         const double b = bias ? load(bdt, bias, v) : 0.0;
         for (int r = 0; r < gr; ++r) z[(size_t)r * V + v] = acc[r] + b;
       }
@@ -310,13 +352,8 @@ int orc_lm_head_backward(const void* X, int xdt, const void* W, int wdt,
         double acc[32];
         std::vector<double>& dxp = part[wk];
         for (int64_t v = vb; v < ve; ++v) {
-          for (int64_t h = 0; h < H; ++h) w[h] = load(wdt, W, v * H + h);
-          for (int r = 0; r < R; ++r) acc[r] = 0.0;
-          for (int64_t h = 0; h < H; ++h) {
-            const double wh = w[h];
-            const double* xr = &xT[(size_t)h * R];
-            for (int r = 0; r < R; ++r) acc[r] += xr[r] * wh;
-          }
+          load_row(wdt, W, v * H, H, w.data());
+          if (gr <= 4) dot4(xT.data(), w.data(), H, acc); else dot32(xT.data(), w.data(), H, acc);
           const double b = bias ? load(bdt, bias, v) : 0.0;
           for (int r = 0; r < gr; ++r) {
             const int64_t i = idx[r];
@@ -338,30 +375,41 @@ int orc_lm_head_backward(const void* X, int xdt, const void* W, int wdt,
   }
 
   // ---- dW / dbias rows: one vocab row at a time, all N rows --------------
+  // z[i, v] for all rows i comes from the same 32-row group dot products as the
+  // forward (each z still summed over h in order).
   if (n_dw > 0) {
     if (!dw_rows || !dW_out) return 1;
     std::vector<double> Xd((size_t)N * H);
-    for (int64_t i = 0; i < N * H; ++i) Xd[i] = load(xdt, X, i);
+    for (int64_t i = 0; i < N; ++i) load_row(xdt, X, i * H, H, &Xd[(size_t)i * H]);
+    const int64_t ng = (N + 31) / 32;
+    std::vector<double> XT((size_t)ng * H * 32, 0.0);
+    for (int64_t i = 0; i < N; ++i)
+      for (int64_t h = 0; h < H; ++h) XT[(size_t)(i / 32) * H * 32 + (size_t)h * 32 + (i % 32)] = Xd[(size_t)i * H + h];
     for (int64_t k = 0; k < n_dw; ++k)
       if (dw_rows[k] < 0 || dw_rows[k] >= V) return 1;
     parallel_ranges(n_dw, workers, [&](int, int64_t kb, int64_t ke) {
       std::vector<double> w(H);
+      double acc[32];
       for (int64_t k = kb; k < ke; ++k) {
         const int64_t v = dw_rows[k];
-        for (int64_t h = 0; h < H; ++h) w[h] = load(wdt, W, v * H + h);
+        load_row(wdt, W, v * H, H, w.data());
         const double b = bias ? load(bdt, bias, v) : 0.0;
         double* out = &dW_out[k * H];
         for (int64_t h = 0; h < H; ++h) out[h] = 0.0;
         double db = 0.0;
-        for (int64_t i = 0; i < N; ++i) {
-          if (g[i] == 0.0) continue;                 // dz row is exactly zero
-          const double* xi = &Xd[(size_t)i * H];
-          double zi = 0.0;
-          for (int64_t h = 0; h < H; ++h) zi += xi[h] * w[h];
-          zi += b;
-          const double dz = g[i] * ((v == targets[i] ? 1.0 : 0.0) - std::exp(zi - lse[i]));
-          for (int64_t h = 0; h < H; ++h) out[h] += dz * xi[h];
-          db += dz;
+        for (int64_t gi = 0; gi < ng; ++gi) {
+          const int gr = (int)std::min<int64_t>(32, N - gi * 32);
+          const double* xg = &XT[(size_t)gi * H * 32];
+          if (gr <= 4) dot4(xg, w.data(), H, acc); else dot32(xg, w.data(), H, acc);
+          for (int r = 0; r < gr; ++r) {
+            const int64_t i = gi * 32 + r;
+            if (g[i] == 0.0) continue;               // dz row is exactly zero
+            const double zi = acc[r] + b;
+            const double dz = g[i] * ((v == targets[i] ? 1.0 : 0.0) - std::exp(zi - lse[i]));
+            const double* xi = &Xd[(size_t)i * H];
+            for (int64_t h = 0; h < H; ++h) out[h] += dz * xi[h];
+            db += dz;
+          }
         }
         if (dbias_out) dbias_out[k] = db;
       }

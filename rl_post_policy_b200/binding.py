@@ -67,13 +67,15 @@ _lib.pl_debug_timing_read.argtypes = [_P, _P]
 _lib.pl_debug_timing_read.restype = _I
 _lib.pl_debug_set_wait.argtypes = [ctypes.c_ulonglong, ctypes.c_uint, ctypes.c_uint]
 _lib.pl_debug_set_wait.restype = None
+_lib.pl_debug_pair_tiles.argtypes = [_I, _I, _I, _I, _I, _P]
+_lib.pl_debug_pair_tiles.restype = _I
 _lib.pl_debug_launch_count.argtypes = []
 _lib.pl_debug_launch_count.restype = _I64
 
 EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_static", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
             "pl_version", "pl_debug_gemm", "pl_debug_timing", "pl_debug_timing_read",
-            "pl_debug_launch_count", "pl_debug_set_wait")
+            "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_pair_tiles")
 
 
 class PLError(RuntimeError):
@@ -190,3 +192,10 @@ def pl_debug_launch_count() -> int:
 def pl_debug_set_wait(wait_ns: int, extra_arrivals: int = 0, extra_tx: int = 0) -> None:
     """Test knob (include/pl_debug.h): wait bound and wait-run-out injection."""
     _lib.pl_debug_set_wait(int(wait_ns), int(extra_arrivals), int(extra_tx))
+
+
+def pl_debug_pair_tiles(t0: int, t1: int, c0: int, c1: int, pairs: int):
+    """Test hook: (status, [pair running tile t for each t]) of the GEMM tile schedule."""
+    out = (ctypes.c_int32 * max(t0 + t1, 1))()
+    rc = _lib.pl_debug_pair_tiles(t0, t1, c0, c1, pairs, out)
+    return int(rc), list(out)[: t0 + t1]

@@ -26,7 +26,7 @@ extern "C" pl_status pl_debug_gemm(const void* A, int a_mn, int64_t lda, const v
   bool ok = a_mn ? make_tmap_2d(&p.maps[0], A, dt, M, K, lda * 2, 64, kBK)
                  : make_tmap_2d(&p.maps[0], A, dt, K, M, lda * 2, kBK, kBM);
   ok = ok && (b_mn ? make_tmap_2d(&p.maps[1], B, dt, N, K, ldb * 2, 64, kBK)
-                   : make_tmap_2d(&p.maps[1], B, dt, K, N, ldb * 2, kBK, kBN));
+                   : make_tmap_2d(&p.maps[1], B, dt, K, N, ldb * 2, kBK, kBNh));
   if (!ok) return PL_ERR_CUDA;
   GemmJob& j = p.jobs[0];
   j.a_map = 0; j.b_map = 1; j.a_mn = a_mn ? 1 : 0; j.b_mn = b_mn ? 1 : 0;
@@ -35,6 +35,32 @@ extern "C" pl_status pl_debug_gemm(const void* A, int a_mn, int64_t lda, const v
   p.njobs = 1;
   gemm_finalize_jobs(&p);
   return launch_gemm(p, dt, s) == cudaSuccess ? PL_OK : PL_ERR_CUDA;
+}
+
+// pl_debug_pair_tiles: the GEMM's tile schedule for two jobs (t0 tiles of c0
+// k-steps, then t1 tiles of c1 k-steps) over `pairs` CTA pairs.  Writes, for
+// every tile, the pair that runs it (out_pair[t0 + t1]) and returns 0, or -1 if
+// a tile is given to no pair or to two.
+extern "C" int pl_debug_pair_tiles(int t0, int t1, int c0, int c1, int pairs, int32_t* out_pair) {
+  if (t0 < 0 || t1 < 0 || pairs < 1 || !out_pair) return -1;
+  GemmParams p{};
+  p.njobs = 2;
+  p.jobs[0].tiles_m = t0; p.jobs[0].tiles_n = 1; p.jobs[0].k_steps = c0; p.jobs[0].tile_begin = 0;
+  p.jobs[1].tiles_m = t1; p.jobs[1].tiles_n = 1; p.jobs[1].k_steps = c1; p.jobs[1].tile_begin = t0;
+  p.total_tiles = t0 + t1;
+  balance_schedule(&p, pairs);
+  for (int t = 0; t < t0 + t1; ++t) out_pair[t] = -1;
+  for (int q = 0; q < pairs; ++q) {
+    for (int i = 0;; ++i) {
+      const int t = pair_tile(p, q, pairs, i);
+      if (t < 0) break;
+      if (t >= t0 + t1 || out_pair[t] != -1) return -1;
+      out_pair[t] = q;
+    }
+  }
+  for (int t = 0; t < t0 + t1; ++t)
+    if (out_pair[t] < 0) return -1;
+  return 0;
 }
 
 // ---------------------------------------------------------------- launch bookkeeping

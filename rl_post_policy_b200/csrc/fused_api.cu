@@ -157,7 +157,7 @@ pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias, c
     int nj = 0;
     if (has_kl) {
       if (!make_tmap_2d(&fp.maps[0], Xrb + r0 * H * esz, dt, H, rows, H * esz, kBK, kBM) ||
-          !make_tmap_2d(&fp.maps[1], Wref, dt, H, V, H * esz, kBK, kBN))
+          !make_tmap_2d(&fp.maps[1], Wref, dt, H, V, H * esz, kBK, kBNh))
         return PL_ERR_CUDA;
       GemmJob& j = fp.jobs[nj++];
       j.a_map = 0; j.b_map = 1; j.a_mn = 0; j.b_mn = 0;
@@ -167,7 +167,7 @@ pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias, c
       j.zt = reinterpret_cast<float*>(ws + plan.off.zt_ref); j.logits = nullptr;
     }
     if (!make_tmap_2d(&fp.maps[2], Xb + r0 * H * esz, dt, H, rows, H * esz, kBK, kBM) ||
-        !make_tmap_2d(&fp.maps[3], W, dt, H, V, H * esz, kBK, kBN))
+        !make_tmap_2d(&fp.maps[3], W, dt, H, V, H * esz, kBK, kBNh))
       return PL_ERR_CUDA;
     {
       GemmJob& j = fp.jobs[nj++];

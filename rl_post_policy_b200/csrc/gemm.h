@@ -8,10 +8,15 @@
 
 namespace pl {
 
-constexpr int kBM = 128;       // tile rows (tensor-memory lanes)
+// A CTA pair (a cluster of two CTAs on two SMs) owns one kPairM x kBN output
+// tile: each CTA holds kBM rows of A, kBNh rows of B and kBM x kBN fp32
+// accumulators in its tensor memory; the pair leader issues M=256 MMAs.
+constexpr int kBM = 128;       // rows per CTA (tensor-memory lanes)
+constexpr int kPairM = 256;    // rows per CTA pair (the MMA's M)
 constexpr int kBN = 256;       // tile columns (tensor-memory columns per accumulator)
+constexpr int kBNh = 128;      // B rows (N) held by each CTA of the pair
 constexpr int kBK = 64;        // K per pipeline stage (one 128-byte swizzle row)
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
 
 enum EpiKind : int {
@@ -19,7 +24,7 @@ enum EpiKind : int {
   kEpiStore = 1,  // acc * scale (+ fp32 acc_in) -> out (model dtype or fp32)
 };
 
-// One GEMM problem D[M,N] = sum_k A(m,k) B(n,k), tiled kBM x kBN.
+// One GEMM problem D[M,N] = sum_k A(m,k) B(n,k), tiled kPairM x kBN.
 //   A(m,k): K-major means A[m*lda + k]; MN-major means A[k*lda + m] (likewise B).
 struct GemmJob {
   int a_map, b_map;        // tensor-map indices in GemmParams::maps
@@ -50,11 +55,19 @@ struct __align__(64) GemmParams {
   GemmJob jobs[2];
   int njobs;
   int total_tiles;
+  // Tile schedule (set by launch_gemm).  0: pair p takes tiles p, p+P, p+2P ...
+  // 1: two jobs of very different tile cost -- pair p < T0 takes job-0 tile p,
+  //    then every pair takes a contiguous run of job-1 tiles, `na` (p < T0) or
+  //    `nb` long plus one for the first `rem` pairs, so that all pairs carry
+  //    about the same number of k-steps.
+  int sched, na, nb, rem;
   unsigned* err;
   unsigned long long wait_ns;
   unsigned extra_tx;       // test-only: extra bytes each stage expects (0 in normal use)
 };
 
+// Tensor-map boxes: K-major operands load {kBK, kBM} (A) or {kBK, kBNh} (B)
+// boxes; MN-major operands load {64, kBK} boxes, two per 128 rows/columns.
 // Encodes a 2-D tensor map over a row-major [outer, inner] array of 16-bit
 // elements with a row pitch of `pitch_bytes`, box {box_inner, box_outer},
 // 128-byte swizzle, zero fill outside the extent.
@@ -65,5 +78,10 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, 
 void gemm_finalize_jobs(GemmParams* p);
 
 cudaError_t launch_gemm(const GemmParams& p, DType dt, cudaStream_t stream);
+
+// Tile schedule (host side of what the kernel runs): balance_schedule fills
+// sched/na/nb/rem for P pairs; pair_tile gives the i-th tile of a pair or -1.
+void balance_schedule(GemmParams* p, int P);
+__host__ __device__ int pair_tile(const GemmParams& p, int pair, int npairs, int i);
 
 }  // namespace pl

@@ -1,16 +1,25 @@
 // Persistent tcgen05 GEMM for sm_100a with the epilogues of the fused path.
 //
-// Each CTA owns one SM (grid = min(tiles, SMs)) and walks the concatenated tile
-// list of up to two GEMM problems in a static round-robin.  Roles:
-//   warp 0    one elected lane issues TMA tile loads (128-byte swizzle) into a
-//             4-stage shared-memory ring (48 KB per stage);
-//   warp 1    allocates 512 tensor-memory columns (two 128x256 fp32
-//             accumulators) and one elected lane issues tcgen05.mma
-//             (M=128, N=256, K=16, bf16/fp16 -> fp32), committing each stage
-//             back to the producer and each finished tile to the epilogue;
+// CTAs run in pairs (clusters of two, one CTA per SM); a pair owns a 256 x 256
+// output tile and the grid holds as many pairs as can be resident, each
+// walking the concatenated tile list of up to two GEMM problems round-robin.
+// Per CTA:
+//   warp 0    one lane issues TMA tile loads (128-byte swizzle, no multicast)
+//             of this CTA's 128 rows of A and 128 rows (of the tile's 256
+//             columns) of B into a 6-stage ring (32 KB per stage); the pair
+//             leader's mbarrier counts both CTAs' bytes;
+//   warp 1    allocates 512 tensor-memory columns (two 128 x 256 fp32
+//             accumulators, cta_group::2); in the leader one lane issues
+//             tcgen05.mma.cta_group::2 (M=256, N=256, K=16), which reads the A
+//             and B halves from both CTAs' shared memory and writes each CTA's
+//             128 accumulator rows into its own tensor memory, and commits each
+//             stage back to both producers and each tile to both epilogues;
 //   warps 2-5 the epilogue: one accumulator row per thread (tcgen05.ld
 //             32x32b), 32 columns at a time, overlapping the next tile's
-//             mainloop thanks to the second accumulator.
+//             mainloop thanks to the second accumulator; both CTAs release the
+//             accumulator on the leader's barrier.
+// Splitting B across the pair halves each SM's shared-memory operand traffic
+// compared with one CTA computing a 128 x 256 tile alone.
 // Operands may be K-major or MN-major (the backward GEMMs read the logits
 // workspace and the weights transposed without copying them).
 //
@@ -24,8 +33,9 @@
 //                or in fp32 (dX; dW / dbias with fp32 accumulation across chunks).
 //
 // Every wait is bounded (GemmParams::wait_ns); when one runs out the CTA sets a
-// shared abort flag, every role drains out, tensor memory is released and the
-// sticky device error flag is raised.
+// shared abort flag, every role drains out, the leader waits (bounded) for its
+// issued MMAs, tensor memory is released and the sticky device error flag is
+// raised.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -37,9 +47,9 @@ namespace {
 
 using namespace sm100;
 
-constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB
-constexpr uint32_t kBBytes = kBN * kBK * 2;             // 32 KB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 48 KB
+constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB: this CTA's 128 rows of A
+constexpr uint32_t kBBytes = kBNh * kBK * 2;            // 16 KB: this CTA's 128 rows of B
+constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 32 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr size_t kGemmSmem = 1024 + kStages * kStageBytes + 256;
 
@@ -83,6 +93,30 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmParams& p, int tile) {
   }
   return c;
 }
+
+}  // namespace
+
+// Global tile id of the i-th tile of `pair`, or -1 once the pair is done.
+__host__ __device__ int pair_tile(const GemmParams& p, int pair, int npairs, int i) {
+  if (p.sched == 0) {
+    const int t = pair + i * npairs;
+    return t < p.total_tiles ? t : -1;
+  }
+  const int T0 = p.jobs[1].tile_begin;
+  int k = i;
+  if (pair < T0) {
+    if (k == 0) return pair;
+    k -= 1;
+  }
+  const int cnt = (pair < T0 ? p.na : p.nb) + (pair < p.rem ? 1 : 0);
+  if (k >= cnt) return -1;
+  const int lo = pair < T0 ? pair : T0;
+  const int hi = pair > T0 ? pair - T0 : 0;
+  const int rm = pair < p.rem ? pair : p.rem;
+  return T0 + lo * p.na + hi * p.nb + rm + k;
+}
+
+namespace {
 
 // Stores 32 consecutive values (or the first `nvalid`) of one row.
 template <typename T>
@@ -162,11 +196,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: pair leader (issues the MMAs), 1: peer
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -175,8 +214,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+      mbar_init(&tempty[b], 2 * 128);  // both CTAs' epilogue threads release the leader's accumulator
     }
+    mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
     for (int q = 0; q < p.njobs; ++q) {
@@ -185,43 +225,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // the peer's barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const unsigned long long lim = p.wait_ns;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (both CTAs; completions counted by the leader) ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < p.total_tiles && !*abort_flag; tile += gridDim.x) {
+      for (int it = 0; !*abort_flag; ++it) {
+        const int tile = pair_tile(p, pair, npairs, it);
+        if (tile < 0) break;
         const TileCoord tc = tile_coord(p, tile);
         const GemmJob& j = p.jobs[tc.job];
-        const int m0 = tc.mb * kBM, n0 = tc.nb * kBN;
+        const int m0 = tc.mb * kPairM + (int)rank * kBM;
+        const int n0 = tc.nb * kBN + (int)rank * kBNh;
         const CUtensorMap* amap = &p.maps[j.a_map];
         const CUtensorMap* bmap = &p.maps[j.b_map];
         for (int k = 0; k < j.k_steps; ++k) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, lim)) break;
-          mbar_arrive_expect_tx(&full[stage], kStageBytes + p.extra_tx);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes + p.extra_tx);
+          const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = ring + stage * kStageBytes;
           uint8_t* b_dst = a_dst + kABytes;
           const int k0 = k * kBK;
           if (!j.a_mn) {
-            tma_load_2d(a_dst, amap, &full[stage], k0, m0);
+            tma_load_2d_pair(a_dst, amap, bar, k0, m0);
           } else {
-            tma_load_2d(a_dst, amap, &full[stage], m0, k0);
-            tma_load_2d(a_dst + 8192, amap, &full[stage], m0 + 64, k0);
+            tma_load_2d_pair(a_dst, amap, bar, m0, k0);
+            tma_load_2d_pair(a_dst + 8192, amap, bar, m0 + 64, k0);
           }
           if (!j.b_mn) {
-            tma_load_2d(b_dst, bmap, &full[stage], k0, n0);
+            tma_load_2d_pair(b_dst, bmap, bar, k0, n0);
           } else {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) tma_load_2d(b_dst + q * 8192, bmap, &full[stage], n0 + 64 * q, k0);
+            tma_load_2d_pair(b_dst, bmap, bar, n0, k0);
+            tma_load_2d_pair(b_dst + 8192, bmap, bar, n0 + 64, k0);
           }
           if (++stage == kStages) {
             stage = 0;
@@ -236,20 +281,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+    // ---------------- MMA issuer (leader CTA only) ----------------
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       const uint32_t ring_addr = smem_u32(ring);
-      for (int tile = blockIdx.x; tile < p.total_tiles && !*abort_flag; tile += gridDim.x) {
+      for (int it = 0; !*abort_flag; ++it) {
+        const int tile = pair_tile(p, pair, npairs, it);
+        if (tile < 0) break;
         const TileCoord tc = tile_coord(p, tile);
         const GemmJob& j = p.jobs[tc.job];
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, lim)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kBN;
-        const uint32_t idesc = instr_desc_f16(AbFormat<T>::v, j.a_mn, j.b_mn, kBM, kBN);
+        const uint32_t idesc = instr_desc_f16(AbFormat<T>::v, j.a_mn, j.b_mn, kPairM, kBN);
         bool ok = true;
         for (int k = 0; k < j.k_steps; ++k) {
           if (!mbar_wait(&full[stage], phase, abort_flag, lim)) { ok = false; break; }
@@ -262,35 +309,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                                        : smem_desc(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = j.b_mn ? smem_desc(b_addr + kk * 2048, 8192, 1024)
                                        : smem_desc(b_addr + kk * 32, 16, 1024);
-            mma_f16_ss(d_tmem, ad, bd, idesc, (k | kk) != 0 ? 1u : 0u);
+            mma_f16_ss_pair(d_tmem, ad, bd, idesc, (k | kk) != 0 ? 1u : 0u);
           }
-          mma_commit(&empty[stage]);
+          mma_commit_pair(&empty[stage], 0x3);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        mma_commit(&tfull[acc]);
+        mma_commit_pair(&tfull[acc], 0x3);
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
         }
       }
+      // Every MMA this thread issued has completed before tensor memory is released.
+      mma_commit_pair(done, 0x1);
+      volatile int no_abort = 0;
+      mbar_wait(done, 0, &no_abort, lim);
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..5, both CTAs) ----------------
     const int quarter = warp & 3;  // tensor-memory lanes [32*quarter, 32*quarter+32)
     const int r_local = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     constexpr float kLog2e = 1.4426950408889634f;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+    for (int it = 0;; ++it) {
+      const int tile = pair_tile(p, pair, npairs, it);
+      if (tile < 0) break;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, lim)) break;
       tc_fence_after();
       const TileCoord tc = tile_coord(p, tile);
       const GemmJob& j = p.jobs[tc.job];
-      const int m0 = tc.mb * kBM, n0 = tc.nb * kBN;
+      const int m0 = tc.mb * kPairM + (int)rank * kBM, n0 = tc.nb * kBN;
       const int row = m0 + r_local;
       const bool row_ok = row < j.M;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kBN;
@@ -351,7 +404,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -361,8 +414,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // no remote arrival or pair MMA is still aimed at either CTA
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kDevErrTimeout);
 }
 
@@ -372,7 +426,7 @@ void gemm_finalize_jobs(GemmParams* p) {
   int begin = 0;
   for (int i = 0; i < p->njobs; ++i) {
     GemmJob& j = p->jobs[i];
-    j.tiles_m = (j.M + kBM - 1) / kBM;
+    j.tiles_m = (j.M + kPairM - 1) / kPairM;
     j.tiles_n = (j.N + kBN - 1) / kBN;
     j.k_steps = (j.K + kBK - 1) / kBK;
     j.tile_begin = begin;
@@ -381,41 +435,81 @@ void gemm_finalize_jobs(GemmParams* p) {
   p->total_tiles = begin;
 }
 
+// Chooses the tile schedule for `P` pairs (see GemmParams::sched).
+void balance_schedule(GemmParams* p, int P) {
+  p->sched = 0;
+  p->na = p->nb = p->rem = 0;
+  if (p->njobs != 2) return;
+  const GemmJob& j0 = p->jobs[0];
+  const GemmJob& j1 = p->jobs[1];
+  const long T0 = (long)j0.tiles_m * j0.tiles_n, T1 = (long)j1.tiles_m * j1.tiles_n;
+  const long c0 = j0.k_steps, c1 = j1.k_steps > 0 ? j1.k_steps : 1;
+  if (T0 > P || c0 < 4 * c1 || T1 == 0) return;  // equal-cost tiles: round-robin is balanced
+  const double ideal = (double)(T0 * c0 + T1 * c1) / P;
+  long nb = (long)(ideal / c1);
+  long na = (long)((ideal - c0) / c1);
+  if (na < 0) na = 0;
+  auto total = [&] { return T0 * na + (P - T0) * nb; };
+  while (total() > T1) {
+    if (P - T0 > 0 && nb > 0 && (na == 0 || nb * c1 >= c0 + na * c1)) --nb;
+    else if (na > 0) --na;
+    else --nb;
+  }
+  while (T1 - total() >= P) {
+    if (P - T0 > 0) ++nb;
+    else ++na;
+  }
+  p->sched = 1;
+  p->na = (int)na;
+  p->nb = (int)nb;
+  p->rem = (int)(T1 - total());
+}
+
+namespace {
+template <typename T>
+cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
+  static int max_pairs = 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kGemmSmem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_pairs == 0) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
+    if (e != cudaSuccess) return e;
+    DevInfo di;
+    if ((e = dev_info(&di)) != cudaSuccess) return e;
+    cfg.gridDim = dim3(di.sm_count & ~1);
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<T>, &cfg);
+    if (e != cudaSuccess) return e;
+    max_pairs = n > 0 ? n : 1;
+  }
+  const int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
+  cfg.gridDim = dim3(2 * pairs);
+  GemmParams q = p;
+  balance_schedule(&q, pairs);
+  launch_begin(0, stream);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<T>, q);
+  launch_end(0, stream);
+  return e;
+}
+}  // namespace
+
 cudaError_t launch_gemm(const GemmParams& p0, DType dt, cudaStream_t stream) {
   if (p0.total_tiles <= 0) return cudaSuccess;
   GemmParams p = p0;
   p.wait_ns = debug_knobs().wait_ns;
   p.extra_tx = debug_knobs().extra_tx;
-  DevInfo di;
-  cudaError_t e = dev_info(&di);
-  if (e != cudaSuccess) return e;
-  const int grid = p.total_tiles < di.sm_count ? p.total_tiles : di.sm_count;
-  if (dt == DType::BF16) {
-    static bool attr = false;
-    if (!attr) {
-      e = cudaFuncSetAttribute(gemm_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kGemmSmem);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
-    launch_begin(0, stream);
-    gemm_kernel<__nv_bfloat16><<<grid, kGemmThreads, kGemmSmem, stream>>>(p);
-    launch_end(0, stream);
-  } else if (dt == DType::F16) {
-    static bool attr = false;
-    if (!attr) {
-      e = cudaFuncSetAttribute(gemm_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kGemmSmem);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
-    launch_begin(0, stream);
-    gemm_kernel<__half><<<grid, kGemmThreads, kGemmSmem, stream>>>(p);
-    launch_end(0, stream);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  if (dt == DType::BF16) return launch_t<__nv_bfloat16>(p, stream);
+  if (dt == DType::F16) return launch_t<__half>(p, stream);
+  return cudaErrorInvalidValue;
 }
 
 // ---------------------------------------------------------------- tensor maps

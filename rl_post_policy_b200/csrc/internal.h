@@ -56,7 +56,24 @@ struct LossArgs {
   int64_t partial_offset;  // byte offset of the f64 block partials inside ws
   unsigned long long wait_ns;
   unsigned extra_arrivals;
+  // Division by seq with a multiply (used when n < 2^32): see seq_divider().
+  unsigned seq_magic, seq_sh1, seq_sh2;
+  int div32;
+  int mask_bits_smem;   // phase A keeps the block's mask bits in shared memory
 };
+
+// Constants of unsigned 32-bit division by an invariant d >= 1 with one
+// multiply-high, after Granlund & Montgomery, "Division by invariant integers
+// using multiplication" (PLDI 1994), section 4:
+//   l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1,
+//   q = (t + ((n - t) >> min(l,1))) >> max(l-1,0) with t = mulhi(m, n).
+inline void seq_divider(uint64_t d, unsigned* magic, unsigned* sh1, unsigned* sh2) {
+  unsigned l = 0;
+  while ((1ull << l) < d) ++l;
+  *magic = (unsigned)(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+  *sh1 = l < 1 ? l : 1;
+  *sh2 = l > 0 ? l - 1 : 0;
+}
 
 // Argument checks shared by the loss entry points (no device call); sets *dt.
 pl_status validate_loss(const void* lp, const void* old, const void* ref, const void* adv,

@@ -28,6 +28,7 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kSmemRows = 64;
+constexpr size_t kMaskBitsBytes = 64 * 1024;  // one byte per vector: up to 512K tokens per block (bf16)
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
@@ -71,6 +72,21 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
   return t;
 }
 
+// Row (sequence) index of token t: one multiply-high when n < 2^32 (see seq_divider).
+__device__ __forceinline__ int64_t row_of(const LossArgs& a, int64_t t) {
+  if (a.div32) {
+    const unsigned n = (unsigned)t;
+    const unsigned q = __umulhi(a.seq_magic, n);
+    return (int64_t)((q + ((n - q) >> a.seq_sh1)) >> a.seq_sh2);
+  }
+  return t / a.seq;
+}
+
+// Number of nonzero bytes in a 32-bit word.
+__device__ __forceinline__ unsigned nonzero_bytes(unsigned w) {
+  return __popc((((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w) & 0x80808080u);
+}
+
 template <typename T>
 __device__ __forceinline__ float load_adv(const LossArgs& a, int64_t r) {
   if (a.adv_lp_dtype) return to_f(reinterpret_cast<const T*>(a.adv)[r]);
@@ -78,8 +94,11 @@ __device__ __forceinline__ float load_adv(const LossArgs& a, int64_t r) {
 }
 
 template <typename T, bool HAS_KL, bool HAS_GRAD, bool TWO_SIDED, bool VEC>
-__global__ void __launch_bounds__(kThreads) loss_kernel(LossArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
   constexpr int VW = VEC ? (int)(16 / sizeof(T)) : 1;
+  // Phase A leaves the block's mask in shared memory as one bit per token (one
+  // byte per vector of VW tokens), so phase B does not read it from HBM again.
+  extern __shared__ uint8_t s_maskbits[];
   __shared__ unsigned long long s_rows[kSmemRows];
   __shared__ double s_red[kThreads / 32];
   __shared__ unsigned long long s_cnt[kThreads / 32];
@@ -106,38 +125,67 @@ __global__ void __launch_bounds__(kThreads) loss_kernel(LossArgs a) {
   __syncthreads();
 
   // ---------------- phase A: valid-token counts ----------------
+  // Same token-to-thread mapping as phase B.  Each thread keeps a run
+  // (row, count) and flushes it when its row changes.
+  const bool bits_in_smem = VEC && a.mask_bits_smem;
   unsigned long long my_total = 0;
   const uint8_t* mk = a.mask;
-  for (int64_t t = t0 + (int64_t)tid * 16; t < t1; t += (int64_t)kThreads * 16) {
-    uint8_t b[16];
-    const int cnt = (int)min((int64_t)16, t1 - t);
-    if (VEC && cnt == 16) {
-      *reinterpret_cast<uint4*>(b) = __ldg(reinterpret_cast<const uint4*>(mk + t));
-    } else {
-      for (int j = 0; j < 16; ++j) b[j] = j < cnt ? mk[t + j] : 0;
-    }
-    int64_t r = t / seq;
-    int64_t boundary = (r + 1) * seq;
-    unsigned c = 0;
-    for (int j = 0; j < cnt; ++j) {
-      if (t + j == boundary) {
-        if (a.need_rows && c) {
-          if (rows_in_smem) atomicAdd(&s_rows[r - r0], (unsigned long long)c);
-          else atomicAdd(&rowcnt[r], (unsigned long long)c);
-        }
-        my_total += c;
-        c = 0;
-        ++r;
-        boundary += seq;
-      }
-      c += b[j] != 0;
-    }
+  int64_t run_row = -1;
+  unsigned run_cnt = 0;
+  auto flush = [&](int64_t r, unsigned c) {
+    my_total += c;
     if (a.need_rows && c) {
       if (rows_in_smem) atomicAdd(&s_rows[r - r0], (unsigned long long)c);
       else atomicAdd(&rowcnt[r], (unsigned long long)c);
     }
-    my_total += c;
+  };
+  auto count_one = [&](int64_t r, unsigned c) {
+    if (r != run_row) {
+      flush(run_row, run_cnt);
+      run_row = r;
+      run_cnt = 0;
+    }
+    run_cnt += c;
+  };
+  for (int64_t t = t0 + (int64_t)tid * VW; t < t1; t += (int64_t)kThreads * VW) {
+    const int64_t r = row_of(a, t);
+    if constexpr (VEC) {
+      if (t + VW <= t1) {
+        unsigned bits = 0;
+        if constexpr (VW == 8) {
+          const uint2 u = __ldg(reinterpret_cast<const uint2*>(mk + t));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            bits |= (((u.x >> (8 * j)) & 0xFFu) != 0u) << j;
+            bits |= (((u.y >> (8 * j)) & 0xFFu) != 0u) << (j + 4);
+          }
+        } else {
+          const unsigned u = __ldg(reinterpret_cast<const unsigned*>(mk + t));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) bits |= (((u >> (8 * j)) & 0xFFu) != 0u) << j;
+        }
+        if (bits_in_smem) s_maskbits[(t - t0) / VW] = (uint8_t)bits;
+        if ((t - r * seq) + VW <= seq) {
+          count_one(r, __popc(bits));
+        } else {
+          int64_t rr = r, boundary = (r + 1) * seq;
+          for (int j = 0; j < VW; ++j) {
+            if (t + j == boundary) { ++rr; boundary += seq; }
+            count_one(rr, (bits >> j) & 1u);
+          }
+        }
+        continue;
+      }
+    }
+    // scalar: unaligned operands, or the ragged tail of the last block
+    const int64_t te = min(t1, t + VW);
+    int64_t rr = r, boundary = (r + 1) * seq;
+    for (int64_t u = t; u < te; ++u) {
+      if (u == boundary) { ++rr; boundary += seq; }
+      count_one(rr, mk[u] != 0);
+    }
   }
+  flush(run_row, run_cnt);
   // block total of valid tokens -> one global atomic
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) my_total += __shfl_xor_sync(0xffffffffu, my_total, o);
@@ -195,10 +243,10 @@ __global__ void __launch_bounds__(kThreads) loss_kernel(LossArgs a) {
     auto scalar_span = [&](int64_t t, int64_t te) {
       // unaligned operands, or the ragged tail of the last block
       for (int64_t u = t; u < te; ++u) {
-        row_state(u / seq);
+        row_state(row_of(a, u));
         float term, dterm;
-        token_math<HAS_KL, TWO_SIDED>(to_f(lp[u]), to_f(od[u]), HAS_KL ? to_f(rf[u]) : 0.0f, A, lo,
-                                      hi, beta, term, dterm);
+        token_math<HAS_KL, TWO_SIDED, true>(to_f(lp[u]), to_f(od[u]), HAS_KL ? to_f(rf[u]) : 0.0f, A, lo,
+                                            hi, beta, term, dterm);
         const bool valid = a.mask[u] != 0;
         acc += valid ? term * scale : 0.0f;
         if (HAS_GRAD) gr[u] = from_f<T>(valid ? dterm * scale : 0.0f);
@@ -214,24 +262,50 @@ __global__ void __launch_bounds__(kThreads) loss_kernel(LossArgs a) {
         load16<T, VW>(lp + t, vl);
         load16<T, VW>(od + t, vo);
         if (HAS_KL) load16<T, VW>(rf + t, vr);
-        uint8_t m[VW];
-        if constexpr (VW == 8) {
-          *reinterpret_cast<uint2*>(m) = __ldg(reinterpret_cast<const uint2*>(a.mask + t));
+        unsigned bits;
+        if (bits_in_smem) {
+          bits = s_maskbits[(t - t0) / VW];
         } else {
-          *reinterpret_cast<unsigned*>(m) = __ldg(reinterpret_cast<const unsigned*>(a.mask + t));
-        }
-        int64_t r = t / seq;
-        int64_t boundary = (r + 1) * seq;
+          bits = 0;
+          if constexpr (VW == 8) {
+            const uint2 u = __ldg(reinterpret_cast<const uint2*>(a.mask + t));
 #pragma unroll
-        for (int j = 0; j < VW; ++j) {
-          if (t + j == boundary) { ++r; boundary += seq; }
+            for (int j = 0; j < 4; ++j) {
+              bits |= (((u.x >> (8 * j)) & 0xFFu) != 0u) << j;
+              bits |= (((u.y >> (8 * j)) & 0xFFu) != 0u) << (j + 4);
+            }
+          } else {
+            const unsigned u = __ldg(reinterpret_cast<const unsigned*>(a.mask + t));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bits |= (((u >> (8 * j)) & 0xFFu) != 0u) << j;
+          }
+        }
+        int64_t r = row_of(a, t);
+        if ((t - r * seq) + VW <= seq) {
+          // the whole vector lies in one sequence
           row_state(r);
-          float term, dterm;
-          token_math<HAS_KL, TWO_SIDED>(vl[j], vo[j], HAS_KL ? vr[j] : 0.0f, A, lo, hi, beta, term,
-                                        dterm);
-          const bool valid = m[j] != 0;
-          acc += valid ? term * scale : 0.0f;
-          vg[j] = valid ? dterm * scale : 0.0f;
+#pragma unroll
+          for (int j = 0; j < VW; ++j) {
+            float term, dterm;
+            token_math<HAS_KL, TWO_SIDED, true>(vl[j], vo[j], HAS_KL ? vr[j] : 0.0f, A, lo, hi, beta,
+                                                term, dterm);
+            const bool valid = (bits >> j) & 1u;
+            acc += valid ? term * scale : 0.0f;
+            vg[j] = valid ? dterm * scale : 0.0f;
+          }
+        } else {
+          int64_t boundary = (r + 1) * seq;
+#pragma unroll
+          for (int j = 0; j < VW; ++j) {
+            if (t + j == boundary) { ++r; boundary += seq; }
+            row_state(r);
+            float term, dterm;
+            token_math<HAS_KL, TWO_SIDED, true>(vl[j], vo[j], HAS_KL ? vr[j] : 0.0f, A, lo, hi, beta,
+                                                term, dterm);
+            const bool valid = (bits >> j) & 1u;
+            acc += valid ? term * scale : 0.0f;
+            vg[j] = valid ? dterm * scale : 0.0f;
+          }
         }
         if (HAS_GRAD) store16<T, VW>(gr + t, vg);
       } else {
@@ -277,9 +351,13 @@ __global__ void __launch_bounds__(kThreads) loss_kernel(LossArgs a) {
 template <typename T, bool HAS_KL, bool HAS_GRAD, bool TWO_SIDED, bool VEC>
 cudaError_t launch_t(const LossArgs& a0, cudaStream_t stream) {
   auto kern = loss_kernel<T, HAS_KL, HAS_GRAD, TWO_SIDED, VEC>;
+  const size_t dyn = VEC ? kMaskBitsBytes : 0;
   static int per_sm = -1;
   if (per_sm < 0) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0);
+    cudaError_t e = cudaSuccess;
+    if (dyn > 48 * 1024)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, dyn);
     if (e != cudaSuccess) { per_sm = -1; return e; }
     if (per_sm < 1) per_sm = 1;
   }
@@ -299,11 +377,13 @@ cudaError_t launch_t(const LossArgs& a0, cudaStream_t stream) {
   if (chunk < 64) chunk = 64;
   grid = a.n > 0 ? (a.n + chunk - 1) / chunk : 1;
   a.chunk = chunk;
+  constexpr int VWh = VEC ? (int)(16 / sizeof(T)) : 1;
+  a.mask_bits_smem = VEC && (chunk / VWh) <= (int64_t)kMaskBitsBytes;
   a.wait_ns = debug_knobs().wait_ns;
   a.extra_arrivals = debug_knobs().extra_arrivals;
   void* args[] = {&a};
   launch_begin(1, stream);
-  e = cudaLaunchCooperativeKernel((const void*)kern, dim3((unsigned)grid), dim3(kThreads), args, 0, stream);
+  e = cudaLaunchCooperativeKernel((const void*)kern, dim3((unsigned)grid), dim3(kThreads), args, dyn, stream);
   launch_end(1, stream);
   return e;
 }

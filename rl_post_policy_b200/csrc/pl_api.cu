@@ -129,6 +129,8 @@ pl_status run_loss(const void* lp, const void* old, const void* ref, const void*
   a.adv_lp_dtype = (mode & PL_ADV_LP_DTYPE) != 0;
   a.need_rows = a.grpo || row_valid_out != nullptr;
   a.partial_offset = (int64_t)loss_partial_offset(bs);
+  a.div32 = seq > 0 && a.n < (1ll << 32) && seq < (1ll << 32);
+  if (a.div32) seq_divider((uint64_t)seq, &a.seq_magic, &a.seq_sh1, &a.seq_sh2);
   const bool has_kl = beta != 0.0f;
   const bool has_grad = grad_out != nullptr;
   const bool vec = aligned(lp, 16) && aligned(old, 16) && (!has_kl || aligned(ref, 16)) &&

@@ -10,10 +10,14 @@
 
 namespace pl {
 
-template <bool HAS_KL, bool TWO_SIDED>
+// FAST selects the hardware exponential (__expf) for both exponentials: a few
+// instructions instead of a few dozen, with a relative error of a few fp32 ulps,
+// far inside every tolerance of the path; the memory-bound loss kernel needs it
+// to stay under its per-token instruction budget at full HBM bandwidth.
+template <bool HAS_KL, bool TWO_SIDED, bool FAST = false>
 __device__ __forceinline__ void token_math(float lp, float old, float ref, float A, float lo, float hi,
                                            float beta, float& term, float& dterm) {
-  const float ratio = expf(lp - old);
+  const float ratio = FAST ? __expf(lp - old) : expf(lp - old);
   const float clipped = fminf(fmaxf(ratio, lo), hi);
   if (!TWO_SIDED) {
     term = -A * fminf(ratio, clipped);
@@ -25,7 +29,7 @@ __device__ __forceinline__ void token_math(float lp, float old, float ref, float
   }
   if (HAS_KL) {
     const float e = ref - lp;
-    const float em1 = expm1f(e);
+    const float em1 = FAST ? __expf(e) - 1.0f : expm1f(e);
     term += beta * (em1 - e);
     dterm -= beta * em1;
   }
