@@ -169,6 +169,14 @@ __device__ __forceinline__ void add_row32_f32(const float* src, float (&v)[32], 
   }
 }
 
+// 2^x with the hardware approximation (flushes subnormal results to zero);
+// the epilogue only takes it of values <= 0, whose results lie in (0, 1].
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <typename T>
 __device__ __forceinline__ void add_bias32(const T* bias, float (&v)[32], int nvalid) {
   if (nvalid >= 32 && ((reinterpret_cast<uintptr_t>(bias) & 15) == 0)) {
@@ -361,18 +369,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           const int nvalid = min(32, j.N - col0);
           if (nvalid <= 0) continue;
           if (bias) add_bias32<T>(bias + col0, v, nvalid);
-          float cmax = -INFINITY;
+          if (nvalid == 32) {
+            // full chunk: no per-column predicates; two columns per packed instruction
+            float cmax = v[0];
 #pragma unroll
-          for (int q = 0; q < 32; ++q)
-            if (q < nvalid) cmax = fmaxf(cmax, v[q]);
-          const float m_new = fmaxf(m_run, cmax);
-          const float mb = m_new * kLog2e;
-          float s = 0.0f;
+            for (int q = 1; q < 32; ++q) cmax = fmaxf(cmax, v[q]);
+            const float m_new = fmaxf(m_run, cmax);
+            const float2 nmb = make_float2(-m_new * kLog2e, -m_new * kLog2e);
+            const float2 l2e = make_float2(kLog2e, kLog2e);
+            float2 s2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-          for (int q = 0; q < 32; ++q)
-            if (q < nvalid) s += exp2f(fmaf(v[q], kLog2e, -mb));
-          s_run = s_run * exp2f(fmaf(m_run, kLog2e, -mb)) + s;
-          m_run = m_new;
+            for (int q = 0; q < 32; q += 2) {
+              const float2 x = __ffma2_rn(make_float2(v[q], v[q + 1]), l2e, nmb);
+              s2 = __fadd2_rn(s2, make_float2(ex2_approx(x.x), ex2_approx(x.y)));
+            }
+            s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, nmb.x)) + (s2.x + s2.y);
+            m_run = m_new;
+          } else {
+            float cmax = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (q < nvalid) cmax = fmaxf(cmax, v[q]);
+            const float m_new = fmaxf(m_run, cmax);
+            const float mb = m_new * kLog2e;
+            float s = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (q < nvalid) s += ex2_approx(fmaf(v[q], kLog2e, -mb));
+            s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, -mb)) + s;
+            m_run = m_new;
+          }
           const int64_t rel = tgt_rel - c * 32;
           if (rel >= 0 && rel < 32) {
 #pragma unroll

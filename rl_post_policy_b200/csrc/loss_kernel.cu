@@ -51,6 +51,49 @@ __device__ __forceinline__ void load16(const T* p, float (&v)[VW]) {
   for (int j = 0; j < VW; ++j) v[j] = to_f(e[j]);
 }
 
+// 16-byte vector of log-probs -> VW/2 float2 pairs (bf16: one shift or mask per element).
+__device__ __forceinline__ void load16_pairs(const __nv_bfloat16* p, float2 (&v)[4]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const unsigned w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) v[k] = make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u));
+}
+__device__ __forceinline__ void load16_pairs(const __half* p, float2 (&v)[4]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const unsigned w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) v[k] = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+}
+__device__ __forceinline__ void load16_pairs(const float* p, float2 (&v)[2]) {
+  const float4 u = __ldg(reinterpret_cast<const float4*>(p));
+  v[0] = make_float2(u.x, u.y);
+  v[1] = make_float2(u.z, u.w);
+}
+
+__device__ __forceinline__ void store16_pairs(__nv_bfloat16* p, const float2 (&g)[4]) {
+  uint4 u;
+  unsigned* w = reinterpret_cast<unsigned*>(&u);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(g[k].x, g[k].y);
+    w[k] = *reinterpret_cast<const unsigned*>(&h);
+  }
+  *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void store16_pairs(__half* p, const float2 (&g)[4]) {
+  uint4 u;
+  unsigned* w = reinterpret_cast<unsigned*>(&u);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __half2 h = __floats2half2_rn(g[k].x, g[k].y);
+    w[k] = *reinterpret_cast<const unsigned*>(&h);
+  }
+  *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void store16_pairs(float* p, const float2 (&g)[2]) {
+  *reinterpret_cast<float4*>(p) = make_float4(g[0].x, g[0].y, g[1].x, g[1].y);
+}
+
 template <typename T, int VW>
 __device__ __forceinline__ void store16(T* p, const float (&v)[VW]) {
   uint4 u;
@@ -70,6 +113,10 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // Row (sequence) index of token t: one multiply-high when n < 2^32 (see seq_divider).
@@ -218,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
 
   // ---------------- phase B: per-token loss and gradient ----------------
   float acc = 0.0f;
+  float2 acc2 = make_float2(0.0f, 0.0f);
   if (!s_flag && any) {
     const unsigned long long total = __ldcg(nvalid);
     const float inv_total = (float)(1.0 / (double)(total > 0 ? total : 1));
@@ -258,10 +306,20 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
           scalar_span(t, t1);
           continue;
         }
-        float vl[VW], vo[VW], vr[VW], vg[VW];
-        load16<T, VW>(lp + t, vl);
-        load16<T, VW>(od + t, vo);
-        if (HAS_KL) load16<T, VW>(rf + t, vr);
+        constexpr int NP = VW / 2;
+        {
+          // bring this thread's next vector toward the SM while this one is computed
+          const int64_t tn = t + (int64_t)kThreads * VW;
+          if (tn + VW <= t1) {
+            prefetch_l2(lp + tn);
+            prefetch_l2(od + tn);
+            if (HAS_KL) prefetch_l2(rf + tn);
+          }
+        }
+        float2 pl[NP], po[NP], pr[NP], pg[NP];
+        load16_pairs(lp + t, pl);
+        load16_pairs(od + t, po);
+        if (HAS_KL) load16_pairs(rf + t, pr);
         unsigned bits;
         if (bits_in_smem) {
           bits = s_maskbits[(t - t0) / VW];
@@ -282,16 +340,17 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
         }
         int64_t r = row_of(a, t);
         if ((t - r * seq) + VW <= seq) {
-          // the whole vector lies in one sequence
+          // the whole vector lies in one sequence: two tokens per packed instruction
           row_state(r);
 #pragma unroll
-          for (int j = 0; j < VW; ++j) {
-            float term, dterm;
-            token_math<HAS_KL, TWO_SIDED, true>(vl[j], vo[j], HAS_KL ? vr[j] : 0.0f, A, lo, hi, beta,
-                                                term, dterm);
-            const bool valid = (bits >> j) & 1u;
-            acc += valid ? term * scale : 0.0f;
-            vg[j] = valid ? dterm * scale : 0.0f;
+          for (int k = 0; k < NP; ++k) {
+            float2 term, dterm;
+            token_math2<HAS_KL, TWO_SIDED>(pl[k], po[k], HAS_KL ? pr[k] : make_float2(0.0f, 0.0f), A, lo, hi,
+                                           beta, term, dterm);
+            const float2 sc = make_float2(((bits >> (2 * k)) & 1u) ? scale : 0.0f,
+                                          ((bits >> (2 * k + 1)) & 1u) ? scale : 0.0f);
+            acc2 = __ffma2_rn(term, sc, acc2);
+            pg[k] = __fmul2_rn(dterm, sc);
           }
         } else {
           int64_t boundary = (r + 1) * seq;
@@ -299,15 +358,18 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
           for (int j = 0; j < VW; ++j) {
             if (t + j == boundary) { ++r; boundary += seq; }
             row_state(r);
+            const float l = (j & 1) ? pl[j >> 1].y : pl[j >> 1].x;
+            const float o = (j & 1) ? po[j >> 1].y : po[j >> 1].x;
+            const float f = HAS_KL ? ((j & 1) ? pr[j >> 1].y : pr[j >> 1].x) : 0.0f;
             float term, dterm;
-            token_math<HAS_KL, TWO_SIDED, true>(vl[j], vo[j], HAS_KL ? vr[j] : 0.0f, A, lo, hi, beta,
-                                                term, dterm);
+            token_math<HAS_KL, TWO_SIDED, true>(l, o, f, A, lo, hi, beta, term, dterm);
             const bool valid = (bits >> j) & 1u;
             acc += valid ? term * scale : 0.0f;
-            vg[j] = valid ? dterm * scale : 0.0f;
+            const float gv = valid ? dterm * scale : 0.0f;
+            if (j & 1) pg[j >> 1].y = gv; else pg[j >> 1].x = gv;
           }
         }
-        if (HAS_GRAD) store16<T, VW>(gr + t, vg);
+        if (HAS_GRAD) store16_pairs(gr + t, pg);
       } else {
         scalar_span(t, t + 1);
       }
@@ -315,6 +377,7 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
   }
 
   // block partial (warp shuffle in fp32, then fp64 across warps)
+  acc += acc2.x + acc2.y;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) s_red[warp] = (double)acc;
@@ -332,10 +395,19 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
   __syncthreads();
   if (s_flag == 2) {
     __threadfence();
+    // Fixed-order fp64 sum of the block partials: thread i takes partials i,
+    // i+512, ... in order, then a fixed shuffle tree and warp order -- the same
+    // result on every run for a given grid.
+    double ps = 0.0;
+    for (unsigned b = tid; b < gridDim.x; b += kThreads) ps += __ldcg(&partial[b]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+    if (lane == 0) s_red[warp] = ps;
+    __syncthreads();
     if (tid == 0) {
-      double s = 0.0;
-      for (unsigned b = 0; b < gridDim.x; ++b) s += __ldcg(&partial[b]);
-      *a.loss_out = (float)s;
+      double sum = 0.0;
+      for (int w = 0; w < kThreads / 32; ++w) sum += s_red[w];
+      *a.loss_out = (float)sum;
       if (a.n_valid_out) *a.n_valid_out = (int64_t)__ldcg(nvalid);
       *nvalid = 0ull;
       *arrive = 0u;
