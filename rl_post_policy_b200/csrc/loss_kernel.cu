@@ -172,8 +172,10 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
   __syncthreads();
 
   // ---------------- phase A: valid-token counts ----------------
-  // Same token-to-thread mapping as phase B.  Each thread keeps a run
-  // (row, count) and flushes it when its row changes.
+  // Each thread reads 16 mask bytes per load, four independent loads at a time
+  // (64 KB in flight per SM), keeps a run (row, count) that it flushes when its
+  // row changes, and -- on the vector path -- leaves the block's mask in shared
+  // memory as one bit per token (one byte per VW-token vector) for phase B.
   const bool bits_in_smem = VEC && a.mask_bits_smem;
   unsigned long long my_total = 0;
   const uint8_t* mk = a.mask;
@@ -194,42 +196,67 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
     }
     run_cnt += c;
   };
-  for (int64_t t = t0 + (int64_t)tid * VW; t < t1; t += (int64_t)kThreads * VW) {
-    const int64_t r = row_of(a, t);
-    if constexpr (VEC) {
-      if (t + VW <= t1) {
-        unsigned bits = 0;
-        if constexpr (VW == 8) {
-          const uint2 u = __ldg(reinterpret_cast<const uint2*>(mk + t));
+  // 16 mask bytes starting at token t (t - t0 a multiple of 16): counts, and bits into shared memory.
+  auto mask16 = [&](int64_t t, const uint4 u) {
+    const unsigned w[4] = {u.x, u.y, u.z, u.w};
+    unsigned h[4], nib[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            bits |= (((u.x >> (8 * j)) & 0xFFu) != 0u) << j;
-            bits |= (((u.y >> (8 * j)) & 0xFFu) != 0u) << (j + 4);
-          }
-        } else {
-          const unsigned u = __ldg(reinterpret_cast<const unsigned*>(mk + t));
+    for (int q = 0; q < 4; ++q) {
+      h[q] = (((w[q] & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w[q]) & 0x80808080u;   // high bit of each nonzero byte
+      nib[q] = ((h[q] >> 7) | (h[q] >> 14) | (h[q] >> 21) | (h[q] >> 28)) & 0xFu;
+    }
+    if (bits_in_smem) {
+      const int64_t vi = (t - t0) / VW;
+      if constexpr (VW == 8) {
+        s_maskbits[vi] = (uint8_t)(nib[0] | (nib[1] << 4));
+        s_maskbits[vi + 1] = (uint8_t)(nib[2] | (nib[3] << 4));
+      } else {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) bits |= (((u >> (8 * j)) & 0xFFu) != 0u) << j;
-        }
-        if (bits_in_smem) s_maskbits[(t - t0) / VW] = (uint8_t)bits;
-        if ((t - r * seq) + VW <= seq) {
-          count_one(r, __popc(bits));
-        } else {
-          int64_t rr = r, boundary = (r + 1) * seq;
-          for (int j = 0; j < VW; ++j) {
-            if (t + j == boundary) { ++rr; boundary += seq; }
-            count_one(rr, (bits >> j) & 1u);
-          }
-        }
-        continue;
+        for (int q = 0; q < 4; ++q) s_maskbits[vi + q] = (uint8_t)nib[q];
       }
     }
-    // scalar: unaligned operands, or the ragged tail of the last block
-    const int64_t te = min(t1, t + VW);
-    int64_t rr = r, boundary = (r + 1) * seq;
-    for (int64_t u = t; u < te; ++u) {
-      if (u == boundary) { ++rr; boundary += seq; }
-      count_one(rr, mk[u] != 0);
+    const int64_t r = row_of(a, t);
+    if ((t - r * seq) + 16 <= seq) {
+      count_one(r, __popc(h[0]) + __popc(h[1]) + __popc(h[2]) + __popc(h[3]));
+    } else {
+      int64_t rr = r, boundary = (r + 1) * seq;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (t + j == boundary) { ++rr; boundary += seq; }
+        count_one(rr, (nib[j >> 2] >> (j & 3)) & 1u);
+      }
+    }
+  };
+  constexpr int kU = 4;
+  for (int64_t base = t0 + (int64_t)tid * 16; base < t1; base += (int64_t)kThreads * 16 * kU) {
+    uint4 u[kU];
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      const int64_t t = base + (int64_t)k * kThreads * 16;
+      if (VEC && t + 16 <= t1) u[k] = __ldg(reinterpret_cast<const uint4*>(mk + t));
+    }
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      const int64_t t = base + (int64_t)k * kThreads * 16;
+      if (t >= t1) break;
+      if (VEC && t + 16 <= t1) {
+        mask16(t, u[k]);
+      } else {
+        // ragged tail of the last block, or unaligned operands: byte by byte
+        const int64_t te = min(t1, t + 16);
+        int64_t rr = row_of(a, t), boundary = (rr + 1) * seq;
+        unsigned vbits = 0;
+        for (int64_t v = t; v < te; ++v) {
+          if (v == boundary) { ++rr; boundary += seq; }
+          const unsigned m = mk[v] != 0;
+          count_one(rr, m);
+          vbits |= m << ((v - t0) % VW);
+          if (bits_in_smem && ((v - t0) % VW == VW - 1 || v == te - 1)) {
+            s_maskbits[(v - t0) / VW] = (uint8_t)vbits;
+            vbits = 0;
+          }
+        }
+      }
     }
   }
   flush(run_row, run_cnt);
