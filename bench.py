@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5])
+    ap.add_argument("--chunk-rows", type=int, default=-1,
+                    help="rows per chunk (multiple of 128); -1: the whole batch in one chunk")
     ap.add_argument("--no-loss-only", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256, help="rows in the oracle's timed sample")
@@ -203,7 +205,15 @@ def workload_desc(w: int) -> dict:
     return d
 
 
-def make_fused_inputs(w: int, rank: int):
+def chunk_mode(N: int, chunk_rows: int) -> int:
+    """PL_CHUNK_ROWS bits: -1 = one chunk covering the batch (up to 32640 rows)."""
+    import rl_post_policy_b200 as pl
+    c = N if chunk_rows < 0 else chunk_rows
+    c = max(128, min(32640, (c + 127) // 128 * 128))
+    return pl.PL_CHUNK_ROWS(c), c
+
+
+def make_fused_inputs(w: int, rank: int, chunk_rows: int = -1):
     """Synthetic inputs on the GPU; old_lp = policy log-prob (from a forward-only
     call of the same entry point) + N(0, 0.1)."""
     import rl_post_policy_b200 as pl
@@ -213,7 +223,8 @@ def make_fused_inputs(w: int, rank: int):
                              bias=d.get("bias", False), len_lo=d["len_lo"], len_hi=d["len_hi"],
                              fully_masked_last=d.get("fully_masked_last", False), device="cuda")
     N, V, H, bs, T = d["N"], d["V"], d["H"], d["bs"], d["T"]
-    mode = pl.dtype_mode(d["dtype"]) | pl.PL_GRPO
+    cbits, d["chunk_rows"] = chunk_mode(N, chunk_rows)
+    mode = pl.dtype_mode(d["dtype"]) | pl.PL_GRPO | cbits
     wsb = pl.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, 1, int(inp["bias"] is not None))
     ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
     loss = torch.zeros(1, device="cuda")
@@ -374,7 +385,7 @@ def run_ours(args):
     ws_world, rank = dist_init(args)
     import rl_post_policy_b200 as pl
     peaks, peak_kind = load_peaks()
-    d, inp, ws, wsb, mode = make_fused_inputs(args.workload, rank)
+    d, inp, ws, wsb, mode = make_fused_inputs(args.workload, rank, args.chunk_rows)
     step = FusedStep(d, inp, ws, wsb, mode)
     N, H, V = d["N"], d["H"], d["V"]
     for _ in range(args.warmup):
@@ -460,7 +471,7 @@ def run_ours(args):
             "dtype": "bf16" if d["dtype"] == torch.bfloat16 else "fp16", "data": "synthetic",
             "config": {"workload": f"fused GRPO fwd+bwd, bs={d['bs']} x T={d['T']} (N={N}), H={H}, V={V}, "
                                    f"beta={d['beta']}, GRPO, eps=0.2/0.28",
-                       "per_gpu_rows": N, "chunk_rows": 1024,
+                       "per_gpu_rows": N, "chunk_rows": d["chunk_rows"],
                        "l2": "inputs larger than L2 (W and Wref are 1 GB each); no flush",
                        "parallelism": f"dp{ws_world} (independent batches)"},
             "clocks": clk, "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,

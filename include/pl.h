@@ -202,6 +202,58 @@ pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias,
 size_t pl_fused_linear_grpo_workspace_bytes(int64_t bs, int64_t T, int64_t H, int64_t V,
                                             uint32_t mode, int need_dW, int need_dbias);
 
+/* pl_fused_linear_grpo_temp: pl_fused_linear_grpo at a sampling temperature
+ * tau > 0 (finite); pl_fused_linear_grpo is this call with tau = 1.  The logits
+ * of both models are z = (X W^T (+ bias)) / tau, so logp = log_softmax(z)[target];
+ * the gradients returned are with respect to X, W and bias (the 1/tau of the
+ * chain rule included).  ("Add SM100 CuTe DSL GRPO fast path", "Native scope",
+ * names temperature 1.0 as that design's scope; other temperatures went to its
+ * older path.)  Same workspace as pl_fused_linear_grpo.
+ */
+pl_status pl_fused_linear_grpo_temp(const void* X, const void* W, const void* bias,
+                                    const int64_t* targets, const void* Xref, const void* Wref,
+                                    const float* old_lp, const void* adv, const uint8_t* mask,
+                                    int64_t bs, int64_t T, int64_t H, int64_t V,
+                                    float eps_lo, float eps_hi, float beta, float temperature,
+                                    uint32_t mode, float* loss, void* dX, void* dW, void* dbias,
+                                    float* logp_out, float* ref_logp_out, int64_t* n_valid_out,
+                                    void* workspace, size_t ws_bytes, pl_stream_t stream);
+
+/* pl_fused_selective_logprob: the fused linear path without the loss step, the
+ * shape of the "fused-linear selective-logprob autograd path" of "Add SM100 CuTe
+ * DSL GRPO fast path" (Liger-Kernel PR #1363, "Summary"):
+ *   forward  : logp_out[i] = log_softmax(X[i] W^T + bias)[targets[i]]   (fp32, [N])
+ *   backward : with grad_logp[i] = dL/dlogp_i supplied (fp32, [N]),
+ *              dz = grad_logp * (onehot(target) - softmax(z)),
+ *              dX = dz W [N,H], dW = dz^T X [V,H], dbias = sum over rows of dz [V].
+ * The same kernels as pl_fused_linear_grpo run: one tcgen05 GEMM per chunk of rows
+ * with the logsumexp / target-logit epilogue, then (for the backward) the in-place
+ * dlogits pass and the dX / dW GEMMs with fp32 dW accumulation across chunks.
+ *   X [N,H], W [V,H], bias [V] or NULL : PL_F16 / PL_BF16 (mode bits 4-7; bits 16-23 chunk rows).
+ *   targets [N] int64; an id outside [0, V) gives logp NaN, zero gradient and
+ *   PL_ERR_BAD_TARGET in pl_device_status.
+ *   grad_logp [N] fp32 or NULL; dX / dW / dbias (model dtype) require it.
+ *   logp_out [N] fp32 or NULL (at least one output must be requested).
+ *   workspace: pl_fused_selective_logprob_workspace_bytes() bytes, 256-byte aligned,
+ *   zero-filled once after allocation.
+ */
+pl_status pl_fused_selective_logprob(const void* X, const void* W, const void* bias,
+                                     const int64_t* targets, int64_t N, int64_t H, int64_t V,
+                                     uint32_t mode, const float* grad_logp, float* logp_out,
+                                     void* dX, void* dW, void* dbias, void* workspace,
+                                     size_t ws_bytes, pl_stream_t stream);
+
+size_t pl_fused_selective_logprob_workspace_bytes(int64_t N, int64_t H, int64_t V, uint32_t mode,
+                                                  int need_dW, int need_dbias);
+
+/* pl_scale: x[i] *= *scale for n elements of the mode's dtype (bits 4-7), in place
+ * on `stream`; `scale` is a device fp32 scalar, so the host never waits.  It
+ * carries the chain rule for the autograd wrappers: the gradient of a scalar
+ * loss times the loss's incoming gradient (the card's "Entry points" section:
+ * the autograd-aware variant runs the same fused kernel).
+ */
+pl_status pl_scale(void* x, int64_t n, uint32_t mode, const float* scale, pl_stream_t stream);
+
 /* ---- status ---------------------------------------------------------------------
  * pl_device_status: synchronises `stream`, reads the sticky device error flag of
  * `workspace` (NULL = pl_loss's own scratch for the current device and `stream`),

@@ -59,10 +59,10 @@ def _load():
                                         P, P, P, P, P]
         lib.orc_policy_loss.restype = I32
         lib.orc_lm_head_logprob.argtypes = [P, I32, P, I32, P, I32, P, P, I64, I64, I64,
-                                            I64, I32, P, P, P]
+                                            I64, I32, D, P, P, P]
         lib.orc_lm_head_logprob.restype = I32
         lib.orc_lm_head_backward.argtypes = [P, I32, P, I32, P, I32, P, P, P, I64, I64,
-                                             I64, I32, P, I64, P, P, I64, P, P]
+                                             I64, I32, D, P, I64, P, P, I64, P, P]
         lib.orc_lm_head_backward.restype = I32
         _lib = lib
     return _lib
@@ -127,8 +127,9 @@ def policy_loss(lp, old_lp, ref_lp, adv, mask, *, eps_lo: float, eps_hi: float,
             "row_valid": rv[:bs].copy(), "abs_sum": float(ab[0])}
 
 
-def lm_head_logprob(X, W, bias, targets, rows=None, nthreads: int = 0):
-    """(lse, logp, target_logit) for the selected rows (all rows if ``rows`` is None)."""
+def lm_head_logprob(X, W, bias, targets, rows=None, nthreads: int = 0, temperature: float = 1.0):
+    """(lse, logp, target_logit) for the selected rows (all rows if ``rows`` is None);
+    logits are (X W^T + bias) / temperature."""
     Xt, Wt = _t(X), _t(W)
     N, H = Xt.shape
     V = Wt.shape[0]
@@ -141,13 +142,15 @@ def lm_head_logprob(X, W, bias, targets, rows=None, nthreads: int = 0):
     zt = np.zeros(n)
     rc = _load().orc_lm_head_logprob(_p(Xt), _DT[Xt.dtype], _p(Wt), _DT[Wt.dtype], _p(bt),
                                      _DT[bt.dtype] if bt is not None else 0, _p(tg), _p(ri),
-                                     n, N, H, V, nthreads, _p(lse), _p(logp), _p(zt))
+                                     n, N, H, V, nthreads, float(temperature), _p(lse), _p(logp),
+                                     _p(zt))
     if rc:
         raise ValueError(f"oracle: lm_head_logprob failed (rc={rc})")
     return lse, logp, zt
 
 
-def lm_head_backward(X, W, bias, targets, lse, g, dx_rows, dw_rows, nthreads: int = 0):
+def lm_head_backward(X, W, bias, targets, lse, g, dx_rows, dw_rows, nthreads: int = 0,
+                     temperature: float = 1.0):
     """(dX[dx_rows], dW[dw_rows], dbias[dw_rows]) in fp64 given per-row lse and g."""
     Xt, Wt = _t(X), _t(W)
     N, H = Xt.shape
@@ -163,7 +166,8 @@ def lm_head_backward(X, W, bias, targets, lse, g, dx_rows, dw_rows, nthreads: in
     db = np.zeros(len(dwr))
     rc = _load().orc_lm_head_backward(_p(Xt), _DT[Xt.dtype], _p(Wt), _DT[Wt.dtype], _p(bt),
                                       _DT[bt.dtype] if bt is not None else 0, _p(tg),
-                                      _p(lse), _p(g), N, H, V, nthreads, _p(dxr), len(dxr),
+                                      _p(lse), _p(g), N, H, V, nthreads, float(temperature),
+                                      _p(dxr), len(dxr),
                                       _p(dX), _p(dwr), len(dwr), _p(dW), _p(db))
     if rc:
         raise ValueError(f"oracle: lm_head_backward failed (rc={rc})")
@@ -172,7 +176,7 @@ def lm_head_backward(X, W, bias, targets, lse, g, dx_rows, dw_rows, nthreads: in
 
 def fused_grpo(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, *, eps_lo: float,
                eps_hi: float, beta: float, reduction: int, two_sided: bool = False,
-               dx_rows="all", dw_rows="all", nthreads: int = 0) -> dict:
+               dx_rows="all", dw_rows="all", nthreads: int = 0, temperature: float = 1.0) -> dict:
     """Fused linear GRPO/BNPO forward + backward, composed from the three steps.
 
     ``mask`` is (bs, T); the N = bs*T rows of X are sequence-major.  The
@@ -186,9 +190,9 @@ def fused_grpo(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, *, eps_lo: fl
     V = _t(W).shape[0]
     if N != bs * T:
         raise ValueError("oracle: X rows must equal bs*T")
-    lse, logp, _ = lm_head_logprob(X, W, bias, targets, None, nthreads)
+    lse, logp, _ = lm_head_logprob(X, W, bias, targets, None, nthreads, temperature)
     if beta != 0.0:
-        _, ref_logp, _ = lm_head_logprob(Xref, Wref, None, targets, None, nthreads)
+        _, ref_logp, _ = lm_head_logprob(Xref, Wref, None, targets, None, nthreads, temperature)
     else:
         ref_logp = None
     lo = policy_loss(logp.reshape(bs, T), old_lp, None if ref_logp is None else ref_logp.reshape(bs, T),
@@ -197,7 +201,7 @@ def fused_grpo(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, *, eps_lo: fl
     g = lo["grad"].reshape(N)
     dxr = np.arange(N) if isinstance(dx_rows, str) else np.asarray(dx_rows, dtype=np.int64)
     dwr = np.arange(V) if isinstance(dw_rows, str) else np.asarray(dw_rows, dtype=np.int64)
-    dX, dW, db = lm_head_backward(X, W, bias, targets, lse, g, dxr, dwr, nthreads)
+    dX, dW, db = lm_head_backward(X, W, bias, targets, lse, g, dxr, dwr, nthreads, temperature)
     return {"loss": lo["loss"], "abs_sum": lo["abs_sum"], "n_valid": lo["n_valid"],
             "row_valid": lo["row_valid"], "logp": logp, "ref_logp": ref_logp, "lse": lse,
             "g": g, "dX": dX, "dW": dW, "dbias": db, "dx_rows": dxr, "dw_rows": dwr}

@@ -12,10 +12,11 @@
 //                      with respect to the policy log-probs is the analytic
 //                      derivative of that loss (the card's fused forward+backward
 //                      returns (loss, grad_logprobs)).
-//   * lm_head_logprob -- selective log-probability at temperature 1.0:
-//                      z = X W^T (+ b), logp = z[target] - logsumexp(z), as used by
-//                      "Add SM100 CuTe DSL GRPO fast path" (Liger-Kernel PR #1363),
-//                      "Summary" and "Native scope".
+//   * lm_head_logprob -- selective log-probability: z = (X W^T (+ b)) / temperature,
+//                      logp = z[target] - logsumexp(z), as used by "Add SM100 CuTe
+//                      DSL GRPO fast path" (Liger-Kernel PR #1363), "Summary" and
+//                      "Native scope" (temperature 1.0 natively, other temperatures
+//                      handled by the page's older path).
 //   * lm_head_backward -- the chain rule through log-softmax and the linear layer:
 //                      dz = g * (onehot(target) - softmax(z)), dX = dz W,
 //                      dW = dz^T X, dbias = sum over rows of dz.
@@ -258,8 +259,8 @@ int orc_policy_loss(const double* lp, const double* old_lp, const double* ref_lp
 }
 
 // Selective log-probability: for each selected row i,
-//   z_v = sum_h X[i,h] * W[v,h] (+ bias[v]),   lse = M + log(sum_v exp(z_v - M)),
-//   logp = z[target_i] - lse.
+//   z_v = (sum_h X[i,h] * W[v,h] (+ bias[v])) / temperature,
+//   lse = M + log(sum_v exp(z_v - M)),   logp = z[target_i] - lse.
 //   X [N,H] (dtype xdt), W [V,H] (wdt), bias [V] (bdt) or NULL, targets [N].
 //   rows: indices of the rows to evaluate (NULL = all N rows, in order).
 // Writes lse_out[k], logp_out[k] and, if ztgt_out, the target logit, for the
@@ -267,8 +268,9 @@ int orc_policy_loss(const double* lp, const double* old_lp, const double* ref_lp
 int orc_lm_head_logprob(const void* X, int xdt, const void* W, int wdt,
                         const void* bias, int bdt, const int64_t* targets,
                         const int64_t* rows, int64_t nsel, int64_t N, int64_t H,
-                        int64_t V, int nthreads, double* lse_out, double* logp_out,
-                        double* ztgt_out) {
+                        int64_t V, int nthreads, double temperature, double* lse_out,
+                        double* logp_out, double* ztgt_out) {
+  if (!(temperature > 0.0)) return 1;
   if (!X || !W || !targets || !lse_out || !logp_out || H <= 0 || V <= 0) return 1;
   if (!rows) nsel = N;
   const int workers = worker_count(nthreads);
@@ -294,7 +296,7 @@ int orc_lm_head_logprob(const void* X, int xdt, const void* W, int wdt,
         load_row(wdt, W, v * H, H, w.data());
         if (gr <= 4) dot4(xT.data(), w.data(), H, acc); else dot32(xT.data(), w.data(), H, acc);
         const double b = bias ? load(bdt, bias, v) : 0.0;
-        for (int r = 0; r < gr; ++r) z[(size_t)r * V + v] = acc[r] + b;
+        for (int r = 0; r < gr; ++r) z[(size_t)r * V + v] = (acc[r] + b) / temperature;
       }
     });
 
@@ -314,9 +316,10 @@ int orc_lm_head_logprob(const void* X, int xdt, const void* W, int wdt,
   return 0;
 }
 
-// Backward through log-softmax and the linear layer.
+// Backward through log-softmax, the temperature and the linear layer.
 //   lse [N], g [N]: per-row logsumexp and dLoss/dlogp for ALL N rows.
-//   dz[i,v] = g_i * ([v == target_i] - exp(z_iv - lse_i))
+//   dz[i,v] = g_i * ([v == target_i] - exp(z_iv - lse_i)) / temperature
+//   (the gradient with respect to the raw logit X W^T + b)
 //   dX rows : for each index in dx_rows (n_dx of them)  dX[i,:] = sum_v dz[i,v] W[v,:]
 //   dW rows : for each vocab index in dw_rows (n_dw)    dW[v,:] = sum_i dz[i,v] X[i,:]
 //             and dbias[v] = sum_i dz[i,v]
@@ -324,9 +327,10 @@ int orc_lm_head_logprob(const void* X, int xdt, const void* W, int wdt,
 int orc_lm_head_backward(const void* X, int xdt, const void* W, int wdt,
                          const void* bias, int bdt, const int64_t* targets,
                          const double* lse, const double* g, int64_t N, int64_t H,
-                         int64_t V, int nthreads, const int64_t* dx_rows, int64_t n_dx,
-                         double* dX_out, const int64_t* dw_rows, int64_t n_dw,
+                         int64_t V, int nthreads, double temperature, const int64_t* dx_rows,
+                         int64_t n_dx, double* dX_out, const int64_t* dw_rows, int64_t n_dw,
                          double* dW_out, double* dbias_out) {
+  if (!(temperature > 0.0)) return 1;
   if (!X || !W || !targets || !lse || !g || H <= 0 || V <= 0 || N < 0) return 1;
   const int workers = worker_count(nthreads);
 
@@ -358,8 +362,9 @@ int orc_lm_head_backward(const void* X, int xdt, const void* W, int wdt,
           for (int r = 0; r < gr; ++r) {
             const int64_t i = idx[r];
             if (g[i] == 0.0) continue;               // dz row is exactly zero
-            const double p = std::exp(acc[r] + b - lse[i]);
-            const double dz = g[i] * ((v == targets[i] ? 1.0 : 0.0) - p);
+            const double p = std::exp((acc[r] + b) / temperature - lse[i]);
+            // dLoss/d(raw logit) = dLoss/dz / temperature, z = raw / temperature
+            const double dz = g[i] * ((v == targets[i] ? 1.0 : 0.0) - p) / temperature;
             double* out = &dxp[(size_t)r * H];
             for (int64_t h = 0; h < H; ++h) out[h] += dz * w[h];
           }
@@ -404,8 +409,8 @@ int orc_lm_head_backward(const void* X, int xdt, const void* W, int wdt,
           for (int r = 0; r < gr; ++r) {
             const int64_t i = gi * 32 + r;
             if (g[i] == 0.0) continue;               // dz row is exactly zero
-            const double zi = acc[r] + b;
-            const double dz = g[i] * ((v == targets[i] ? 1.0 : 0.0) - std::exp(zi - lse[i]));
+            const double zi = (acc[r] + b) / temperature;
+            const double dz = g[i] * ((v == targets[i] ? 1.0 : 0.0) - std::exp(zi - lse[i])) / temperature;
             const double* xi = &Xd[(size_t)i * H];
             for (int64_t h = 0; h < H; ++h) out[h] += dz * xi[h];
             db += dz;

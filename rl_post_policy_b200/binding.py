@@ -51,8 +51,19 @@ _lib.pl_loss_workspace_bytes.restype = _SZ
 _lib.pl_fused_linear_grpo.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64,
                                       _F, _F, _F, _U32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
 _lib.pl_fused_linear_grpo.restype = _I
+_lib.pl_fused_linear_grpo_temp.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64,
+                                           _F, _F, _F, _F, _U32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                                           _P]
+_lib.pl_fused_linear_grpo_temp.restype = _I
 _lib.pl_fused_linear_grpo_workspace_bytes.argtypes = [_I64, _I64, _I64, _I64, _U32, _I, _I]
 _lib.pl_fused_linear_grpo_workspace_bytes.restype = _SZ
+_lib.pl_fused_selective_logprob.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _U32, _P, _P, _P, _P, _P,
+                                            _P, _SZ, _P]
+_lib.pl_fused_selective_logprob.restype = _I
+_lib.pl_fused_selective_logprob_workspace_bytes.argtypes = [_I64, _I64, _I64, _U32, _I, _I]
+_lib.pl_fused_selective_logprob_workspace_bytes.restype = _SZ
+_lib.pl_scale.argtypes = [_P, _I64, _U32, _P, _P]
+_lib.pl_scale.restype = _I
 _lib.pl_device_status.argtypes = [_P, _P]
 _lib.pl_device_status.restype = _I
 _lib.pl_status_string.argtypes = [_I]
@@ -72,7 +83,8 @@ _lib.pl_debug_pair_tiles.restype = _I
 _lib.pl_debug_launch_count.argtypes = []
 _lib.pl_debug_launch_count.restype = _I64
 
-EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_static", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
+EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_linear_grpo_temp", "pl_fused_selective_logprob",
+            "pl_fused_selective_logprob_workspace_bytes", "pl_scale", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
             "pl_version", "pl_debug_gemm", "pl_debug_timing", "pl_debug_timing_read",
             "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_pair_tiles")
@@ -150,9 +162,35 @@ def pl_fused_linear_grpo(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, bs,
         _ptr(workspace), ws_bytes, _stream(stream))
 
 
+def pl_fused_linear_grpo_temp(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, bs, T, H, V, eps_lo,
+                              eps_hi, beta, temperature, mode, loss, dX, dW, dbias, logp_out, ref_logp_out,
+                              n_valid_out, workspace, ws_bytes, stream=None) -> int:
+    return _lib.pl_fused_linear_grpo_temp(
+        _ptr(X), _ptr(W), _ptr(bias), _ptr(targets), _ptr(Xref), _ptr(Wref), _ptr(old_lp),
+        _ptr(adv), _ptr(mask), bs, T, H, V, eps_lo, eps_hi, beta, temperature, mode, _ptr(loss),
+        _ptr(dX), _ptr(dW), _ptr(dbias), _ptr(logp_out), _ptr(ref_logp_out), _ptr(n_valid_out),
+        _ptr(workspace), ws_bytes, _stream(stream))
+
+
 def pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, need_dW, need_dbias) -> int:
     return int(_lib.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, int(need_dW),
                                                          int(need_dbias)))
+
+
+def pl_fused_selective_logprob(X, W, bias, targets, N, H, V, mode, grad_logp, logp_out, dX, dW, dbias,
+                               workspace, ws_bytes, stream=None) -> int:
+    return _lib.pl_fused_selective_logprob(_ptr(X), _ptr(W), _ptr(bias), _ptr(targets), N, H, V, mode,
+                                           _ptr(grad_logp), _ptr(logp_out), _ptr(dX), _ptr(dW),
+                                           _ptr(dbias), _ptr(workspace), ws_bytes, _stream(stream))
+
+
+def pl_fused_selective_logprob_workspace_bytes(N, H, V, mode, need_dW, need_dbias) -> int:
+    return int(_lib.pl_fused_selective_logprob_workspace_bytes(N, H, V, mode, int(need_dW),
+                                                               int(need_dbias)))
+
+
+def pl_scale(x, n, mode, scale, stream=None) -> int:
+    return _lib.pl_scale(_ptr(x), n, mode, _ptr(scale), _stream(stream))
 
 
 def pl_device_status(workspace=None, stream=None) -> int:

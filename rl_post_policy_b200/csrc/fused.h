@@ -49,6 +49,8 @@ struct CombineArgs {
   int chunk, part_stride;
   float lo, hi, beta;
   int grpo, adv_lp_dtype, bf16;
+  const float* grad_logp;   // selective log-prob form: external dLoss/dlogp [N]
+  float g_scale;            // 1 / temperature: dLoss/dlogp -> gradient of the raw logits
 };
 
 struct DlogitsArgs {
@@ -68,6 +70,10 @@ cudaError_t launch_count(const uint8_t* mask, int64_t bs, int64_t T, unsigned ch
                          const FusedOffsets& off, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, bool has_kl, bool two_sided, cudaStream_t s);
 cudaError_t launch_dlogits(const DlogitsArgs& a, DType dt, cudaStream_t s);
+// Selective log-prob form: lse and logp per row, g_i = grad_logp[i] (0 when null).
+cudaError_t launch_combine_ext(const CombineArgs& a, cudaStream_t s);
+// Zeroes the per-chunk max|g| slots (the count kernel does it in the loss form).
+cudaError_t launch_clear_gmax(unsigned char* ws, int nchunks, const FusedOffsets& off, cudaStream_t s);
 cudaError_t launch_finalize(const unsigned char* ws, const FusedOffsets& off, int nchunks, int part_stride,
                             int nblocks_last, float* loss, int64_t* n_valid_out, cudaStream_t s);
 

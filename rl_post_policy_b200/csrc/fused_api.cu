@@ -82,66 +82,62 @@ AccMode acc_mode(int64_t chunk, int64_t nchunks) {
 }  // namespace
 }  // namespace pl
 
-using namespace pl;
 
-extern "C" {
+namespace pl {
+namespace {
 
-size_t pl_fused_linear_grpo_workspace_bytes(int64_t bs, int64_t T, int64_t H, int64_t V, uint32_t mode,
-                                            int need_dW, int need_dbias) {
-  if (bs < 0 || T < 0 || H < 0 || V < 0) return 0;
-  return (size_t)make_plan(bs, T, H, V, mode, need_dW != 0, need_dbias != 0).off.total;
-}
+// Everything the per-chunk pipeline needs.  `ext_g` selects the selective
+// log-prob form: no loss, g_i = grad_logp[i] (external), no counts/finalize.
+struct Pipe {
+  const void* X; const void* W; const void* bias; const int64_t* targets;
+  const void* Xref; const void* Wref; const float* old_lp; const void* adv; const uint8_t* mask;
+  int64_t bs, T, H, V;
+  float eps_lo, eps_hi, beta;
+  uint32_t mode;
+  float* loss; void* dX; void* dW; void* dbias; float* logp_out; float* ref_logp_out; int64_t* n_valid_out;
+  const float* grad_logp;
+  bool ext_g;
+  float inv_temp;
+  void* workspace;
+  pl_stream_t stream;
+  DType dt;
+  Plan plan;
+};
 
-pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias, const int64_t* targets,
-                               const void* Xref, const void* Wref, const float* old_lp, const void* adv,
-                               const uint8_t* mask, int64_t bs, int64_t T, int64_t H, int64_t V,
-                               float eps_lo, float eps_hi, float beta, uint32_t mode, float* loss,
-                               void* dX, void* dW, void* dbias, float* logp_out, float* ref_logp_out,
-                               int64_t* n_valid_out, void* workspace, size_t ws_bytes,
-                               pl_stream_t stream) {
-  // ---------------- host-side validation (no device call) ----------------
-  if (bs < 0 || T < 0 || H < 0 || V < 0 || !loss) return PL_ERR_ARG;
-  if (T > 0 && bs > INT64_MAX / T) return PL_ERR_ARG;
-  if (mode & ~kFusedModeBits) return PL_ERR_ARG;
-  if ((mode & PL_REDUCTION_MASK) > PL_GRPO) return PL_ERR_ARG;
-  const uint32_t dcode = (mode & PL_DTYPE_MASK) >> 4;
-  if (dcode != 1 && dcode != 2) return PL_ERR_DTYPE;
-  const DType dt = (DType)dcode;
-  if (!finite_nonneg(eps_lo) || !finite_nonneg(eps_hi) || !finite_nonneg(beta) || eps_lo > 1.0f)
-    return PL_ERR_ARG;
-  const int64_t N = bs * T;
-  const bool has_kl = beta != 0.0f;
-  if (N > 0) {
-    if (!X || !W || !targets || !old_lp || !adv || !mask) return PL_ERR_ARG;
-    if (H < 1 || V < 1) return PL_ERR_ARG;
-    if (has_kl && (!Xref || !Wref)) return PL_ERR_ARG;
-    if (H % 8) return PL_ERR_ALIGN;
-    if (H > (1 << 24) || V > (1ll << 31) - 1) return PL_ERR_ARG;
-    if (!aligned(X, 16) || !aligned(W, 16) || (has_kl && (!aligned(Xref, 16) || !aligned(Wref, 16))))
-      return PL_ERR_ALIGN;
-    if (bias && !aligned(bias, 2)) return PL_ERR_ALIGN;
-  }
-  const Plan plan = make_plan(bs, T, H, V, mode, dW != nullptr, dbias != nullptr);
-  if (!workspace || ws_bytes < (size_t)plan.off.total || !aligned(workspace, 256)) return PL_ERR_WORKSPACE;
-  pl_status st = check_arch();
-  if (st != PL_OK) return st;
-
+pl_status run_pipeline(const Pipe& q) {
+  const void* X = q.X; const void* W = q.W; const void* bias = q.bias; const int64_t* targets = q.targets;
+  const void* Xref = q.Xref; const void* Wref = q.Wref; const float* old_lp = q.old_lp; const void* adv = q.adv;
+  const uint8_t* mask = q.mask;
+  const int64_t bs = q.bs, T = q.T, H = q.H, V = q.V, N = bs * T;
+  const float eps_lo = q.eps_lo, eps_hi = q.eps_hi, beta = q.beta;
+  const uint32_t mode = q.mode;
+  float* loss = q.loss; void* dX = q.dX; void* dW = q.dW; void* dbias = q.dbias;
+  float* logp_out = q.logp_out; float* ref_logp_out = q.ref_logp_out; int64_t* n_valid_out = q.n_valid_out;
+  pl_stream_t stream = q.stream;
+  const DType dt = q.dt;
+  const Plan& plan = q.plan;
+  const bool has_kl = beta != 0.0f && !q.ext_g;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  unsigned char* ws = static_cast<unsigned char*>(q.workspace);
   const size_t esz = 2;
   const bool two_sided = (mode & PL_CLIP_TWO_SIDED) != 0;
-  const bool need_bwd = dX || dW || dbias;
+  const bool need_bwd = (dX || dW || dbias) && (!q.ext_g || q.grad_logp);
   auto ok = [](cudaError_t e) { return e == cudaSuccess; };
 
   if (N == 0) {
     if (dW && V > 0 && H > 0 && !ok(cudaMemsetAsync(dW, 0, (size_t)V * H * esz, s))) return PL_ERR_CUDA;
     if (dbias && V > 0 && !ok(cudaMemsetAsync(dbias, 0, (size_t)V * esz, s))) return PL_ERR_CUDA;
+    if (q.ext_g) return PL_OK;
     if (!ok(cudaMemsetAsync(ws + 16, 0, 8, s))) return PL_ERR_CUDA;
     if (!ok(launch_finalize(ws, plan.off, 0, plan.part_stride, 0, loss, n_valid_out, s))) return PL_ERR_CUDA;
     return PL_OK;
   }
 
-  if (!ok(launch_count(mask, bs, T, ws, (int)plan.nchunks, plan.off, s))) return PL_ERR_CUDA;
+  if (q.ext_g) {
+    if (!ok(launch_clear_gmax(ws, (int)plan.nchunks, plan.off, s))) return PL_ERR_CUDA;
+  } else if (!ok(launch_count(mask, bs, T, ws, (int)plan.nchunks, plan.off, s))) {
+    return PL_ERR_CUDA;
+  }
 
   const unsigned char* Xb = static_cast<const unsigned char*>(X);
   const unsigned char* Xrb = static_cast<const unsigned char*>(Xref);
@@ -165,6 +161,7 @@ pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias, c
       j.bias = nullptr; j.targets = targets + r0;
       j.part = reinterpret_cast<float2*>(ws + plan.off.part_ref); j.part_ld = plan.ntv;
       j.zt = reinterpret_cast<float*>(ws + plan.off.zt_ref); j.logits = nullptr;
+      j.logit_scale = q.inv_temp;
     }
     if (!make_tmap_2d(&fp.maps[2], Xb + r0 * H * esz, dt, H, rows, H * esz, kBK, kBM) ||
         !make_tmap_2d(&fp.maps[3], W, dt, H, V, H * esz, kBK, kBNh))
@@ -177,6 +174,7 @@ pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias, c
       j.part = reinterpret_cast<float2*>(ws + plan.off.part); j.part_ld = plan.ntv;
       j.zt = reinterpret_cast<float*>(ws + plan.off.zt);
       j.logits = need_bwd ? ws + plan.off.logits : nullptr; j.logits_ld = plan.ld;
+      j.logit_scale = q.inv_temp;
     }
     fp.njobs = nj;
     gemm_finalize_jobs(&fp);
@@ -191,7 +189,13 @@ pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias, c
     ca.lo = 1.0f - eps_lo; ca.hi = 1.0f + eps_hi; ca.beta = beta;
     ca.grpo = (mode & PL_REDUCTION_MASK) == PL_GRPO; ca.adv_lp_dtype = (mode & PL_ADV_LP_DTYPE) != 0;
     ca.bf16 = dt == DType::BF16;
-    if (!ok(launch_combine(ca, has_kl, two_sided, s))) return PL_ERR_CUDA;
+    ca.grad_logp = q.grad_logp;
+    ca.g_scale = q.inv_temp;
+    if (q.ext_g) {
+      if (!ok(launch_combine_ext(ca, s))) return PL_ERR_CUDA;
+    } else if (!ok(launch_combine(ca, has_kl, two_sided, s))) {
+      return PL_ERR_CUDA;
+    }
     last_blocks = (int)((rows + 7) / 8);
 
     if (!need_bwd) continue;
@@ -243,9 +247,110 @@ pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias, c
     if (!ok(launch_gemm(bp, dt, s))) return PL_ERR_CUDA;
   }
 
+  if (q.ext_g) return PL_OK;
   if (!ok(launch_finalize(ws, plan.off, (int)plan.nchunks, plan.part_stride, last_blocks, loss, n_valid_out, s)))
     return PL_ERR_CUDA;
   return PL_OK;
+}
+
+}  // namespace
+}  // namespace pl
+
+using namespace pl;
+
+extern "C" {
+
+size_t pl_fused_linear_grpo_workspace_bytes(int64_t bs, int64_t T, int64_t H, int64_t V, uint32_t mode,
+                                            int need_dW, int need_dbias) {
+  if (bs < 0 || T < 0 || H < 0 || V < 0) return 0;
+  return (size_t)make_plan(bs, T, H, V, mode, need_dW != 0, need_dbias != 0).off.total;
+}
+
+pl_status pl_fused_linear_grpo_temp(const void* X, const void* W, const void* bias, const int64_t* targets,
+                                    const void* Xref, const void* Wref, const float* old_lp, const void* adv,
+                                    const uint8_t* mask, int64_t bs, int64_t T, int64_t H, int64_t V,
+                                    float eps_lo, float eps_hi, float beta, float temperature, uint32_t mode,
+                                    float* loss, void* dX, void* dW, void* dbias, float* logp_out,
+                                    float* ref_logp_out, int64_t* n_valid_out, void* workspace,
+                                    size_t ws_bytes, pl_stream_t stream) {
+  if (!std::isfinite(temperature) || !(temperature > 0.0f)) return PL_ERR_ARG;
+  // ---------------- host-side validation (no device call) ----------------
+  if (bs < 0 || T < 0 || H < 0 || V < 0 || !loss) return PL_ERR_ARG;
+  if (T > 0 && bs > INT64_MAX / T) return PL_ERR_ARG;
+  if (mode & ~kFusedModeBits) return PL_ERR_ARG;
+  if ((mode & PL_REDUCTION_MASK) > PL_GRPO) return PL_ERR_ARG;
+  const uint32_t dcode = (mode & PL_DTYPE_MASK) >> 4;
+  if (dcode != 1 && dcode != 2) return PL_ERR_DTYPE;
+  const DType dt = (DType)dcode;
+  if (!finite_nonneg(eps_lo) || !finite_nonneg(eps_hi) || !finite_nonneg(beta) || eps_lo > 1.0f)
+    return PL_ERR_ARG;
+  const int64_t N = bs * T;
+  const bool has_kl = beta != 0.0f;
+  if (N > 0) {
+    if (!X || !W || !targets || !old_lp || !adv || !mask) return PL_ERR_ARG;
+    if (H < 1 || V < 1) return PL_ERR_ARG;
+    if (has_kl && (!Xref || !Wref)) return PL_ERR_ARG;
+    if (H % 8) return PL_ERR_ALIGN;
+    if (H > (1 << 24) || V > (1ll << 31) - 1) return PL_ERR_ARG;
+    if (!aligned(X, 16) || !aligned(W, 16) || (has_kl && (!aligned(Xref, 16) || !aligned(Wref, 16))))
+      return PL_ERR_ALIGN;
+    if (bias && !aligned(bias, 2)) return PL_ERR_ALIGN;
+  }
+  const Plan plan = make_plan(bs, T, H, V, mode, dW != nullptr, dbias != nullptr);
+  if (!workspace || ws_bytes < (size_t)plan.off.total || !aligned(workspace, 256)) return PL_ERR_WORKSPACE;
+  pl_status st = check_arch();
+  if (st != PL_OK) return st;
+  Pipe q{X, W, bias, targets, Xref, Wref, old_lp, adv, mask, bs, T, H, V, eps_lo, eps_hi, beta, mode,
+         loss, dX, dW, dbias, logp_out, ref_logp_out, n_valid_out, nullptr, false, 1.0f / temperature,
+         workspace, stream, dt, plan};
+  return run_pipeline(q);
+}
+
+pl_status pl_fused_linear_grpo(const void* X, const void* W, const void* bias, const int64_t* targets,
+                               const void* Xref, const void* Wref, const float* old_lp, const void* adv,
+                               const uint8_t* mask, int64_t bs, int64_t T, int64_t H, int64_t V,
+                               float eps_lo, float eps_hi, float beta, uint32_t mode, float* loss,
+                               void* dX, void* dW, void* dbias, float* logp_out, float* ref_logp_out,
+                               int64_t* n_valid_out, void* workspace, size_t ws_bytes,
+                               pl_stream_t stream) {
+  return pl_fused_linear_grpo_temp(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, bs, T, H, V, eps_lo,
+                                   eps_hi, beta, 1.0f, mode, loss, dX, dW, dbias, logp_out, ref_logp_out,
+                                   n_valid_out, workspace, ws_bytes, stream);
+}
+
+
+pl_status pl_fused_selective_logprob(const void* X, const void* W, const void* bias, const int64_t* targets,
+                                     int64_t N, int64_t H, int64_t V, uint32_t mode, const float* grad_logp,
+                                     float* logp_out, void* dX, void* dW, void* dbias, void* workspace,
+                                     size_t ws_bytes, pl_stream_t stream) {
+  if (N < 0 || H < 0 || V < 0) return PL_ERR_ARG;
+  if (mode & ~(PL_DTYPE_MASK | (0xFFu << PL_CHUNK_SHIFT))) return PL_ERR_ARG;
+  const uint32_t dcode = (mode & PL_DTYPE_MASK) >> 4;
+  if (dcode != 1 && dcode != 2) return PL_ERR_DTYPE;
+  const DType dt = (DType)dcode;
+  if ((dX || dW || dbias) && !grad_logp) return PL_ERR_ARG;
+  if (!logp_out && !dX && !dW && !dbias) return PL_ERR_ARG;
+  if (N > 0) {
+    if (!X || !W || !targets || H < 1 || V < 1) return PL_ERR_ARG;
+    if (H % 8) return PL_ERR_ALIGN;
+    if (H > (1 << 24) || V > (1ll << 31) - 1) return PL_ERR_ARG;
+    if (!aligned(X, 16) || !aligned(W, 16)) return PL_ERR_ALIGN;
+    if (bias && !aligned(bias, 2)) return PL_ERR_ALIGN;
+  }
+  const Plan plan = make_plan(1, N, H, V, mode, dW != nullptr, dbias != nullptr);
+  if (!workspace || ws_bytes < (size_t)plan.off.total || !aligned(workspace, 256)) return PL_ERR_WORKSPACE;
+  pl_status st = check_arch();
+  if (st != PL_OK) return st;
+  Pipe q{X, W, bias, targets, nullptr, nullptr, nullptr, nullptr, nullptr, 1, N, H, V, 0.0f, 0.0f, 0.0f,
+         mode, nullptr, dX, dW, dbias, logp_out, nullptr, nullptr, grad_logp, true, 1.0f, workspace, stream,
+         dt, plan};
+  return run_pipeline(q);
+}
+
+size_t pl_fused_selective_logprob_workspace_bytes(int64_t N, int64_t H, int64_t V, uint32_t mode, int need_dW,
+                                                  int need_dbias) {
+  if (N < 0 || H < 0 || V < 0) return 0;
+  return (size_t)make_plan(1, N, H, V, mode, need_dW != 0, need_dbias != 0).off.total;
 }
 
 }  // extern "C"

@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
       float term = 0.0f, dterm = 0.0f;
       if (valid)
         token_math<HAS_KL, TWO_SIDED>(logp, a.old_lp[g], ref_lp, A, a.lo, a.hi, a.beta, term, dterm);
-      const float gv = valid ? dterm * scale : 0.0f;
+      const float gv = valid ? dterm * scale * a.g_scale : 0.0f;
       contrib = valid ? term * scale : 0.0f;
       gabs = fabsf(gv);
       reinterpret_cast<float*>(a.ws + a.off.g)[i] = gv;
@@ -149,23 +149,63 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- combine (selective log-prob form)
+// One warp per row: lse from the vocabulary-tile partials, logp = z[target] - lse,
+// and g_i = grad_logp[i] supplied by the caller (the backward of the selective
+// log-prob, "Add SM100 CuTe DSL GRPO fast path": the fused-linear selective-logprob
+// autograd path receives the upstream gradient of the log-probs).
+__global__ void __launch_bounds__(256) combine_ext_kernel(CombineArgs a) {
+  __shared__ float s_gmax[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t i = (int64_t)blockIdx.x * 8 + warp;
+  float gabs = 0.0f;
+  if (i < a.rows) {
+    const int64_t g = a.row0 + i;
+    const float2* part = reinterpret_cast<const float2*>(a.ws + a.off.part) + i * a.ntv;
+    float M = -INFINITY;
+    for (int j = lane; j < a.ntv; j += 32) M = fmaxf(M, part[j].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float S = 0.0f;
+    for (int j = lane; j < a.ntv; j += 32) S += part[j].y * expf(part[j].x - M);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+    if (lane == 0) {
+      const float lse = M + logf(S);
+      const int64_t tgt = a.targets[g];
+      const bool tvalid = tgt >= 0 && tgt < a.V;
+      if (!tvalid) atomicOr(reinterpret_cast<unsigned*>(a.ws), kDevErrTarget);
+      const float zt = reinterpret_cast<const float*>(a.ws + a.off.zt)[i];
+      const float gv = (tvalid && a.grad_logp) ? a.grad_logp[g] * a.g_scale : 0.0f;
+      gabs = fabsf(gv);
+      reinterpret_cast<float*>(a.ws + a.off.g)[i] = gv;
+      reinterpret_cast<float*>(a.ws + a.off.lse)[i] = lse;
+      if (a.logp_out) a.logp_out[g] = tvalid ? zt - lse : __int_as_float(0x7fc00000);
+    }
+  }
+  if (lane == 0) s_gmax[warp] = gabs;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float gm = 0.0f;
+    for (int w = 0; w < 8; ++w) gm = fmaxf(gm, s_gmax[w]);
+    if (gm > 0.0f) atomicMax(reinterpret_cast<unsigned*>(a.ws + a.off.gmax) + a.chunk, __float_as_uint(gm));
+  }
+}
+
+__global__ void clear_gmax_kernel(unsigned char* ws, int nchunks, FusedOffsets off) {
+  unsigned* gmax = reinterpret_cast<unsigned*>(ws + off.gmax);
+  for (int c = threadIdx.x; c < nchunks; c += blockDim.x) gmax[c] = 0u;
+}
+
 // ---------------------------------------------------------------- dlogits
 // Block = 256 threads = 8 warps over a 256-column strip of the chunk's logits;
 // lane l owns columns [8l, 8l+8) of the strip, warp w rows w, w+8, ...
 template <typename T>
 __global__ void __launch_bounds__(256) dlogits_kernel(DlogitsArgs a) {
-  extern __shared__ float s_dyn[];
-  float* s_lse = s_dyn;                                    // [rows]
-  float* s_g = s_lse + a.rows;                             // [rows]
-  int* s_t = reinterpret_cast<int*>(s_g + a.rows);         // [rows]
   __shared__ float s_col[8][256];
   const unsigned char* ws = a.ws;
-  for (int64_t i = threadIdx.x; i < a.rows; i += 256) {
-    s_lse[i] = reinterpret_cast<const float*>(ws + a.off.lse)[i];
-    s_g[i] = reinterpret_cast<const float*>(ws + a.off.g)[i];
-    const int64_t tg = a.targets[a.row0 + i];
-    s_t[i] = (tg >= 0 && tg < a.V) ? (int)tg : -1;
-  }
+  const float* row_lse = reinterpret_cast<const float*>(ws + a.off.lse);
+  const float* row_g = reinterpret_cast<const float*>(ws + a.off.g);
   // power-of-two scale 2^e keeping max|dz| * 2^e <= 2^14 (fp16 range), exact to undo
   const float gm = __uint_as_float(reinterpret_cast<const unsigned*>(ws + a.off.gmax)[a.chunk]);
   int e = 0;
@@ -176,7 +216,6 @@ __global__ void __launch_bounds__(256) dlogits_kernel(DlogitsArgs a) {
   const float sc = ldexpf(1.0f, e);
   if (blockIdx.x == 0 && threadIdx.x == 0)
     reinterpret_cast<float*>(a.ws + a.off.inv_scale)[a.chunk] = ldexpf(1.0f, -e);
-  __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t col = (int64_t)blockIdx.x * 256 + lane * 8;
@@ -190,9 +229,10 @@ __global__ void __launch_bounds__(256) dlogits_kernel(DlogitsArgs a) {
 #pragma unroll 4
     for (int64_t i = warp; i < a.rows; i += 8) {
       T* p = L + i * a.ld + col;
-      const float gi = s_g[i];
-      const float lsei = s_lse[i] * kLog2e;
-      const int ti = s_t[i];
+      const float gi = __ldg(row_g + i);
+      const float lsei = __ldg(row_lse + i) * kLog2e;
+      const int64_t tg = __ldg(a.targets + a.row0 + i);
+      const int ti = (tg >= 0 && tg < a.V) ? (int)tg : -1;
       float z[8];
       if (full8) {
         uint4 u = *reinterpret_cast<const uint4*>(p);
@@ -281,18 +321,24 @@ cudaError_t launch_combine(const CombineArgs& a, bool has_kl, bool two_sided, cu
   return cudaGetLastError();
 }
 
+cudaError_t launch_combine_ext(const CombineArgs& a, cudaStream_t s) {
+  const unsigned grid = (unsigned)((a.rows + 7) / 8);
+  if (grid == 0) return cudaSuccess;
+  { launch_begin(2, s); combine_ext_kernel<<<grid, 256, 0, s>>>(a); launch_end(2, s); }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_clear_gmax(unsigned char* ws, int nchunks, const FusedOffsets& off, cudaStream_t s) {
+  { launch_begin(2, s); clear_gmax_kernel<<<1, 256, 0, s>>>(ws, nchunks, off); launch_end(2, s); }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dlogits(const DlogitsArgs& a, DType dt, cudaStream_t s) {
   const unsigned grid = (unsigned)((a.V + 255) / 256);
-  const size_t smem = (size_t)a.rows * 12;
   if (dt == DType::BF16) {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(dlogits_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
-    { launch_begin(2, s); dlogits_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(a); launch_end(2, s); }
+    { launch_begin(2, s); dlogits_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
   } else {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(dlogits_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    { launch_begin(2, s); dlogits_kernel<__half><<<grid, 256, smem, s>>>(a); launch_end(2, s); }
+    { launch_begin(2, s); dlogits_kernel<__half><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
   }
   return cudaGetLastError();
 }

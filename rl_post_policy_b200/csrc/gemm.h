@@ -42,6 +42,7 @@ struct GemmJob {
   float* zt;               // [M] target logit
   void* logits;            // [M, logits_ld] model dtype or null
   int64_t logits_ld;
+  float logit_scale;       // 1 / temperature, applied after the bias (1 for temperature 1)
   // kEpiStore
   void* out;
   int out_f32;

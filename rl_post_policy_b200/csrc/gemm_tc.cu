@@ -369,6 +369,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           const int nvalid = min(32, j.N - col0);
           if (nvalid <= 0) continue;
           if (bias) add_bias32<T>(bias + col0, v, nvalid);
+          if (j.logit_scale != 1.0f) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) v[q] *= j.logit_scale;
+          }
           if (nvalid == 32) {
             // full chunk: no per-column predicates; two columns per packed instruction
             float cmax = v[0];

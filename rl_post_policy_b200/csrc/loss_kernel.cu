@@ -129,10 +129,6 @@ __device__ __forceinline__ int64_t row_of(const LossArgs& a, int64_t t) {
   return t / a.seq;
 }
 
-// Number of nonzero bytes in a 32-bit word.
-__device__ __forceinline__ unsigned nonzero_bytes(unsigned w) {
-  return __popc((((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w) & 0x80808080u);
-}
 
 template <typename T>
 __device__ __forceinline__ float load_adv(const LossArgs& a, int64_t r) {

@@ -94,3 +94,48 @@ def test_beta_zero_allows_null_ref_validation():
     # beta == 0 and ref NULL passes validation (it then fails only for lack of a device)
     rc = _loss(ref_lp=None, beta=0.0)
     assert rc != pl.PL_ERR_ARG
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(N=-1), pl.PL_ERR_ARG),
+    (dict(X=None), pl.PL_ERR_ARG),
+    (dict(targets=None), pl.PL_ERR_ARG),
+    (dict(grad_logp=None), pl.PL_ERR_ARG),          # gradients requested without dL/dlogp
+    (dict(logp_out=None, dX=None, dW=None, dbias=None), pl.PL_ERR_ARG),  # nothing requested
+    (dict(mode=pl.PL_F32), pl.PL_ERR_DTYPE),
+    (dict(H=100), pl.PL_ERR_ALIGN),                  # 200-byte row pitch is not a multiple of 16
+    (dict(mode=pl.PL_BF16 | 1), pl.PL_ERR_ARG),      # reduction bits are not part of this entry
+    (dict(ws_bytes=16), pl.PL_ERR_WORKSPACE),
+])
+def test_selective_logprob_rejects_invalid_arguments(over, code):
+    args = dict(X=FAKE, W=FAKE, bias=None, targets=FAKE, N=64, H=128, V=512, mode=pl.PL_BF16,
+                grad_logp=FAKE, logp_out=FAKE, dX=FAKE, dW=FAKE, dbias=None, workspace=FAKE,
+                ws_bytes=1 << 40)
+    args.update(over)
+    assert pl.pl_fused_selective_logprob(**args, stream=0) == code
+
+
+def test_fused_rejects_invalid_arguments():
+    base = dict(X=FAKE, W=FAKE, bias=None, targets=FAKE, Xref=FAKE, Wref=FAKE, old_lp=FAKE, adv=FAKE,
+                mask=FAKE, bs=2, T=8, H=64, V=512, eps_lo=0.2, eps_hi=0.28, beta=0.04,
+                mode=pl.PL_BF16 | pl.PL_GRPO, loss=FAKE, dX=None, dW=None, dbias=None, logp_out=None,
+                ref_logp_out=None, n_valid_out=None, workspace=FAKE, ws_bytes=1 << 40)
+    for over, code in [(dict(loss=None), pl.PL_ERR_ARG), (dict(Wref=None), pl.PL_ERR_ARG),
+                       (dict(mode=pl.PL_F32), pl.PL_ERR_DTYPE), (dict(H=60), pl.PL_ERR_ALIGN),
+                       (dict(X=FAKE + 8), pl.PL_ERR_ALIGN), (dict(ws_bytes=1), pl.PL_ERR_WORKSPACE),
+                       (dict(eps_hi=-1.0), pl.PL_ERR_ARG), (dict(mode=pl.PL_BF16 | (1 << 10)), pl.PL_ERR_ARG)]:
+        args = dict(base)
+        args.update(over)
+        assert pl.pl_fused_linear_grpo(**args, stream=0) == code, over
+        assert pl.pl_fused_linear_grpo_temp(**args, temperature=1.0, stream=0) == code, over
+    for tau in (0.0, -1.0, float("inf"), float("nan")):
+        assert pl.pl_fused_linear_grpo_temp(**base, temperature=tau, stream=0) == pl.PL_ERR_ARG, tau
+
+
+def test_scale_rejects_invalid_arguments():
+    assert pl.pl_scale(FAKE, -1, pl.PL_BF16, FAKE, stream=0) == pl.PL_ERR_ARG
+    assert pl.pl_scale(None, 10, pl.PL_BF16, FAKE, stream=0) == pl.PL_ERR_ARG
+    assert pl.pl_scale(FAKE, 10, pl.PL_BF16, None, stream=0) == pl.PL_ERR_ARG
+    assert pl.pl_scale(FAKE, 10, 3 << 4, FAKE, stream=0) == pl.PL_ERR_DTYPE
+    assert pl.pl_scale(FAKE, 10, pl.PL_BF16 | pl.PL_GRPO, FAKE, stream=0) == pl.PL_ERR_ARG
+    assert pl.pl_scale(None, 0, pl.PL_BF16, None, stream=0) == pl.PL_OK   # nothing to do

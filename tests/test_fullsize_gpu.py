@@ -1,5 +1,6 @@
-"""Full-size parity of the fused path, in the launch configuration bench.py times
-(1024-row chunks, GRPO, eps 0.2 / 0.28).
+"""Full-size parity of the fused path, in the launch configurations bench.py times
+(GRPO, eps 0.2 / 0.28): the default 1024-row chunks with fp32 dW accumulation
+across chunks and, for multi-chunk batches, one chunk spanning the whole batch.
 
 Compared in full: every row's policy and reference log-prob (abs <= 2e-3), the
 loss (relative <= 1e-3) and the valid-token count (exact).  Sampled: dX rows
@@ -27,7 +28,7 @@ EPS_LO, EPS_HI = 0.2, 0.28
 LN_HI = float(np.log(np.float32(1) + np.float32(EPS_HI)))
 
 
-def _run(inp, d):
+def _run(inp, d, chunk=None):
     import rl_post_policy_b200 as pl
     dev = "cuda"
     bs, T, H, V, dt = d["bs"], d["T"], d["H"], d["V"], d["dtype"]
@@ -43,7 +44,7 @@ def _run(inp, d):
     lp = torch.empty(N, device=dev)
     rlp = torch.empty(N, device=dev)
     nv = torch.zeros(1, dtype=torch.int64, device=dev)
-    mode = pl.dtype_mode(dt) | pl.PL_GRPO
+    mode = pl.dtype_mode(dt) | pl.PL_GRPO | (pl.PL_CHUNK_ROWS(chunk) if chunk else 0)
     wsb = pl.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, 1, int(db is not None))
     ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
     pl.check(pl.pl_fused_linear_grpo(g["X"], g["W"], g["bias"], g["targets"], g["Xref"], g["Wref"],
@@ -75,7 +76,16 @@ def test_full_size(workload):
     if d["beta"] != 0:
         _, ref_logp, _ = oracle.lm_head_logprob(inp["Xref"], inp["Wref"], None, inp["targets"])
 
-    got = _run(inp, d)
+    runs = [_run(inp, d)]
+    if N > 1024:  # also one chunk spanning the whole batch: dW as a single K = N GEMM
+        runs.append(_run(inp, d, chunk=N))
+    for got in runs:
+        _check(inp, d, got, workload, lse, logp, ref_logp)
+
+
+def _check(inp, d, got, workload, lse, logp, ref_logp):
+    bs, T, H, V = d["bs"], d["T"], d["H"], d["V"]
+    N = bs * T
     mask = inp["mask"]
     old = inp["old_lp"].double().numpy()
     lo = oracle.policy_loss(logp.reshape(bs, T), inp["old_lp"].reshape(bs, T),

@@ -2,8 +2,9 @@
 
 Tolerances: selected log-probs abs <= 2e-3; loss relative <= 1e-3; dX, dW and
 dbias relative Frobenius <= 1e-2; the valid-token count bit-exact.  Inputs are
-seeded; a test asserts that no token sits within 1e-4 (in log space) of the clip
-bound, where fp32 and fp64 may legitimately choose different sides of the min().
+seeded; the behaviour log-probs are moved at least 2e-4 (in log space) off the
+clip bounds, where fp32 and fp64 may legitimately choose different sides of the
+min(), and a test asserts that none is left within 1e-4.
 """
 import numpy as np
 import pytest
@@ -27,7 +28,13 @@ def build_inputs(bs, T, H, V, dtype, seed, bias=False, beta=0.04, len_lo=1, len_
     inp = synth.fused_inputs(bs, T, H, V, dtype, seed, bias=bias, len_lo=len_lo, len_hi=len_hi,
                              fully_masked_last=fully_masked_last, need_ref=True)
     _, logp, _ = oracle.lm_head_logprob(inp["X"], inp["W"], inp["bias"], inp["targets"])
-    inp["old_lp"] = (torch.from_numpy(logp) + inp["old_noise"].double()).float()
+    old = torch.from_numpy(logp) + inp["old_noise"].double()
+    for bound in (np.log(float(np.float32(1) + np.float32(EPS_HI))),
+                  np.log(float(np.float32(1) - np.float32(EPS_LO)))):
+        d = torch.from_numpy(logp) - old - bound
+        near = d.abs() < 2e-4
+        old[near] -= torch.where(d[near] >= 0, 2e-4, -2e-4).double()
+    inp["old_lp"] = old.float()
     return inp
 
 
@@ -154,3 +161,50 @@ def test_bad_target_is_flagged_and_masked():
     assert got["n_valid"] == n_orig
     assert abs(got["loss"] - expect) <= 1e-3 * abs(expect)
     assert np.all(got["dX"][0] == 0.0)
+
+
+@pytest.mark.parametrize("chunk", [4096, 8192])
+def test_large_chunk_small_model(chunk):
+    # many rows in one chunk (the per-row buffers grow with the chunk), fp16 with bias
+    inp = build_inputs(36, 128, 64, 512, torch.float16, 77 + chunk, bias=True, len_lo=0, len_hi=128)
+    got = run_fused(inp, torch.float16, 1, 0.04, chunk=chunk)
+    check(inp, got, 1, 0.04)
+
+
+@pytest.mark.parametrize("tau", [0.7, 1.5])
+@pytest.mark.parametrize("chunk", [None, 128], ids=["one_chunk", "chunks128"])
+def test_temperature(tau, chunk):
+    # logits (X W^T + b) / tau for both models; gradients with respect to the raw weights
+    m = pl()
+    dev = "cuda"
+    inp = synth.fused_inputs(3, 100, 200, 1000, torch.bfloat16, 4343, bias=True, need_ref=True)
+    _, logp, _ = oracle.lm_head_logprob(inp["X"], inp["W"], inp["bias"], inp["targets"], temperature=tau)
+    old = torch.from_numpy(logp) + inp["old_noise"].double()
+    d = torch.from_numpy(logp) - old - np.log(float(np.float32(1) + np.float32(EPS_HI)))
+    old[d.abs() < 2e-4] -= 4e-4
+    inp["old_lp"] = old.float()
+    want = oracle.fused_grpo(inp["X"], inp["W"], inp["bias"], inp["targets"], inp["Xref"], inp["Wref"],
+                             inp["old_lp"].reshape(3, 100), inp["adv"], inp["mask"], eps_lo=EPS_LO,
+                             eps_hi=EPS_HI, beta=0.04, reduction=1, temperature=tau)
+    bs, T, H, V, N = 3, 100, 200, 1000, 300
+    g = {k: inp[k].to(dev) for k in ("X", "W", "bias", "targets", "Xref", "Wref", "old_lp", "adv", "mask")}
+    loss = torch.zeros(1, device=dev)
+    dX = torch.empty(N, H, dtype=torch.bfloat16, device=dev)
+    dW = torch.empty(V, H, dtype=torch.bfloat16, device=dev)
+    db = torch.empty(V, dtype=torch.bfloat16, device=dev)
+    lp, rlp = torch.empty(N, device=dev), torch.empty(N, device=dev)
+    nv = torch.zeros(1, dtype=torch.int64, device=dev)
+    mode = m.PL_BF16 | m.PL_GRPO | (m.PL_CHUNK_ROWS(chunk) if chunk else 0)
+    wsb = m.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, 1, 1)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    m.check(m.pl_fused_linear_grpo_temp(g["X"], g["W"], g["bias"], g["targets"], g["Xref"], g["Wref"],
+                                        g["old_lp"], g["adv"], g["mask"], bs, T, H, V, EPS_LO, EPS_HI, 0.04,
+                                        tau, mode, loss, dX, dW, db, lp, rlp, nv, ws, wsb))
+    torch.cuda.synchronize()
+    assert m.pl_device_status(ws) == 0
+    assert int(nv.item()) == want["n_valid"]
+    assert np.max(np.abs(lp.cpu().double().numpy() - want["logp"])) <= 2e-3
+    assert np.max(np.abs(rlp.cpu().double().numpy() - want["ref_logp"])) <= 2e-3
+    assert abs(loss.item() - want["loss"]) <= 1e-3 * abs(want["loss"])
+    for k, t in (("dX", dX), ("dW", dW), ("dbias", db)):
+        assert rel_fro(t.cpu().double().numpy(), want[k]) <= 1e-2, k

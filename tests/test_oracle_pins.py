@@ -316,3 +316,55 @@ def test_fused_beta_zero_skips_reference():
     inp2 = dict(inp, Xref=None, Wref=None)
     b = oracle.fused_grpo(**inp2, **kw)
     assert a["loss"] == b["loss"] and np.array_equal(a["dX"], b["dX"])
+
+
+@pytest.mark.parametrize("tau", [0.6, 1.7])
+def test_temperature_equals_scaled_weights(tau):
+    # logits (X W^T + b) / tau are the logits of the weights W / tau and bias b / tau
+    g = torch.Generator().manual_seed(21)
+    X = torch.randn(6, 40, generator=g, dtype=torch.float64)
+    W = 0.4 * torch.randn(90, 40, generator=g, dtype=torch.float64)
+    b = 0.1 * torch.randn(90, generator=g, dtype=torch.float64)
+    tg = torch.randint(0, 90, (6,), generator=g)
+    lse_t, lp_t, zt_t = oracle.lm_head_logprob(X, W, b, tg, temperature=tau)
+    lse_s, lp_s, zt_s = oracle.lm_head_logprob(X, W / tau, b / tau, tg)
+    np.testing.assert_allclose(lp_t, lp_s, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse_t, lse_s, rtol=0, atol=1e-12)
+    # temperature 1 is the untempered path
+    a = oracle.lm_head_logprob(X, W, b, tg, temperature=1.0)
+    c = oracle.lm_head_logprob(X, W, b, tg)
+    for x, y in zip(a, c):
+        assert np.array_equal(x, y)
+
+
+@pytest.mark.parametrize("tau", [0.7, 1.5])
+def test_tempered_gradients_match_finite_differences(tau):
+    inp, kw = _tiny_fused(14, GRPO)
+    base = oracle.fused_grpo(**inp, **kw, temperature=tau)
+    r = np.exp(base["logp"] - inp["old_lp"].reshape(-1).numpy())
+    hi = float(np.float32(1.0) + np.float32(EPS_HI))
+    assert np.all(np.abs(r - hi) > 1e-4)
+
+    def loss_with(**over):
+        d = dict(inp)
+        d.update(over)
+        return oracle.fused_grpo(**d, **kw, dx_rows=[], dw_rows=[], temperature=tau)["loss"]
+
+    h = 1e-6
+    N, H = inp["X"].shape
+    V = inp["W"].shape[0]
+    for (name, t, grad) in (("X", inp["X"], base["dX"]), ("W", inp["W"], base["dW"])):
+        fd = np.zeros(tuple(t.shape))
+        for idx in np.ndindex(*t.shape):
+            p, m = t.clone(), t.clone()
+            p[idx] += h
+            m[idx] -= h
+            fd[idx] = (loss_with(**{name: p}) - loss_with(**{name: m})) / (2 * h)
+        np.testing.assert_allclose(grad, fd, atol=1e-8, rtol=1e-5)
+    fdb = np.zeros(V)
+    for v in range(V):
+        p, m = inp["bias"].clone(), inp["bias"].clone()
+        p[v] += h
+        m[v] -= h
+        fdb[v] = (loss_with(bias=p) - loss_with(bias=m)) / (2 * h)
+    np.testing.assert_allclose(base["dbias"], fdb, atol=1e-8, rtol=1e-5)
