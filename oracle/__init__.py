@@ -64,6 +64,8 @@ def _load():
         lib.orc_lm_head_backward.argtypes = [P, I32, P, I32, P, I32, P, P, P, I64, I64,
                                              I64, I32, D, P, I64, P, P, I64, P, P]
         lib.orc_lm_head_backward.restype = I32
+        lib.orc_reverse_kl.argtypes = [P, P, I32, P, I64, I64, I32, P, P, P, P]
+        lib.orc_reverse_kl.restype = I32
         _lib = lib
     return _lib
 
@@ -205,3 +207,35 @@ def fused_grpo(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, *, eps_lo: fl
     return {"loss": lo["loss"], "abs_sum": lo["abs_sum"], "n_valid": lo["n_valid"],
             "row_valid": lo["row_valid"], "logp": logp, "ref_logp": ref_logp, "lse": lse,
             "g": g, "dX": dX, "dW": dW, "dbias": db, "dx_rows": dxr, "dw_rows": dwr}
+
+
+def reverse_kl(student, teacher, mask=None, *, want_grad: bool = True, nthreads: int = 0) -> dict:
+    """Reverse-KL self-distillation KL(softmax(student) || softmax(teacher)) per row,
+    masked mean over rows (denominator max(n_valid, 1)), and its gradient with
+    respect to the student logits, all in fp64.
+
+    ``student``, ``teacher``: (..., V) of one float dtype (decoded exactly);
+    ``mask``: shape of the leading dims, nonzero = valid, or None (all valid).
+    Returns loss, grad (same shape as student, or None), kl_rows (leading
+    shape; every row) and n_valid.
+    """
+    s = _t(student)
+    t = _t(teacher)
+    if s.shape != t.shape or s.dtype != t.dtype:
+        raise ValueError("oracle: student and teacher must share shape and dtype")
+    lead = tuple(s.shape[:-1])
+    V = int(s.shape[-1])
+    N = int(np.prod(lead)) if lead else 1
+    m = None
+    if mask is not None:
+        m = _t(mask, False).to(torch.bool).to(torch.uint8).reshape(N).contiguous()
+    loss = np.zeros(1)
+    grad = np.zeros((N, V)) if want_grad else None
+    kl = np.zeros(max(N, 1))
+    nv = np.zeros(1, dtype=np.int64)
+    rc = _load().orc_reverse_kl(_p(s), _p(t), _DT[s.dtype], _p(m), N, V, nthreads, _p(loss),
+                                _p(grad), _p(kl), _p(nv))
+    if rc:
+        raise ValueError(f"oracle: reverse_kl rejected its arguments (rc={rc})")
+    return {"loss": float(loss[0]), "grad": None if grad is None else grad.reshape(lead + (V,)),
+            "kl_rows": kl[:N].reshape(lead), "n_valid": int(nv[0])}

@@ -20,6 +20,12 @@
 //   * lm_head_backward -- the chain rule through log-softmax and the linear layer:
 //                      dz = g * (onehot(target) - softmax(z)), dX = dz W,
 //                      dW = dz^T X, dbias = sum over rows of dz.
+//   * reverse_kl    -- reverse-KL self-distillation of the "Geometric-AI Kernels"
+//                      model card, section "Reverse KL": p = softmax(student row),
+//                      q = softmax(teacher row), kl_r = sum_v p_v (log p_v - log q_v),
+//                      loss = sum_r mask_r kl_r / n_valid, and the gradient with
+//                      respect to the student logits
+//                      mask_r / n_valid * p_v (log p_v - log q_v - kl_r).
 //
 // Everything is fp64.  Low-precision inputs (binary16, bfloat16, binary32) are
 // decoded exactly by the decoders below, written from the IEEE-754 / bfloat16
@@ -37,6 +43,9 @@
 //     A*r <= A*clip(r), else 0;
 //   * a mask entry counts as valid when it is nonzero;
 //   * GRPO divides by bs, counting fully masked rows (which contribute 0).
+//   * reverse KL divides by max(n_valid, 1): the card leaves the all-masked
+//     batch undefined (inf/NaN); clamping makes it loss 0, gradient 0, and
+//     changes nothing when any row is valid.
 
 #include <cmath>
 #include <cstdint>
@@ -420,6 +429,57 @@ int orc_lm_head_backward(const void* X, int xdt, const void* W, int wdt,
       }
     });
   }
+  return 0;
+}
+
+// Reverse-KL self-distillation over N rows of V logits.
+//   student, teacher: [N, V] (dtype dt, decoded exactly); mask [N] (nonzero =
+//   valid) or NULL (every row valid).
+//   Per row, in fp64 and natural v order:
+//     log p_v = s_v - lse(s),  log q_v = t_v - lse(t)
+//     (lse(x) = M + log(sum_v exp(x_v - M)), M = max_v x_v),
+//     kl_r = sum_v p_v (log p_v - log q_v).
+//   loss = sum_r [mask_r != 0] kl_r / max(n_valid, 1).
+//   grad (if not NULL) [N, V]: [mask_r != 0] / max(n_valid, 1) * p_v * (log p_v - log q_v - kl_r).
+//   kl_rows (if not NULL) [N]: kl_r of every row, masked or not.
+int orc_reverse_kl(const void* student, const void* teacher, int dt, const uint8_t* mask,
+                   int64_t N, int64_t V, int nthreads, double* loss_out, double* grad,
+                   double* kl_rows, int64_t* n_valid_out) {
+  if (!student || !teacher || !loss_out || N < 0 || V <= 0) return 1;
+  int64_t n = 0;
+  for (int64_t r = 0; r < N; ++r) n += (!mask || mask[r] != 0) ? 1 : 0;
+  const double inv_n = 1.0 / (double)std::max<int64_t>(n, 1);
+  std::vector<double> kl(N > 0 ? N : 1, 0.0);
+  parallel_ranges(N, worker_count(nthreads), [&](int, int64_t rb, int64_t re) {
+    std::vector<double> ls(V), lq(V);
+    for (int64_t r = rb; r < re; ++r) {
+      load_row(dt, student, r * V, V, ls.data());
+      load_row(dt, teacher, r * V, V, lq.data());
+      for (std::vector<double>* x : {&ls, &lq}) {
+        double M = -INFINITY;
+        for (int64_t v = 0; v < V; ++v) M = std::max(M, (*x)[v]);
+        double S = 0.0;
+        for (int64_t v = 0; v < V; ++v) S += std::exp((*x)[v] - M);
+        const double lse = M + std::log(S);
+        for (int64_t v = 0; v < V; ++v) (*x)[v] -= lse;
+      }
+      double k = 0.0;
+      for (int64_t v = 0; v < V; ++v) k += std::exp(ls[v]) * (ls[v] - lq[v]);
+      kl[r] = k;
+      if (grad) {
+        const double scale = (!mask || mask[r] != 0) ? inv_n : 0.0;
+        double* gr = grad + r * V;
+        for (int64_t v = 0; v < V; ++v) gr[v] = scale * std::exp(ls[v]) * (ls[v] - lq[v] - k);
+      }
+    }
+  });
+  double sum = 0.0;
+  for (int64_t r = 0; r < N; ++r)
+    if (!mask || mask[r] != 0) sum += kl[r];
+  *loss_out = sum * inv_n;
+  if (kl_rows)
+    for (int64_t r = 0; r < N; ++r) kl_rows[r] = kl[r];
+  if (n_valid_out) *n_valid_out = n;
   return 0;
 }
 
