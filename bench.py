@@ -41,6 +41,7 @@ EPS_LO, EPS_HI = 0.2, 0.28
 GEMM_SOURCES = ["rl_post_policy_b200/csrc/gemm_tc.cu", "rl_post_policy_b200/csrc/sm100.cuh",
                 "rl_post_policy_b200/csrc/gemm.h"]
 LOSS_SOURCES = ["rl_post_policy_b200/csrc/loss_kernel.cu", "rl_post_policy_b200/csrc/policy_math.cuh"]
+RKL_SOURCES = ["rl_post_policy_b200/csrc/reverse_kl.cu"]
 
 
 def parse():
@@ -53,6 +54,10 @@ def parse():
     ap.add_argument("--chunk-rows", type=int, default=-1,
                     help="rows per chunk (multiple of 128); -1: the whole batch in one chunk")
     ap.add_argument("--no-loss-only", action="store_true")
+    ap.add_argument("--no-reverse-kl", action="store_true")
+    ap.add_argument("--only", choices=["reverse_kl", "loss_only"], default=None,
+                    help="run one side measurement alone and print its JSON (for profiling)")
+    ap.add_argument("--reps", type=int, default=30, help="timed calls per side measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256, help="rows in the oracle's timed sample")
     ap.add_argument("--ref-rows", type=int, default=4, help="rows per step of the reference (oracle) arm")
@@ -325,6 +330,64 @@ def loss_only(peaks, peak_kind):
     }
 
 
+# ------------------------------------------------------------------ reverse KL
+def reverse_kl(peaks, peak_kind, reps=30):
+    """Reverse-KL self-distillation at the model card's example shape (bs=4,
+    seq=256, V=248320, bf16, ~1 GB of logits per call, far larger than L2):
+    forward+gradient and forward-only, CUDA events around each launch."""
+    import rl_post_policy_b200 as pl
+    import synth
+    w = synth.RKL_WORKLOADS[1]
+    bs, seq, V = w["bs"], w["seq"], w["V"]
+    N = bs * seq
+    inp = synth.reverse_kl_inputs(bs, seq, V, w["dtype"], synth.seed_for(46, 1), device="cuda")
+    s, t, m = inp["student"], inp["teacher"], inp["mask"]
+    n_valid = int(m.sum().item())
+    g = torch.empty_like(s)
+    loss = torch.zeros(1, device="cuda")
+    wsb = pl.pl_reverse_kl_workspace_bytes(N, V)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    esz = s.element_size()
+    res = {}
+    for name, grad in (("fwd_bwd", g), ("fwd", None)):
+        def call():
+            pl.pl_reverse_kl(s, t, m, N, V, pl.PL_BF16, loss, grad, None, None, ws, wsb)
+
+        for _ in range(min(3, reps)):
+            call()
+        torch.cuda.synchronize()
+        pl.pl_debug_timing_read()
+        pl.pl_debug_timing(True)
+        for _ in range(reps):
+            call()
+        torch.cuda.synchronize()
+        pl.pl_debug_timing(False)
+        ms, n = pl.pl_debug_timing_read()
+        per = ms[2] / max(n[2], 1)
+        # valid rows: read student + teacher (+ write the gradient); masked rows: the zero
+        # gradient only; plus the mask
+        bytes_ = n_valid * V * esz * (3 if grad is not None else 2) + N
+        if grad is not None:
+            bytes_ += (N - n_valid) * V * esz
+        res[name] = {"us_per_call": per * 1e3, "GB_per_s": bytes_ / (per * 1e-3) / 1e9,
+                     "rows_per_s": N / (per * 1e-3), "algorithmic_bytes": bytes_}
+    del s, t, g, inp
+    peak = float(peaks["hbm_gbs"])
+    fb = res["fwd_bwd"]
+    return {
+        "metric": "reverse-KL GB/s", "value": fb["GB_per_s"], "unit": "GB/s",
+        "workload": f"reverse KL fwd+grad, bf16, bs={bs} x seq={seq}, V={V}, mask uniform>0.2 "
+                    f"({n_valid} valid rows)",
+        "roofline": {"bound": "hbm", "achieved": fb["GB_per_s"], "peak": peak, "unit": "GB/s",
+                     "frac": fb["GB_per_s"] / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                     "traffic": recorded_traffic("reverse_kl_kernel_grad", RKL_SOURCES)},
+        "us_per_call": fb["us_per_call"],
+        "forward_only": {"us_per_call": res["fwd"]["us_per_call"], "GB_per_s": res["fwd"]["GB_per_s"],
+                         "frac": res["fwd"]["GB_per_s"] / peak,
+                         "traffic": recorded_traffic("reverse_kl_kernel_fwd", RKL_SOURCES)},
+    }
+
+
 # ------------------------------------------------------------------ CPU oracle
 def oracle_sample(inp, d, rows):
     """The fp64 oracle on the first `rows` rows of the batch (one sequence of
@@ -385,6 +448,11 @@ def run_ours(args):
     ws_world, rank = dist_init(args)
     import rl_post_policy_b200 as pl
     peaks, peak_kind = load_peaks()
+    if args.only:
+        if rank == 0:
+            out = reverse_kl(peaks, peak_kind, args.reps) if args.only == "reverse_kl" else loss_only(peaks, peak_kind)
+            print(json.dumps(out), flush=True)
+        return
     d, inp, ws, wsb, mode = make_fused_inputs(args.workload, rank, args.chunk_rows)
     step = FusedStep(d, inp, ws, wsb, mode)
     N, H, V = d["N"], d["H"], d["V"]
@@ -453,6 +521,8 @@ def run_ours(args):
     extra = {}
     if rank == 0 and ws_world == 1 and not args.no_loss_only:
         extra["loss_only"] = loss_only(peaks, peak_kind)
+    if rank == 0 and ws_world == 1 and not args.no_reverse_kl:
+        extra["reverse_kl"] = reverse_kl(peaks, peak_kind, args.reps)
     cpu = None
     if rank == 0 and ws_world == 1 and not args.no_cpu_baseline:
         rows = max(1, min(args.cpu_rows, N))

@@ -246,6 +246,40 @@ pl_status pl_fused_selective_logprob(const void* X, const void* W, const void* b
 size_t pl_fused_selective_logprob_workspace_bytes(int64_t N, int64_t H, int64_t V, uint32_t mode,
                                                   int need_dW, int need_dbias);
 
+/* pl_reverse_kl: reverse-KL self-distillation ("Geometric-AI Kernels" model card,
+ * section "Reverse KL"), forward and, when grad_out is not NULL, the gradient
+ * with respect to the student logits, in one launch:
+ *   p = softmax(student[r,:]), q = softmax(teacher[r,:]),
+ *   kl_r = sum_v p_v (log p_v - log q_v),
+ *   loss = sum_r [mask_r != 0] kl_r / max(n_valid, 1),
+ *   grad[r,v] = [mask_r != 0] / max(n_valid, 1) * p_v (log p_v - log q_v - kl_r).
+ * The card divides by n_valid unclamped (an all-masked batch gives inf/NaN);
+ * here the denominator is max(n_valid, 1), so that batch gives loss 0 and a zero
+ * gradient, and every other batch is unchanged.
+ *   student, teacher [N, V] : one dtype, mode bits 4-7 (PL_F32 / PL_F16 / PL_BF16);
+ *                             no other mode bit may be set.  Finite logits.
+ *   mask [N] uint8/bool, nonzero = valid, or NULL (every row valid).
+ *   loss_out : device fp32 scalar.      grad_out [N, V] student dtype, or NULL (forward only).
+ *   kl_rows_out [N] fp32 or NULL : kl_r of each valid row, 0 for masked rows.
+ *   n_valid_out : device int64 or NULL.
+ *   workspace : pl_reverse_kl_workspace_bytes() bytes, 256-byte aligned and
+ *               zero-filled once after allocation; NULL uses a library-owned one
+ *               for (device, stream).  Calls sharing a workspace are stream-ordered.
+ * Rows that are masked are not read.  Any element alignment is accepted; the
+ * 16-byte vector path runs when student, teacher and grad share their address
+ * modulo 16.  N = 0 writes loss 0 (student and teacher may then be NULL).
+ * Errors: PL_ERR_ARG (NULL loss_out, NULL student/teacher with N > 0, N < 0, V < 1,
+ * unknown mode bits), PL_ERR_DTYPE, PL_ERR_ALIGN (a pointer not aligned to its
+ * element, or a workspace not 256-byte aligned), PL_ERR_WORKSPACE, PL_ERR_ARCH,
+ * PL_ERR_CUDA; all are returned before any launch.
+ */
+pl_status pl_reverse_kl(const void* student, const void* teacher, const uint8_t* mask, int64_t N,
+                        int64_t V, uint32_t mode, float* loss_out, void* grad_out,
+                        float* kl_rows_out, int64_t* n_valid_out, void* workspace, size_t ws_bytes,
+                        pl_stream_t stream);
+
+size_t pl_reverse_kl_workspace_bytes(int64_t N, int64_t V);
+
 /* pl_scale: x[i] *= *scale for n elements of the mode's dtype (bits 4-7), in place
  * on `stream`; `scale` is a device fp32 scalar, so the host never waits.  It
  * carries the chain rule for the autograd wrappers: the gradient of a scalar

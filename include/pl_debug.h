@@ -51,6 +51,13 @@ pl_status pl_debug_timing_read(double* ms, int64_t* launches);
 void pl_debug_set_wait(unsigned long long wait_ns, unsigned extra_arrivals, unsigned extra_tx);
 
 /*
+ * Forces the reverse-KL kernel's cluster size (CTAs sharing one row: 1, 2, 4 or
+ * 8) for later calls on this process, so tests reach every row split; 0
+ * restores the host's choice.  Returns PL_ERR_ARG for any other value.
+ */
+int pl_debug_set_rkl_cluster(int cl);
+
+/*
  * The persistent GEMM's tile schedule, for a host-side check: two problems of
  * t0 tiles (c0 k-steps each) and t1 tiles (c1 k-steps each) over `pairs` CTA
  * pairs.  out_pair[t] (t0 + t1 entries) receives the pair that runs tile t.

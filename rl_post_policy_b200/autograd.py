@@ -5,6 +5,9 @@
   fused forward+backward kernel (pl_loss_ex) registered with autograd, so
   ``loss.backward()`` works.  The forward keeps dLoss/dlp; the backward scales
   it by the incoming gradient with pl_scale (a device scalar, no host sync).
+* ``reverse_kl_autograd`` -- the card's autograd-aware reverse-KL entry point:
+  pl_reverse_kl's fused forward + student-logit gradient, scaled by the
+  incoming gradient in the backward (pl_scale).
 * ``fused_selective_logprob`` -- the fused-linear selective log-prob autograd
   path of "Add SM100 CuTe DSL GRPO fast path" (Liger-Kernel PR #1363,
   "Summary"): forward = pl_fused_selective_logprob (log-probs), backward = the
@@ -72,6 +75,37 @@ def grpo_loss_autograd(policy_lp, old_lp, ref_lp, adv, mask, epsilon=0.2, epsilo
     """GRPO loss (per-sequence mean, then batch mean) with autograd support."""
     return _PolicyLoss.apply(policy_lp, old_lp, ref_lp, adv, mask, float(epsilon), float(epsilon_high),
                              float(beta), pl.PL_GRPO, bool(two_sided))
+
+
+class _ReverseKL(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, student, teacher, mask):
+        V = student.shape[-1]
+        N = student.numel() // V if V else 0
+        s = student.detach().contiguous()
+        t = teacher.detach().to(s.dtype).contiguous()
+        m = mask.detach().to(torch.uint8).contiguous() if mask is not None else None
+        grad = torch.empty_like(s)
+        loss = torch.empty(1, dtype=torch.float32, device=s.device)
+        pl.check(pl.pl_reverse_kl(s, t, m, N, V, pl.dtype_mode(s.dtype), loss, grad, None, None, None, 0),
+                 "pl_reverse_kl")
+        ctx.save_for_backward(grad)
+        ctx.mode = pl.dtype_mode(s.dtype)
+        return loss[0]
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        (grad,) = ctx.saved_tensors
+        g = grad.clone()
+        scale = grad_out.detach().to(torch.float32).reshape(1).contiguous()
+        pl.check(pl.pl_scale(g, g.numel(), ctx.mode, scale), "pl_scale")
+        return g, None, None
+
+
+def reverse_kl_autograd(student_logits, teacher_logits, completions_mask=None):
+    """Masked mean over rows of KL(softmax(student) || softmax(teacher)), differentiable
+    in the student logits (shape (..., V); mask of the leading shape, or None)."""
+    return _ReverseKL.apply(student_logits, teacher_logits, completions_mask)
 
 
 class _SelectiveLogprob(torch.autograd.Function):

@@ -62,6 +62,10 @@ _lib.pl_fused_selective_logprob.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _U
 _lib.pl_fused_selective_logprob.restype = _I
 _lib.pl_fused_selective_logprob_workspace_bytes.argtypes = [_I64, _I64, _I64, _U32, _I, _I]
 _lib.pl_fused_selective_logprob_workspace_bytes.restype = _SZ
+_lib.pl_reverse_kl.argtypes = [_P, _P, _P, _I64, _I64, _U32, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.pl_reverse_kl.restype = _I
+_lib.pl_reverse_kl_workspace_bytes.argtypes = [_I64, _I64]
+_lib.pl_reverse_kl_workspace_bytes.restype = _SZ
 _lib.pl_scale.argtypes = [_P, _I64, _U32, _P, _P]
 _lib.pl_scale.restype = _I
 _lib.pl_device_status.argtypes = [_P, _P]
@@ -80,14 +84,16 @@ _lib.pl_debug_set_wait.argtypes = [ctypes.c_ulonglong, ctypes.c_uint, ctypes.c_u
 _lib.pl_debug_set_wait.restype = None
 _lib.pl_debug_pair_tiles.argtypes = [_I, _I, _I, _I, _I, _P]
 _lib.pl_debug_pair_tiles.restype = _I
+_lib.pl_debug_set_rkl_cluster.argtypes = [_I]
+_lib.pl_debug_set_rkl_cluster.restype = _I
 _lib.pl_debug_launch_count.argtypes = []
 _lib.pl_debug_launch_count.restype = _I64
 
 EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_linear_grpo_temp", "pl_fused_selective_logprob",
-            "pl_fused_selective_logprob_workspace_bytes", "pl_scale", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
+            "pl_fused_selective_logprob_workspace_bytes", "pl_reverse_kl", "pl_reverse_kl_workspace_bytes", "pl_scale", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
             "pl_version", "pl_debug_gemm", "pl_debug_timing", "pl_debug_timing_read",
-            "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_pair_tiles")
+            "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_pair_tiles")
 
 
 class PLError(RuntimeError):
@@ -189,6 +195,17 @@ def pl_fused_selective_logprob_workspace_bytes(N, H, V, mode, need_dW, need_dbia
                                                                int(need_dbias)))
 
 
+def pl_reverse_kl(student, teacher, mask, N, V, mode, loss_out, grad_out, kl_rows_out, n_valid_out, workspace,
+                  ws_bytes, stream=None) -> int:
+    return _lib.pl_reverse_kl(_ptr(student), _ptr(teacher), _ptr(mask), N, V, mode, _ptr(loss_out),
+                              _ptr(grad_out), _ptr(kl_rows_out), _ptr(n_valid_out), _ptr(workspace), ws_bytes,
+                              _stream(stream))
+
+
+def pl_reverse_kl_workspace_bytes(N, V) -> int:
+    return _lib.pl_reverse_kl_workspace_bytes(N, V)
+
+
 def pl_scale(x, n, mode, scale, stream=None) -> int:
     return _lib.pl_scale(_ptr(x), n, mode, _ptr(scale), _stream(stream))
 
@@ -230,6 +247,10 @@ def pl_debug_launch_count() -> int:
 def pl_debug_set_wait(wait_ns: int, extra_arrivals: int = 0, extra_tx: int = 0) -> None:
     """Test knob (include/pl_debug.h): wait bound and wait-run-out injection."""
     _lib.pl_debug_set_wait(int(wait_ns), int(extra_arrivals), int(extra_tx))
+
+
+def pl_debug_set_rkl_cluster(cl: int) -> int:
+    return _lib.pl_debug_set_rkl_cluster(cl)
 
 
 def pl_debug_pair_tiles(t0: int, t1: int, c0: int, c1: int, pairs: int):

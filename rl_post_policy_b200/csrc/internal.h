@@ -99,6 +99,7 @@ struct DebugKnobs {
   unsigned long long wait_ns = kWaitLimitNs;
   unsigned extra_arrivals = 0;
   unsigned extra_tx = 0;
+  int rkl_cluster = 0;   // reverse-KL CTAs per cluster (1, 2, 4 or 8; 0 = the host's choice)
 };
 DebugKnobs& debug_knobs();
 

@@ -16,7 +16,11 @@ integers includes both ends):
 * fused linear: X ~ N(0,1) [N,H], W ~ N(0,0.02) [V,H], Xref = X + N(0,0.01),
   Wref = W + N(0,0.002), optional bias ~ N(0,0.01), targets uniform in [0,V),
   advantages N(0,1) per sequence, prefix mask, and the N(0,0.1) noise that is
-  added to the policy log-prob to make the behaviour log-probs (old_lp).
+  added to the policy log-prob to make the behaviour log-probs (old_lp);
+* reverse KL: student logits N(0,1) [bs, seq, V]; teacher logits independent
+  N(0,1), or (``teacher_std`` given) student + N(0, teacher_std) for a teacher
+  close to the student; mask = uniform(0,1) > 0.2 per token (as the model card's
+  reverse-KL example draws it).
 
 Seeds are ``0x5EED0000 + 16*workload + variant``.
 """
@@ -104,6 +108,27 @@ def fused_inputs(bs: int, T: int, H: int, V: int, dtype: torch.dtype, seed: int,
     out["mask"] = prefix_mask(lens, T)
     out["old_noise"] = normal((N,), s + 9, std=0.1, device=device)
     return out
+
+
+def reverse_kl_inputs(bs: int, seq: int, V: int, dtype: torch.dtype, seed: int, *,
+                      teacher_std: float | None = None, device="cpu") -> dict:
+    s = int(seed)
+    student = normal((bs, seq, V), s + 1, device=device)
+    if teacher_std is None:
+        teacher = normal((bs, seq, V), s + 2, device=device)
+    else:
+        teacher = student + normal((bs, seq, V), s + 2, std=teacher_std, device=device)
+    u = torch.rand((bs, seq), generator=_gen(s + 3, device), device=device)
+    return {"student": student.to(dtype), "teacher": teacher.to(dtype), "mask": (u > 0.2).to(torch.uint8)}
+
+
+# Reverse-KL workloads: the model card's example shape (bs=4, seq=256,
+# V=248320) and the fused path's vocabulary at a loss-only-sized batch.
+RKL_WORKLOADS = {
+    0: dict(bs=2, seq=8, V=1000, dtype=torch.bfloat16),
+    1: dict(bs=4, seq=256, V=248320, dtype=torch.bfloat16),
+    2: dict(bs=16, seq=128, V=128256, dtype=torch.bfloat16),
+}
 
 
 # The workloads, by number, as (kind, shape) records.

@@ -139,3 +139,29 @@ def test_scale_rejects_invalid_arguments():
     assert pl.pl_scale(FAKE, 10, 3 << 4, FAKE, stream=0) == pl.PL_ERR_DTYPE
     assert pl.pl_scale(FAKE, 10, pl.PL_BF16 | pl.PL_GRPO, FAKE, stream=0) == pl.PL_ERR_ARG
     assert pl.pl_scale(None, 0, pl.PL_BF16, None, stream=0) == pl.PL_OK   # nothing to do
+
+
+def _rkl(**over):
+    args = dict(student=FAKE, teacher=FAKE, mask=None, N=8, V=512, mode=pl.PL_BF16, loss_out=FAKE,
+                grad_out=FAKE, kl_rows_out=None, n_valid_out=None, workspace=FAKE * 16,
+                ws_bytes=pl.pl_reverse_kl_workspace_bytes(8, 512))
+    args.update(over)
+    return pl.pl_reverse_kl(**args, stream=0)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(student=None), pl.PL_ERR_ARG), (dict(teacher=None), pl.PL_ERR_ARG),
+    (dict(loss_out=None), pl.PL_ERR_ARG), (dict(N=-1), pl.PL_ERR_ARG), (dict(V=0), pl.PL_ERR_ARG),
+    (dict(mode=pl.PL_BF16 | pl.PL_GRPO), pl.PL_ERR_ARG), (dict(mode=3 << 4), pl.PL_ERR_DTYPE),
+    (dict(student=FAKE + 1), pl.PL_ERR_ALIGN), (dict(grad_out=FAKE + 1), pl.PL_ERR_ALIGN),
+    (dict(mode=pl.PL_F32, teacher=FAKE + 2), pl.PL_ERR_ALIGN), (dict(workspace=FAKE + 16), pl.PL_ERR_ALIGN),
+    (dict(ws_bytes=100), pl.PL_ERR_WORKSPACE),
+])
+def test_reverse_kl_rejects_invalid_arguments(over, code):
+    assert _rkl(**over) == code
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="would launch on fake pointers")
+def test_reverse_kl_valid_call_without_device():
+    # element-aligned (not 16-byte aligned) pointers and a NULL workspace pass validation
+    assert _rkl(student=FAKE + 2, workspace=None, ws_bytes=0) in (pl.PL_ERR_CUDA, pl.PL_ERR_ARCH)
