@@ -288,6 +288,20 @@ size_t pl_reverse_kl_workspace_bytes(int64_t N, int64_t V);
  */
 pl_status pl_scale(void* x, int64_t n, uint32_t mode, const float* scale, pl_stream_t stream);
 
+/* pl_count_ratio: *factor_out = max(*local, 1) / max(*global_, 1) (fp32), all three
+ * device scalars, computed on `stream` with no host synchronisation.
+ * Data-parallel callers shard the sequences over ranks.  A rank's loss and
+ * gradients come out of the fused call normalised by its own count: its
+ * valid-token count n_l for BNPO, its sequence count bs_l for GRPO.  Times this
+ * factor (with the all-reduced global count), they are the rank's exact share of
+ * the global BNPO / GRPO loss of the "Geometric-AI Kernels" card ("BNPO Loss":
+ * sum / max(n, 1); "GRPO Loss": mean over sequences), and summing the shares
+ * over ranks gives the loss and dW / dbias of the whole batch.
+ * Errors: PL_ERR_ARG (a NULL pointer), PL_ERR_ARCH, PL_ERR_CUDA.
+ */
+pl_status pl_count_ratio(const int64_t* local, const int64_t* global_, float* factor_out,
+                         pl_stream_t stream);
+
 /* ---- status ---------------------------------------------------------------------
  * pl_device_status: synchronises `stream`, reads the sticky device error flag of
  * `workspace` (NULL = pl_loss's own scratch for the current device and `stream`),

@@ -66,6 +66,8 @@ _lib.pl_reverse_kl.argtypes = [_P, _P, _P, _I64, _I64, _U32, _P, _P, _P, _P, _P,
 _lib.pl_reverse_kl.restype = _I
 _lib.pl_reverse_kl_workspace_bytes.argtypes = [_I64, _I64]
 _lib.pl_reverse_kl_workspace_bytes.restype = _SZ
+_lib.pl_count_ratio.argtypes = [_P, _P, _P, _P]
+_lib.pl_count_ratio.restype = _I
 _lib.pl_scale.argtypes = [_P, _I64, _U32, _P, _P]
 _lib.pl_scale.restype = _I
 _lib.pl_device_status.argtypes = [_P, _P]
@@ -90,7 +92,7 @@ _lib.pl_debug_launch_count.argtypes = []
 _lib.pl_debug_launch_count.restype = _I64
 
 EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_linear_grpo_temp", "pl_fused_selective_logprob",
-            "pl_fused_selective_logprob_workspace_bytes", "pl_reverse_kl", "pl_reverse_kl_workspace_bytes", "pl_scale", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
+            "pl_fused_selective_logprob_workspace_bytes", "pl_reverse_kl", "pl_reverse_kl_workspace_bytes", "pl_scale", "pl_count_ratio", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
             "pl_version", "pl_debug_gemm", "pl_debug_timing", "pl_debug_timing_read",
             "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_pair_tiles")
@@ -208,6 +210,10 @@ def pl_reverse_kl_workspace_bytes(N, V) -> int:
 
 def pl_scale(x, n, mode, scale, stream=None) -> int:
     return _lib.pl_scale(_ptr(x), n, mode, _ptr(scale), _stream(stream))
+
+
+def pl_count_ratio(local, global_, factor_out, stream=None) -> int:
+    return _lib.pl_count_ratio(_ptr(local), _ptr(global_), _ptr(factor_out), _stream(stream))
 
 
 def pl_device_status(workspace=None, stream=None) -> int:

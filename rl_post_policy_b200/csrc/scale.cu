@@ -23,6 +23,11 @@ __global__ void scale_kernel(T* x, int64_t n, const float* scale) {
   }
 }
 
+__global__ void count_ratio_kernel(const int64_t* local, const int64_t* global_, float* out) {
+  const int64_t l = *local, g = *global_;
+  out[0] = (float)((double)(l > 1 ? l : 1) / (double)(g > 1 ? g : 1));
+}
+
 }  // namespace
 }  // namespace pl
 
@@ -45,6 +50,18 @@ extern "C" pl_status pl_scale(void* x, int64_t n, uint32_t mode, const float* sc
   if (d == 0) scale_kernel<float><<<grid, 256, 0, s>>>(static_cast<float*>(x), n, scale);
   else if (d == 1) scale_kernel<__half><<<grid, 256, 0, s>>>(static_cast<__half*>(x), n, scale);
   else scale_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<__nv_bfloat16*>(x), n, scale);
+  launch_end(2, s);
+  return cudaGetLastError() == cudaSuccess ? PL_OK : PL_ERR_CUDA;
+}
+
+extern "C" pl_status pl_count_ratio(const int64_t* local, const int64_t* global_, float* factor_out,
+                                    pl_stream_t stream) {
+  if (!local || !global_ || !factor_out) return PL_ERR_ARG;
+  pl_status st = check_arch();
+  if (st != PL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  launch_begin(2, s);
+  count_ratio_kernel<<<1, 1, 0, s>>>(local, global_, factor_out);
   launch_end(2, s);
   return cudaGetLastError() == cudaSuccess ? PL_OK : PL_ERR_CUDA;
 }

@@ -1,0 +1,98 @@
+"""The data-parallel step (rl_post_policy_b200.parallel) on two `gloo` CPU ranks.
+
+Each rank takes its share of the sequences of one seeded batch (2 and 3 of 5).  The per-rank
+operations are the CPU oracle (the fused loss and gradients of the rank's
+shard, normalised by the shard's own count) and plain tensor arithmetic for
+the ratio and the scale, so what is under test is the host-side sequence: the
+count all-reduce, each rank's share and the loss / dW / dbias all-reduce.  The
+result must equal the oracle on the whole batch, for BNPO (global valid-token
+denominator) and GRPO (global sequence mean), with unequal shard sizes and a
+fully masked sequence.
+"""
+import os
+import socket
+import subprocess
+import sys
+import textwrap
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+SCRIPT = textwrap.dedent("""
+    import os, sys
+    sys.path.insert(0, {root!r})
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import oracle, synth
+    from rl_post_policy_b200 import parallel
+    import rl_post_policy_b200.binding as pl
+
+    rank, ws = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    red = {red}
+    bs, T, H, V = 5, 12, 32, 96
+    inp = synth.fused_inputs(bs, T, H, V, torch.float32, 4711, bias=True, len_lo=0, len_hi=T,
+                             fully_masked_last=True, need_ref=True)
+    _, logp, _ = oracle.lm_head_logprob(inp["X"], inp["W"], inp["bias"], inp["targets"])
+    inp["old_lp"] = (torch.from_numpy(logp) + inp["old_noise"].double()).float()
+    want = oracle.fused_grpo(inp["X"], inp["W"], inp["bias"], inp["targets"], inp["Xref"], inp["Wref"],
+                             inp["old_lp"].reshape(bs, T), inp["adv"], inp["mask"], eps_lo=0.2, eps_hi=0.28,
+                             beta=0.04, reduction=red)
+    seqs = [range(0, 2), range(2, 5)][rank]          # unequal shards; rank 1 holds the empty sequence
+    rows = [r * T + t for r in seqs for t in range(T)]
+
+    class OracleOps:
+        def local_step(self, X, W, bias, targets, Xref, Wref, old_lp, adv, mask, eps_lo, eps_hi, beta,
+                       reduction, **kw):
+            o = oracle.fused_grpo(X, W, bias, targets, Xref, Wref, old_lp.reshape(mask.shape), adv, mask,
+                                  eps_lo=eps_lo, eps_hi=eps_hi, beta=beta, reduction=reduction)
+            t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).double()
+            return {{"loss": torch.tensor([o["loss"]], dtype=torch.float64), "dX": t(o["dX"]),
+                    "dW": t(o["dW"]), "dbias": t(o["dbias"]),
+                    "n_valid": torch.tensor([o["n_valid"]], dtype=torch.int64)}}
+        def ratio(self, local, total):
+            return (local.clamp(min=1).double() / total.clamp(min=1).double())
+        def scale(self, t, f):
+            t.mul_(f)
+
+    got = parallel.dp_fused_linear_grpo(
+        inp["X"][rows], inp["W"], inp["bias"], inp["targets"][rows], inp["Xref"][rows], inp["Wref"],
+        inp["old_lp"][rows], inp["adv"][list(seqs)], inp["mask"][list(seqs)], eps_lo=0.2, eps_hi=0.28,
+        beta=0.04, reduction=red, ops=OracleOps())
+    rel = lambda a, b: float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+    assert abs(got["loss"].item() - want["loss"]) <= 1e-12 * max(1.0, abs(want["loss"])), (got["loss"], want["loss"])
+    assert rel(got["dW"].numpy(), want["dW"]) <= 1e-12
+    assert rel(got["dbias"].numpy(), want["dbias"]) <= 1e-12
+    assert rel(got["dX"].numpy(), want["dX"][rows]) <= 1e-12
+    expect_count = want["n_valid"] if red == pl.PL_BNPO else bs
+    assert int(got["count"].item()) == expect_count
+    print("RANK_OK", rank, flush=True)
+    dist.destroy_process_group()
+""")
+
+
+@pytest.mark.parametrize("red", [0, 1], ids=["bnpo", "grpo"])
+def test_dp_step_matches_whole_batch_oracle(red):
+    script = SCRIPT.format(root=ROOT, red=red)
+    port = _free_port()
+    procs = []
+    for r in range(2):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE="2", MASTER_ADDR="127.0.0.1",
+                   MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="")
+        procs.append(subprocess.Popen([sys.executable, "-c", script], env=env, stdout=subprocess.PIPE,
+                                      stderr=subprocess.PIPE, text=True))
+    for p in procs:
+        out, err = p.communicate(timeout=180)
+        assert p.returncode == 0, err[-3000:]
+        assert "RANK_OK" in out
