@@ -58,6 +58,14 @@ void pl_debug_set_wait(unsigned long long wait_ns, unsigned extra_arrivals, unsi
 int pl_debug_set_rkl_cluster(int cl);
 
 /*
+ * Forces the GEMM's pair tile for later launches on this process: 1 = 256 x 256
+ * (one N=256 MMA per K step, double-buffered accumulators), 2 = 256 x 512 (two
+ * MMAs sharing the A stage); 0 restores the host's choice (256 x 512 when every
+ * problem of the launch is at least 512 wide).  Returns PL_ERR_ARG otherwise.
+ */
+int pl_debug_set_gemm_tile(int nh);
+
+/*
  * The persistent GEMM's tile schedule, for a host-side check: two problems of
  * t0 tiles (c0 k-steps each) and t1 tiles (c1 k-steps each) over `pairs` CTA
  * pairs.  out_pair[t] (t0 + t1 entries) receives the pair that runs tile t.

@@ -86,6 +86,8 @@ _lib.pl_debug_set_wait.argtypes = [ctypes.c_ulonglong, ctypes.c_uint, ctypes.c_u
 _lib.pl_debug_set_wait.restype = None
 _lib.pl_debug_pair_tiles.argtypes = [_I, _I, _I, _I, _I, _P]
 _lib.pl_debug_pair_tiles.restype = _I
+_lib.pl_debug_set_gemm_tile.argtypes = [_I]
+_lib.pl_debug_set_gemm_tile.restype = _I
 _lib.pl_debug_set_rkl_cluster.argtypes = [_I]
 _lib.pl_debug_set_rkl_cluster.restype = _I
 _lib.pl_debug_launch_count.argtypes = []
@@ -95,7 +97,7 @@ EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_linear_grpo_tem
             "pl_fused_selective_logprob_workspace_bytes", "pl_reverse_kl", "pl_reverse_kl_workspace_bytes", "pl_scale", "pl_count_ratio", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
             "pl_version", "pl_debug_gemm", "pl_debug_timing", "pl_debug_timing_read",
-            "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_pair_tiles")
+            "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_set_gemm_tile", "pl_debug_pair_tiles")
 
 
 class PLError(RuntimeError):
@@ -253,6 +255,10 @@ def pl_debug_launch_count() -> int:
 def pl_debug_set_wait(wait_ns: int, extra_arrivals: int = 0, extra_tx: int = 0) -> None:
     """Test knob (include/pl_debug.h): wait bound and wait-run-out injection."""
     _lib.pl_debug_set_wait(int(wait_ns), int(extra_arrivals), int(extra_tx))
+
+
+def pl_debug_set_gemm_tile(nh: int) -> int:
+    return _lib.pl_debug_set_gemm_tile(nh)
 
 
 def pl_debug_set_rkl_cluster(cl: int) -> int:

@@ -112,6 +112,12 @@ extern "C" void pl_debug_set_wait(unsigned long long wait_ns, unsigned extra_arr
   k.extra_tx = extra_tx;
 }
 
+extern "C" int pl_debug_set_gemm_tile(int nh) {
+  if (nh < 0 || nh > 2) return PL_ERR_ARG;
+  debug_knobs().gemm_nh = nh;
+  return PL_OK;
+}
+
 extern "C" int pl_debug_set_rkl_cluster(int cl) {
   if (cl != 0 && cl != 1 && cl != 2 && cl != 4 && cl != 8) return PL_ERR_ARG;
   debug_knobs().rkl_cluster = cl;

@@ -8,15 +8,15 @@
 
 namespace pl {
 
-// A CTA pair (a cluster of two CTAs on two SMs) owns one kPairM x kBN output
-// tile: each CTA holds kBM rows of A, kBNh rows of B and kBM x kBN fp32
-// accumulators in its tensor memory; the pair leader issues M=256 MMAs.
+// A CTA pair (a cluster of two CTAs on two SMs) owns one kPairM x (NH * kBN)
+// output tile (NH = 1 or 2 N=256 MMAs per K step): each CTA holds kBM rows of A,
+// NH * kBNh rows of B and kBM x (NH * kBN) fp32 accumulators in its tensor
+// memory; the pair leader issues the M=256 MMAs.
 constexpr int kBM = 128;       // rows per CTA (tensor-memory lanes)
 constexpr int kPairM = 256;    // rows per CTA pair (the MMA's M)
 constexpr int kBN = 256;       // tile columns (tensor-memory columns per accumulator)
 constexpr int kBNh = 128;      // B rows (N) held by each CTA of the pair
 constexpr int kBK = 64;        // K per pipeline stage (one 128-byte swizzle row)
-constexpr int kStages = 6;
 constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
 
 enum EpiKind : int {
@@ -62,6 +62,7 @@ struct __align__(64) GemmParams {
   //    `nb` long plus one for the first `rem` pairs, so that all pairs carry
   //    about the same number of k-steps.
   int sched, na, nb, rem;
+  int nh;                  // N=256 MMAs per K step (1 or 2): tiles are kPairM x (nh * kBN)
   unsigned* err;
   unsigned long long wait_ns;
   unsigned extra_tx;       // test-only: extra bytes each stage expects (0 in normal use)
@@ -75,7 +76,8 @@ struct __align__(64) GemmParams {
 bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, uint64_t outer,
                   uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
 
-// Fills tiles_m/tiles_n/k_steps/tile_begin of each job and total_tiles.
+// Fills tiles_m/tiles_n/k_steps/tile_begin of each job and total_tiles, for
+// tiles nh * kBN wide.  launch_gemm picks nh and calls it again.
 void gemm_finalize_jobs(GemmParams* p);
 
 cudaError_t launch_gemm(const GemmParams& p, DType dt, cudaStream_t stream);

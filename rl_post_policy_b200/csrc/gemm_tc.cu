@@ -48,10 +48,21 @@ namespace {
 using namespace sm100;
 
 constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB: this CTA's 128 rows of A
-constexpr uint32_t kBBytes = kBNh * kBK * 2;            // 16 KB: this CTA's 128 rows of B
-constexpr uint32_t kStageBytes = kABytes + kBBytes;     // 32 KB
+constexpr uint32_t kBBytes = kBNh * kBK * 2;            // 16 KB: this CTA's 128 rows of B per MMA
 constexpr uint32_t kTmemCols = 512;
-constexpr size_t kGemmSmem = 1024 + kStages * kStageBytes + 256;
+
+// Pair tile kPairM x (kBN * NH).  NH = 1: one N=256 MMA per K=16 step, two
+// accumulators alternating between tiles (the epilogue of tile t overlaps the
+// mainloop of t+1), 6 stages of 32 KB.  NH = 2: two N=256 MMAs per step share
+// the A stage (25% fewer operand bytes per flop and half the barrier round
+// trips), one 512-column accumulator, 4 stages of 48 KB.
+template <int NH>
+struct TileCfg {
+  static constexpr int kTileN = kBN * NH;
+  static constexpr int kStages = NH == 1 ? 6 : 4;
+  static constexpr uint32_t kStageBytes = kABytes + NH * kBBytes;
+  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256;
+};
 
 __device__ __forceinline__ float cvt_in(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ float cvt_in(__half x) { return __half2float(x); }
@@ -195,8 +206,11 @@ __device__ __forceinline__ void add_bias32(const T* bias, float (&v)[32], int nv
   }
 }
 
-template <typename T>
+template <typename T, int NH>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  using Cfg = TileCfg<NH>;
+  constexpr int kStages = Cfg::kStages;
+  constexpr uint32_t kStageBytes = Cfg::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
@@ -254,7 +268,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         const TileCoord tc = tile_coord(p, tile);
         const GemmJob& j = p.jobs[tc.job];
         const int m0 = tc.mb * kPairM + (int)rank * kBM;
-        const int n0 = tc.nb * kBN + (int)rank * kBNh;
+        const int nt0 = tc.nb * Cfg::kTileN + (int)rank * kBNh;
         const CUtensorMap* amap = &p.maps[j.a_map];
         const CUtensorMap* bmap = &p.maps[j.b_map];
         for (int k = 0; k < j.k_steps; ++k) {
@@ -270,11 +284,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             tma_load_2d_pair(a_dst, amap, bar, m0, k0);
             tma_load_2d_pair(a_dst + 8192, amap, bar, m0 + 64, k0);
           }
-          if (!j.b_mn) {
-            tma_load_2d_pair(b_dst, bmap, bar, k0, n0);
-          } else {
-            tma_load_2d_pair(b_dst, bmap, bar, n0, k0);
-            tma_load_2d_pair(b_dst + 8192, bmap, bar, n0 + 64, k0);
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            // MMA h needs columns [h*kBN, (h+1)*kBN) of the tile; this CTA holds kBNh of them
+            const int n0 = nt0 + h * kBN;
+            uint8_t* bh = b_dst + h * kBBytes;
+            if (!j.b_mn) {
+              tma_load_2d_pair(bh, bmap, bar, k0, n0);
+            } else {
+              tma_load_2d_pair(bh, bmap, bar, n0, k0);
+              tma_load_2d_pair(bh + 8192, bmap, bar, n0 + 64, k0);
+            }
           }
           if (++stage == kStages) {
             stage = 0;
@@ -296,39 +316,104 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       int acc = 0;
       uint32_t acc_phase = 0;
       const uint32_t ring_addr = smem_u32(ring);
+      // The K=16 MMAs of one stage into accumulator half h (column offset d_col).
+      auto issue = [&](int st, int k, const GemmJob& j, uint32_t idesc, int h, uint32_t d_col) {
+        const uint32_t a_addr = ring_addr + st * kStageBytes;
+        const uint32_t b_addr = a_addr + kABytes + h * kBBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = j.a_mn ? smem_desc(a_addr + kk * 2048, 8192, 1024)
+                                     : smem_desc(a_addr + kk * 32, 16, 1024);
+          const uint64_t bd = j.b_mn ? smem_desc(b_addr + kk * 2048, 8192, 1024)
+                                     : smem_desc(b_addr + kk * 32, 16, 1024);
+          mma_f16_ss_pair(tmem_base + d_col, ad, bd, idesc, (k | kk) != 0 ? 1u : 0u);
+        }
+      };
       for (int it = 0; !*abort_flag; ++it) {
         const int tile = pair_tile(p, pair, npairs, it);
         if (tile < 0) break;
         const TileCoord tc = tile_coord(p, tile);
         const GemmJob& j = p.jobs[tc.job];
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, lim)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * kBN;
         const uint32_t idesc = instr_desc_f16(AbFormat<T>::v, j.a_mn, j.b_mn, kPairM, kBN);
         bool ok = true;
-        for (int k = 0; k < j.k_steps; ++k) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, lim)) { ok = false; break; }
+        if constexpr (NH == 1) {
+          if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, lim)) break;
           tc_fence_after();
-          const uint32_t a_addr = ring_addr + stage * kStageBytes;
-          const uint32_t b_addr = a_addr + kABytes;
-#pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = j.a_mn ? smem_desc(a_addr + kk * 2048, 8192, 1024)
-                                       : smem_desc(a_addr + kk * 32, 16, 1024);
-            const uint64_t bd = j.b_mn ? smem_desc(b_addr + kk * 2048, 8192, 1024)
-                                       : smem_desc(b_addr + kk * 32, 16, 1024);
-            mma_f16_ss_pair(d_tmem, ad, bd, idesc, (k | kk) != 0 ? 1u : 0u);
+          for (int k = 0; k < j.k_steps; ++k) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, lim)) { ok = false; break; }
+            tc_fence_after();
+            issue(stage, k, j, idesc, 0, acc * kBN);
+            mma_commit_pair(&empty[stage], 0x3);
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
-          mma_commit_pair(&empty[stage], 0x3);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1;
+          if (!ok) break;
+          mma_commit_pair(&tfull[acc], 0x3);
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1;
           }
-        }
-        if (!ok) break;
-        mma_commit_pair(&tfull[acc], 0x3);
-        if (++acc == 2) {
-          acc = 0;
+        } else {
+          // One 512-column accumulator, drained by the epilogue in two halves
+          // (tempty[0], tempty[1]).  Half 0 of this tile starts once the
+          // previous tile's half 0 is drained; a stage whose half-1 MMAs cannot
+          // be issued yet (half 1 still draining) is held back, uncommitted, and
+          // flushed in k order as soon as half 1 is free (or when every stage
+          // is held).  Each half still accumulates in k order.
+          if (!mbar_wait(&tempty[0], acc_phase ^ 1, abort_flag, lim)) break;
+          tc_fence_after();
+          bool h1 = mbar_try_wait(&tempty[1], acc_phase ^ 1);
+          if (h1) tc_fence_after();
+          int held = 0, held_stage = 0, held_k = 0;
+          auto flush = [&]() {
+            for (int q = 0; q < held; ++q) {
+              const int st = (held_stage + q) % kStages;
+              issue(st, held_k + q, j, idesc, 1, kBN);
+              mma_commit_pair(&empty[st], 0x3);
+            }
+            held = 0;
+          };
+          for (int k = 0; k < j.k_steps; ++k) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, lim)) { ok = false; break; }
+            tc_fence_after();
+            issue(stage, k, j, idesc, 0, 0);
+            if (!h1 && mbar_try_wait(&tempty[1], acc_phase ^ 1)) {
+              tc_fence_after();
+              h1 = true;
+            }
+            if (h1) {
+              flush();
+              issue(stage, k, j, idesc, 1, kBN);
+              mma_commit_pair(&empty[stage], 0x3);
+            } else {
+              if (held == 0) {
+                held_stage = stage;
+                held_k = k;
+              }
+              ++held;
+              if (held == kStages) {
+                if (!mbar_wait(&tempty[1], acc_phase ^ 1, abort_flag, lim)) { ok = false; break; }
+                tc_fence_after();
+                h1 = true;
+                flush();
+              }
+            }
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+          if (ok && held) {
+            if (!mbar_wait(&tempty[1], acc_phase ^ 1, abort_flag, lim)) ok = false;
+            else {
+              tc_fence_after();
+              flush();
+            }
+          }
+          if (!ok) break;
+          mma_commit_pair(&tfull[0], 0x3);
           acc_phase ^= 1;
         }
       }
@@ -347,96 +432,108 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     for (int it = 0;; ++it) {
       const int tile = pair_tile(p, pair, npairs, it);
       if (tile < 0) break;
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, lim)) break;
+      if (!mbar_wait(&tfull[NH == 1 ? acc : 0], acc_phase, abort_flag, lim)) break;
       tc_fence_after();
       const TileCoord tc = tile_coord(p, tile);
       const GemmJob& j = p.jobs[tc.job];
-      const int m0 = tc.mb * kPairM + (int)rank * kBM, n0 = tc.nb * kBN;
+      const int m0 = tc.mb * kPairM + (int)rank * kBM;
       const int row = m0 + r_local;
       const bool row_ok = row < j.M;
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * kBN;
-      if (j.epi == kEpiLse) {
-        const T* bias = reinterpret_cast<const T*>(j.bias);
-        T* logits = reinterpret_cast<T*>(j.logits);
-        const int64_t tgt_rel = row_ok ? (j.targets[row] - (int64_t)n0) : (int64_t)-1;
-        float m_run = -INFINITY, s_run = 0.0f, ztv = 0.0f;
-        bool got = false;
 #pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-          float v[32];
-          tmem_ld_32x32b_x32(taddr + c * 32, v);
-          const int col0 = n0 + c * 32;
-          const int nvalid = min(32, j.N - col0);
-          if (nvalid <= 0) continue;
-          if (bias) add_bias32<T>(bias + col0, v, nvalid);
-          if (j.logit_scale != 1.0f) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) v[q] *= j.logit_scale;
-          }
-          if (nvalid == 32) {
-            // full chunk: no per-column predicates; two columns per packed instruction
-            float cmax = v[0];
-#pragma unroll
-            for (int q = 1; q < 32; ++q) cmax = fmaxf(cmax, v[q]);
-            const float m_new = fmaxf(m_run, cmax);
-            const float2 nmb = make_float2(-m_new * kLog2e, -m_new * kLog2e);
-            const float2 l2e = make_float2(kLog2e, kLog2e);
-            float2 s2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-            for (int q = 0; q < 32; q += 2) {
-              const float2 x = __ffma2_rn(make_float2(v[q], v[q + 1]), l2e, nmb);
-              s2 = __fadd2_rn(s2, make_float2(ex2_approx(x.x), ex2_approx(x.y)));
+      for (int h = 0; h < NH; ++h) {
+        // 256-column group h of the tile: TMEM columns [col_base, col_base + 256)
+        const int n0 = tc.nb * Cfg::kTileN + h * kBN;
+        const int grp = tc.nb * NH + h;     // index of this 256-column group along N
+        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (NH == 1 ? acc : h) * kBN;
+        if (n0 >= j.N) {
+          // past the end of N: zeros only, nothing to store
+        } else if (j.epi == kEpiLse) {
+          const T* bias = reinterpret_cast<const T*>(j.bias);
+          T* logits = reinterpret_cast<T*>(j.logits);
+          const int64_t tgt_rel = row_ok ? (j.targets[row] - (int64_t)n0) : (int64_t)-1;
+          float m_run = -INFINITY, s_run = 0.0f, ztv = 0.0f;
+          bool got = false;
+  #pragma unroll 1
+          for (int c = 0; c < kBN / 32; ++c) {
+            float v[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, v);
+            const int col0 = n0 + c * 32;
+            const int nvalid = min(32, j.N - col0);
+            if (nvalid <= 0) continue;
+            if (bias) add_bias32<T>(bias + col0, v, nvalid);
+            if (j.logit_scale != 1.0f) {
+  #pragma unroll
+              for (int q = 0; q < 32; ++q) v[q] *= j.logit_scale;
             }
-            s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, nmb.x)) + (s2.x + s2.y);
-            m_run = m_new;
-          } else {
-            float cmax = -INFINITY;
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (q < nvalid) cmax = fmaxf(cmax, v[q]);
-            const float m_new = fmaxf(m_run, cmax);
-            const float mb = m_new * kLog2e;
-            float s = 0.0f;
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (q < nvalid) s += ex2_approx(fmaf(v[q], kLog2e, -mb));
-            s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, -mb)) + s;
-            m_run = m_new;
+            if (nvalid == 32) {
+              // full chunk: no per-column predicates; two columns per packed instruction
+              float cmax = v[0];
+  #pragma unroll
+              for (int q = 1; q < 32; ++q) cmax = fmaxf(cmax, v[q]);
+              const float m_new = fmaxf(m_run, cmax);
+              const float2 nmb = make_float2(-m_new * kLog2e, -m_new * kLog2e);
+              const float2 l2e = make_float2(kLog2e, kLog2e);
+              float2 s2 = make_float2(0.0f, 0.0f);
+  #pragma unroll
+              for (int q = 0; q < 32; q += 2) {
+                const float2 x = __ffma2_rn(make_float2(v[q], v[q + 1]), l2e, nmb);
+                s2 = __fadd2_rn(s2, make_float2(ex2_approx(x.x), ex2_approx(x.y)));
+              }
+              s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, nmb.x)) + (s2.x + s2.y);
+              m_run = m_new;
+            } else {
+              float cmax = -INFINITY;
+  #pragma unroll
+              for (int q = 0; q < 32; ++q)
+                if (q < nvalid) cmax = fmaxf(cmax, v[q]);
+              const float m_new = fmaxf(m_run, cmax);
+              const float mb = m_new * kLog2e;
+              float s = 0.0f;
+  #pragma unroll
+              for (int q = 0; q < 32; ++q)
+                if (q < nvalid) s += ex2_approx(fmaf(v[q], kLog2e, -mb));
+              s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, -mb)) + s;
+              m_run = m_new;
+            }
+            const int64_t rel = tgt_rel - c * 32;
+            if (rel >= 0 && rel < 32) {
+  #pragma unroll
+              for (int q = 0; q < 32; ++q)
+                if (q == (int)rel) ztv = v[q];
+              got = true;
+            }
+            if (logits && row_ok) store_row32<T>(logits + (int64_t)row * j.logits_ld + col0, v, nvalid);
           }
-          const int64_t rel = tgt_rel - c * 32;
-          if (rel >= 0 && rel < 32) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (q == (int)rel) ztv = v[q];
-            got = true;
+          if (row_ok) {
+            j.part[(int64_t)row * j.part_ld + grp] = make_float2(m_run, s_run);
+            if (got) j.zt[row] = ztv;
           }
-          if (logits && row_ok) store_row32<T>(logits + (int64_t)row * j.logits_ld + col0, v, nvalid);
+        } else {
+          const float sc = j.scale ? __ldg(j.scale) : 1.0f;
+  #pragma unroll 1
+          for (int c = 0; c < kBN / 32; ++c) {
+            float v[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, v);
+            const int col0 = n0 + c * 32;
+            const int nvalid = min(32, j.N - col0);
+            if (!row_ok || nvalid <= 0) continue;
+  #pragma unroll
+            for (int q = 0; q < 32; ++q) v[q] *= sc;
+            const int64_t off = (int64_t)row * j.out_ld + col0;
+            if (j.acc_in) add_row32_f32(j.acc_in + off, v, nvalid);
+            if (j.out_f32) store_row32_f32(reinterpret_cast<float*>(j.out) + off, v, nvalid);
+            else store_row32<T>(reinterpret_cast<T*>(j.out) + off, v, nvalid);
+          }
         }
-        if (row_ok) {
-          j.part[(int64_t)row * j.part_ld + tc.nb] = make_float2(m_run, s_run);
-          if (got) j.zt[row] = ztv;
+        tc_fence_before();
+        mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[NH == 1 ? acc : h]), 0));
+      }  // groups
+      if (NH == 1) {
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
         }
       } else {
-        const float sc = j.scale ? __ldg(j.scale) : 1.0f;
-#pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-          float v[32];
-          tmem_ld_32x32b_x32(taddr + c * 32, v);
-          const int col0 = n0 + c * 32;
-          const int nvalid = min(32, j.N - col0);
-          if (!row_ok || nvalid <= 0) continue;
-#pragma unroll
-          for (int q = 0; q < 32; ++q) v[q] *= sc;
-          const int64_t off = (int64_t)row * j.out_ld + col0;
-          if (j.acc_in) add_row32_f32(j.acc_in + off, v, nvalid);
-          if (j.out_f32) store_row32_f32(reinterpret_cast<float*>(j.out) + off, v, nvalid);
-          else store_row32<T>(reinterpret_cast<T*>(j.out) + off, v, nvalid);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
-      if (++acc == 2) {
-        acc = 0;
         acc_phase ^= 1;
       }
     }
@@ -454,10 +551,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 
 void gemm_finalize_jobs(GemmParams* p) {
   int begin = 0;
+  const int tile_n = kBN * (p->nh == 2 ? 2 : 1);
   for (int i = 0; i < p->njobs; ++i) {
     GemmJob& j = p->jobs[i];
     j.tiles_m = (j.M + kPairM - 1) / kPairM;
-    j.tiles_n = (j.N + kBN - 1) / kBN;
+    j.tiles_n = (j.N + tile_n - 1) / tile_n;
     j.k_steps = (j.K + kBK - 1) / kBK;
     j.tile_begin = begin;
     begin += j.tiles_m * j.tiles_n;
@@ -496,8 +594,42 @@ void balance_schedule(GemmParams* p, int P) {
 }
 
 namespace {
-template <typename T>
+// Estimated launch length, in N=256 MMA k-steps per pair, for pair tiles nh
+// MMAs wide on P pairs: the larger of the even share of all the work and the
+// longest single tile (a tile runs on one pair), or, for one problem of
+// equal-cost tiles, whole waves of tiles.
+double launch_estimate(GemmParams p, int nh, int P) {
+  p.nh = nh;
+  gemm_finalize_jobs(&p);
+  double work = 0.0, longest = 0.0;
+  for (int i = 0; i < p.njobs; ++i) {
+    const GemmJob& j = p.jobs[i];
+    const double tile = (double)j.k_steps * nh;
+    work += (double)j.tiles_m * j.tiles_n * tile;
+    if (j.tiles_m * j.tiles_n > 0 && tile > longest) longest = tile;
+  }
+  if (p.njobs == 1) {
+    const double waves = (double)((p.total_tiles + P - 1) / P);
+    return waves * longest;
+  }
+  const double share = work / P;
+  return share > longest ? share : longest;
+}
+
+// 256 x 512 tiles move 25% fewer operand bytes per flop and halve the barrier
+// round trips; measured on this kernel they run the same k-step work about 10%
+// faster when the launch stays balanced.  They need every problem to be at
+// least 512 wide.
+int pick_tile_width(const GemmParams& p, int P) {
+  if (P <= 0) return 1;
+  for (int i = 0; i < p.njobs; ++i)
+    if (p.jobs[i].N < 2 * kBN) return 1;
+  return 0.9 * launch_estimate(p, 2, P) < launch_estimate(p, 1, P) ? 2 : 1;
+}
+
+template <typename T, int NH>
 cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
+  constexpr size_t kGemmSmem = TileCfg<NH>::kSmem;
   static int max_pairs = 0;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -511,13 +643,13 @@ cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (max_pairs == 0) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<T, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
     if (e != cudaSuccess) return e;
     DevInfo di;
     if ((e = dev_info(&di)) != cudaSuccess) return e;
     cfg.gridDim = dim3(di.sm_count & ~1);
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<T>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<T, NH>, &cfg);
     if (e != cudaSuccess) return e;
     max_pairs = n > 0 ? n : 1;
   }
@@ -526,19 +658,30 @@ cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
   GemmParams q = p;
   balance_schedule(&q, pairs);
   launch_begin(0, stream);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<T>, q);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<T, NH>, q);
   launch_end(0, stream);
   return e;
 }
 }  // namespace
 
 cudaError_t launch_gemm(const GemmParams& p0, DType dt, cudaStream_t stream) {
-  if (p0.total_tiles <= 0) return cudaSuccess;
   GemmParams p = p0;
   p.wait_ns = debug_knobs().wait_ns;
   p.extra_tx = debug_knobs().extra_tx;
-  if (dt == DType::BF16) return launch_t<__nv_bfloat16>(p, stream);
-  if (dt == DType::F16) return launch_t<__half>(p, stream);
+  // Tile width: 256 x 512 pair tiles (nh = 2) unless a problem is narrower than
+  // 512 or the wider tiles would unbalance the launch (see pick_tile_width).
+  int nh = 1;
+  if (debug_knobs().gemm_nh) {
+    nh = debug_knobs().gemm_nh;
+  } else {
+    DevInfo di;
+    if (dev_info(&di) == cudaSuccess) nh = pick_tile_width(p, di.sm_count / 2);
+  }
+  p.nh = nh;
+  gemm_finalize_jobs(&p);
+  if (p.total_tiles <= 0) return cudaSuccess;
+  if (dt == DType::BF16) return nh == 2 ? launch_t<__nv_bfloat16, 2>(p, stream) : launch_t<__nv_bfloat16, 1>(p, stream);
+  if (dt == DType::F16) return nh == 2 ? launch_t<__half, 2>(p, stream) : launch_t<__half, 1>(p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -100,6 +100,7 @@ struct DebugKnobs {
   unsigned extra_arrivals = 0;
   unsigned extra_tx = 0;
   int rkl_cluster = 0;   // reverse-KL CTAs per cluster (1, 2, 4 or 8; 0 = the host's choice)
+  int gemm_nh = 0;       // GEMM tile width in N=256 MMAs (1 or 2; 0 = the host's choice)
 };
 DebugKnobs& debug_knobs();
 

@@ -21,3 +21,12 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(params=[1, 2], ids=["tile256", "tile512"])
+def gemm_tile(request):
+    """Runs a GPU test once with each GEMM pair tile (256 x 256 and 256 x 512)."""
+    import rl_post_policy_b200 as pl
+    assert pl.pl_debug_set_gemm_tile(request.param) == 0
+    yield request.param
+    pl.pl_debug_set_gemm_tile(0)

@@ -12,7 +12,7 @@ import torch
 import oracle
 import synth
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gemm_tile")]
 
 
 @pytest.fixture

@@ -9,7 +9,7 @@ import torch
 import oracle
 import synth
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gemm_tile")]
 
 
 def run(inp, dtype, grad_logp=None, chunk=None, want=("dX", "dW", "dbias"), targets=None):
