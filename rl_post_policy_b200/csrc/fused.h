@@ -23,6 +23,8 @@ struct FusedOffsets {
   int64_t logits;     // T [C, ld]           logits, then dlogits (if a gradient is wanted)
   int64_t dw_acc;     // f32 [V, H]          dW accumulator (multi-chunk only)
   int64_t db_acc;     // f32 [V]             dbias accumulator (multi-chunk only)
+  int64_t db_part;    // f32 [kDlMaxRowGroups, V]  dbias column sums per dlogits row group
+  int64_t db_cnt;     // u32 [ceil(V/256)]   finished row groups per 256-column strip (self-resetting)
   int64_t total;
 };
 
@@ -53,6 +55,9 @@ struct CombineArgs {
   float g_scale;            // 1 / temperature: dLoss/dlogp -> gradient of the raw logits
 };
 
+// The dlogits pass splits a chunk's rows into at most this many groups.
+constexpr int kDlMaxRowGroups = 16;
+
 struct DlogitsArgs {
   unsigned char* ws;
   FusedOffsets off;
@@ -64,6 +69,10 @@ struct DlogitsArgs {
   int dbias_mode;
   float* dbias_acc;
   void* dbias;
+  float* db_part;     // row-group column sums (when a bias gradient is wanted)
+  unsigned* db_cnt;
+  int64_t rg_rows;    // set by launch_dlogits
+  int n_rg;
 };
 
 cudaError_t launch_count(const uint8_t* mask, int64_t bs, int64_t T, unsigned char* ws, int nchunks,

@@ -65,6 +65,8 @@ Plan make_plan(int64_t bs, int64_t T, int64_t H, int64_t V, uint32_t mode, bool 
   p.off.logits = region(2 * p.Cbuf * p.ld);
   p.off.dw_acc = region((need_dW && p.nchunks > 1) ? 4 * V * H : 0);
   p.off.db_acc = region((need_dbias && p.nchunks > 1) ? 4 * V : 0);
+  p.off.db_part = region(need_dbias ? 4 * (int64_t)kDlMaxRowGroups * V : 0);
+  p.off.db_cnt = region(need_dbias ? 4 * (int64_t)p.ntv : 0);
   p.off.total = align_up(cur, 1024);
   return p;
 }
@@ -206,6 +208,8 @@ pl_status run_pipeline(const Pipe& q) {
     da.row0 = r0; da.rows = rows; da.V = V; da.chunk = (int)c;
     da.dbias_mode = dbias ? acc_mode(c, plan.nchunks) : kAccNone;
     da.dbias_acc = reinterpret_cast<float*>(ws + plan.off.db_acc); da.dbias = dbias;
+    da.db_part = reinterpret_cast<float*>(ws + plan.off.db_part);
+    da.db_cnt = reinterpret_cast<unsigned*>(ws + plan.off.db_cnt);
     if (!ok(launch_dlogits(da, dt, s))) return PL_ERR_CUDA;
 
     if (!dX && !dW) continue;

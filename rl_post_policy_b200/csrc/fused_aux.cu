@@ -198,11 +198,31 @@ __global__ void clear_gmax_kernel(unsigned char* ws, int nchunks, FusedOffsets o
 }
 
 // ---------------------------------------------------------------- dlogits
-// Block = 256 threads = 8 warps over a 256-column strip of the chunk's logits;
-// lane l owns columns [8l, 8l+8) of the strip, warp w rows w, w+8, ...
+// Block = 256 threads = 8 warps over one 256-column strip (blockIdx.x) and one
+// group of rows (blockIdx.y); lane l owns columns [8l, 8l+8) of the strip, warp
+// w rows w, w+8, ... of the group, kDlRows rows loaded before any is stored so
+// that each thread keeps kDlRows 16-byte loads in flight.  Many row groups per
+// strip fill the GPU several times over.  The bias gradient: each block writes
+// its strip's column sums for its row group; the strip's last block to finish
+// adds the row groups in order (deterministic) and stores / accumulates them.
+constexpr int kDlRows = 4;
+
+// 8 consecutive elements as raw 16 bytes (zeros past V on the ragged strip).
 template <typename T>
-__global__ void __launch_bounds__(256) dlogits_kernel(DlogitsArgs a) {
+__device__ __forceinline__ uint4 load8(const T* p, bool full8, int64_t col, int64_t V) {
+  if (full8) return *reinterpret_cast<const uint4*>(p);
+  uint4 u = make_uint4(0, 0, 0, 0);
+  T* e8 = reinterpret_cast<T*>(&u);
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    if (col + q < V) e8[q] = p[q];
+  return u;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256, 3) dlogits_kernel(DlogitsArgs a) {
   __shared__ float s_col[8][256];
+  __shared__ int s_last;
   const unsigned char* ws = a.ws;
   const float* row_lse = reinterpret_cast<const float*>(ws + a.off.lse);
   const float* row_g = reinterpret_cast<const float*>(ws + a.off.g);
@@ -214,53 +234,60 @@ __global__ void __launch_bounds__(256) dlogits_kernel(DlogitsArgs a) {
     e = max(-100, min(100, e));
   }
   const float sc = ldexpf(1.0f, e);
-  if (blockIdx.x == 0 && threadIdx.x == 0)
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
     reinterpret_cast<float*>(a.ws + a.off.inv_scale)[a.chunk] = ldexpf(1.0f, -e);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t col = (int64_t)blockIdx.x * 256 + lane * 8;
   const bool full8 = col + 8 <= a.V;
+  const int64_t r_begin = (int64_t)blockIdx.y * a.rg_rows;
+  const int64_t r_end = min(a.rows, r_begin + a.rg_rows);
   float csum[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) csum[q] = 0.0f;
   T* L = reinterpret_cast<T*>(a.logits);
   constexpr float kLog2e = 1.4426950408889634f;
   if (col < a.V) {
-#pragma unroll 4
-    for (int64_t i = warp; i < a.rows; i += 8) {
-      T* p = L + i * a.ld + col;
-      const float gi = __ldg(row_g + i);
-      const float lsei = __ldg(row_lse + i) * kLog2e;
-      const int64_t tg = __ldg(a.targets + a.row0 + i);
-      const int ti = (tg >= 0 && tg < a.V) ? (int)tg : -1;
-      float z[8];
-      if (full8) {
-        uint4 u = *reinterpret_cast<const uint4*>(p);
-        const T* e8 = reinterpret_cast<const T*>(&u);
+    for (int64_t i0 = r_begin + warp; i0 < r_end; i0 += 8 * kDlRows) {
+      uint4 raw[kDlRows];
+      float gi[kDlRows], lsei[kDlRows];
+      int ti[kDlRows];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) z[q] = cvt(e8[q]);
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) z[q] = (col + q < a.V) ? cvt(p[q]) : 0.0f;
+      for (int u = 0; u < kDlRows; ++u) {
+        const int64_t i = i0 + 8 * u;
+        if (i < r_end) {
+          raw[u] = load8<T>(L + i * a.ld + col, full8, col, a.V);
+          gi[u] = __ldg(row_g + i);
+          lsei[u] = __ldg(row_lse + i) * kLog2e;
+          const int64_t tg = __ldg(a.targets + a.row0 + i);
+          ti[u] = (tg >= 0 && tg < a.V) ? (int)tg : -1;
+        }
       }
-      float d[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float pr = exp2f(fmaf(z[q], kLog2e, -lsei));
-        const float oh = (col + q == ti) ? 1.0f : 0.0f;
-        d[q] = gi * (oh - pr);
-        csum[q] += d[q];
-      }
-      if (full8) {
-        uint4 u;
-        T* e8 = reinterpret_cast<T*>(&u);
+      for (int u = 0; u < kDlRows; ++u) {
+        const int64_t i = i0 + 8 * u;
+        if (i >= r_end) break;
+        const T* z = reinterpret_cast<const T*>(&raw[u]);
+        float d[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) e8[q] = to_t<T>(d[q] * sc);
-        *reinterpret_cast<uint4*>(p) = u;
-      } else {
+        for (int q = 0; q < 8; ++q) {
+          const float pr = exp2f(fmaf(cvt(z[q]), kLog2e, -lsei[u]));
+          const float oh = (col + q == ti[u]) ? 1.0f : 0.0f;
+          d[q] = gi[u] * (oh - pr);
+          csum[q] += d[q];
+        }
+        T* p = L + i * a.ld + col;
+        if (full8) {
+          uint4 w;
+          T* e8 = reinterpret_cast<T*>(&w);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (col + q < a.V) p[q] = to_t<T>(d[q] * sc);
+          for (int q = 0; q < 8; ++q) e8[q] = to_t<T>(d[q] * sc);
+          *reinterpret_cast<uint4*>(p) = w;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (col + q < a.V) p[q] = to_t<T>(d[q] * sc);
+        }
       }
     }
   }
@@ -269,10 +296,24 @@ __global__ void __launch_bounds__(256) dlogits_kernel(DlogitsArgs a) {
   for (int q = 0; q < 8; ++q) s_col[warp][lane * 8 + q] = csum[q];
   __syncthreads();
   const int64_t v = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (v < a.V) {
-    float s = 0.0f;
+  float s = 0.0f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += s_col[w][threadIdx.x];
+  for (int w = 0; w < 8; ++w) s += s_col[w][threadIdx.x];
+  if (a.n_rg > 1) {
+    // this row group's column sums; the strip's last block adds the groups in order
+    if (v < a.V) a.db_part[(int64_t)blockIdx.y * a.V + v] = s;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(a.db_cnt + blockIdx.x, 1u) == (unsigned)a.n_rg - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    s = 0.0f;
+    if (v < a.V)
+      for (int r = 0; r < a.n_rg; ++r) s += __ldcg(a.db_part + (int64_t)r * a.V + v);
+    if (threadIdx.x == 0) a.db_cnt[blockIdx.x] = 0u;
+  }
+  if (v < a.V) {
     float* acc = a.dbias_acc;
     T* out = reinterpret_cast<T*>(a.dbias);
     switch (a.dbias_mode) {
@@ -333,8 +374,15 @@ cudaError_t launch_clear_gmax(unsigned char* ws, int nchunks, const FusedOffsets
   return cudaGetLastError();
 }
 
-cudaError_t launch_dlogits(const DlogitsArgs& a, DType dt, cudaStream_t s) {
-  const unsigned grid = (unsigned)((a.V + 255) / 256);
+cudaError_t launch_dlogits(const DlogitsArgs& a0, DType dt, cudaStream_t s) {
+  if (a0.rows <= 0) return cudaSuccess;
+  DlogitsArgs a = a0;
+  // row groups of >= 128 rows (a multiple of the 32 rows one pass covers), at most kDlMaxRowGroups
+  int64_t rg = (a.rows + kDlMaxRowGroups - 1) / kDlMaxRowGroups;
+  rg = rg < 128 ? 128 : (rg + 31) / 32 * 32;
+  a.rg_rows = rg;
+  a.n_rg = (int)((a.rows + rg - 1) / rg);
+  const dim3 grid((unsigned)((a.V + 255) / 256), (unsigned)a.n_rg);
   if (dt == DType::BF16) {
     { launch_begin(2, s); dlogits_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
   } else {
