@@ -188,3 +188,13 @@ def test_python_entry_points():
     l2 = ag.reverse_kl_autograd(x, t, m)
     (3.0 * l2).backward()
     assert torch.equal(x.grad, (grad.float() * 3.0).to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32], ids=["bf16", "fp16", "fp32"])
+@pytest.mark.parametrize("grad", [True, False], ids=["fwd_bwd", "fwd"])
+def test_aligned_rows(dtype, grad):
+    # V = 3000: every row starts on a 16-byte boundary in every dtype (no scalar head or tail)
+    inp = synth.reverse_kl_inputs(2, 24, 3000, dtype, synth.seed_for(49))
+    want = oracle.reverse_kl(inp["student"], inp["teacher"], inp["mask"], want_grad=grad)
+    got = run(inp["student"], inp["teacher"], inp["mask"], grad=grad)
+    check(got, want, inp["mask"], dtype, 48, 3000)
