@@ -210,12 +210,28 @@ def workload_desc(w: int) -> dict:
     return d
 
 
-def chunk_mode(N: int, chunk_rows: int) -> int:
-    """PL_CHUNK_ROWS bits: -1 = one chunk covering the batch (up to 32640 rows)."""
-    import rl_post_policy_b200 as pl
+def chunk_rows_for(N: int, chunk_rows: int) -> int:
+    """Rows per chunk: -1 = one chunk covering the batch (up to 32640 rows), else a
+    multiple of 128."""
     c = N if chunk_rows < 0 else chunk_rows
-    c = max(128, min(32640, (c + 127) // 128 * 128))
+    return max(128, min(32640, (c + 127) // 128 * 128))
+
+
+def chunk_mode(N: int, chunk_rows: int) -> int:
+    """PL_CHUNK_ROWS bits for chunk_rows_for(N, chunk_rows)."""
+    import rl_post_policy_b200 as pl
+    c = chunk_rows_for(N, chunk_rows)
     return pl.PL_CHUNK_ROWS(c), c
+
+
+def arm_config(d: dict, chunk_rows: int, ws_world: int) -> dict:
+    """The workload named in both arms' JSON lines."""
+    N = d["bs"] * d["T"]
+    return {"workload": f"fused GRPO fwd+bwd, bs={d['bs']} x T={d['T']} (N={N}), H={d['H']}, V={d['V']}, "
+                        f"beta={d['beta']}, GRPO, eps=0.2/0.28",
+            "per_gpu_rows": N, "chunk_rows": chunk_rows,
+            "l2": "inputs larger than L2 (W and Wref are 1 GB each); no flush",
+            "parallelism": f"dp{ws_world} (independent batches)"}
 
 
 def make_fused_inputs(w: int, rank: int, chunk_rows: int = -1):
@@ -430,14 +446,13 @@ def run_reference(args):
             times.append(t)
     per = sum(times) / len(times)
     val = rows / per
-    sample = (f"{rows} rows (one sequence) of the workload per step: policy+reference forward over "
-              f"V={d['V']}, loss, dX/dW/dbias, fp64")
+    sample = (f"{rows} rows (one sequence) of the workload per step, value = rows / time: policy+reference "
+              f"forward over V={d['V']}, loss, dX/dW/dbias, fp64")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"fused GRPO fwd+bwd, bs=1 x T={rows} sample of workload {args.workload}",
-                   "H": d["H"], "V": d["V"]},
+        "config": arm_config(d, chunk_rows_for(d["N"], args.chunk_rows), args.gpus),
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -547,11 +562,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": (value / ws_world) / (N / (pub * 1e-3)) if pub else None,
             "dtype": "bf16" if d["dtype"] == torch.bfloat16 else "fp16", "data": "synthetic",
-            "config": {"workload": f"fused GRPO fwd+bwd, bs={d['bs']} x T={d['T']} (N={N}), H={H}, V={V}, "
-                                   f"beta={d['beta']}, GRPO, eps=0.2/0.28",
-                       "per_gpu_rows": N, "chunk_rows": d["chunk_rows"],
-                       "l2": "inputs larger than L2 (W and Wref are 1 GB each); no flush",
-                       "parallelism": f"dp{ws_world} (independent batches)"},
+            "config": arm_config(d, d["chunk_rows"], ws_world),
             "clocks": clk, "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                                    "d2h_bytes_per_step": 4, "ms_per_step": e2e_ms},
             "gpu_launches": launches, "roofline": roofline, "cpu_baseline": cpu,
