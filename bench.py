@@ -55,6 +55,8 @@ def parse():
                     help="rows per chunk (multiple of 128); -1: the whole batch in one chunk")
     ap.add_argument("--no-loss-only", action="store_true")
     ap.add_argument("--no-reverse-kl", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the temperature and selective log-prob measurements")
     ap.add_argument("--only", choices=["reverse_kl", "loss_only"], default=None,
                     help="run one side measurement alone and print its JSON (for profiling)")
     ap.add_argument("--reps", type=int, default=30, help="timed calls per side measurement")
@@ -346,6 +348,64 @@ def loss_only(peaks, peak_kind):
     }
 
 
+# ------------------------------------------------------------------ temperature, selective log-prob
+def next_rows(d, inp, ws, wsb, mode, peak, reps=20):
+    """The fused step at temperature 0.7 (pl_fused_linear_grpo_temp) and the fused
+    selective log-prob forward + backward with an external dL/dlogp
+    (pl_fused_selective_logprob), on the benchmarked workload's tensors, CUDA
+    events around each library launch."""
+    import rl_post_policy_b200 as pl
+    import synth
+    N, H, V, bs, T = d["N"], d["H"], d["V"], d["bs"], d["T"]
+    dt = d["dtype"]
+    loss = torch.zeros(1, device="cuda")
+    dX = torch.empty(N, H, dtype=dt, device="cuda")
+    dW = torch.empty(V, H, dtype=dt, device="cuda")
+    db = torch.empty(V, dtype=dt, device="cuda") if inp["bias"] is not None else None
+    lp = torch.empty(N, device="cuda")
+
+    def timed(call):
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        pl.pl_debug_timing_read()
+        pl.pl_debug_timing(True)
+        for _ in range(reps):
+            call()
+        torch.cuda.synchronize()
+        pl.pl_debug_timing(False)
+        ms, _ = pl.pl_debug_timing_read()
+        return sum(ms) / reps
+
+    def temp_call():
+        pl.check(pl.pl_fused_linear_grpo_temp(inp["X"], inp["W"], inp["bias"], inp["targets"], inp["Xref"],
+                                              inp["Wref"], inp["old_lp"], inp["adv"], inp["mask"], bs, T, H, V,
+                                              EPS_LO, EPS_HI, d["beta"], 0.7, mode, loss, dX, dW, db, None, None,
+                                              None, ws, wsb), "pl_fused_linear_grpo_temp")
+
+    t_ms = timed(temp_call)
+    smode = pl.dtype_mode(dt) | (mode & (0xFF << pl.PL_CHUNK_SHIFT))
+    swsb = pl.pl_fused_selective_logprob_workspace_bytes(N, H, V, smode, 1, int(db is not None))
+    sws = torch.zeros(swsb, dtype=torch.uint8, device="cuda")
+    g = synth.normal((N,), synth.seed_for(2, 7), std=1e-3, device="cuda")
+
+    def sel_call():
+        pl.check(pl.pl_fused_selective_logprob(inp["X"], inp["W"], inp["bias"], inp["targets"], N, H, V, smode, g,
+                                               lp, dX, dW, db, sws, swsb), "pl_fused_selective_logprob")
+
+    s_ms = timed(sel_call)
+    del sws, dX, dW
+    f_temp, f_sel = 8.0 * N * H * V, 6.0 * N * H * V
+    return {
+        "temperature": {"workload": f"fused GRPO fwd+bwd at temperature 0.7, N={N}, H={H}, V={V}",
+                        "ms": t_ms, "tokens_per_s": N / (t_ms * 1e-3), "tflops": f_temp / (t_ms * 1e-3) / 1e12,
+                        "frac_of_peak": f_temp / (t_ms * 1e-3) / 1e12 / peak},
+        "selective_logprob": {"workload": f"fused selective log-prob fwd + bwd (dX, dW), N={N}, H={H}, V={V}",
+                              "ms": s_ms, "tokens_per_s": N / (s_ms * 1e-3), "tflops": f_sel / (s_ms * 1e-3) / 1e12,
+                              "frac_of_peak": f_sel / (s_ms * 1e-3) / 1e12 / peak},
+    }
+
+
 # ------------------------------------------------------------------ reverse KL
 def reverse_kl(peaks, peak_kind, reps=30):
     """Reverse-KL self-distillation at the model card's example shape (bs=4,
@@ -546,6 +606,8 @@ def run_ours(args):
         extra["loss_only"] = loss_only(peaks, peak_kind)
     if rank == 0 and ws_world == 1 and not args.no_reverse_kl:
         extra["reverse_kl"] = reverse_kl(peaks, peak_kind, args.reps)
+    if rank == 0 and ws_world == 1 and not args.no_next_rows:
+        extra.update(next_rows(d, inp, ws, wsb, mode, float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))))
     cpu = None
     if rank == 0 and ws_world == 1 and not args.no_cpu_baseline:
         rows = max(1, min(args.cpu_rows, N))
