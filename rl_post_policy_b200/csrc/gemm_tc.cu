@@ -429,16 +429,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     int acc = 0;
     uint32_t acc_phase = 0;
     constexpr float kLog2e = 1.4426950408889634f;
+    // the jobs' device scale factors, read once per launch rather than per tile
+    const float job_scale0 = p.jobs[0].scale ? __ldg(p.jobs[0].scale) : 1.0f;
+    const float job_scale1 = (p.njobs > 1 && p.jobs[1].scale) ? __ldg(p.jobs[1].scale) : 1.0f;
     for (int it = 0;; ++it) {
       const int tile = pair_tile(p, pair, npairs, it);
       if (tile < 0) break;
-      if (!mbar_wait(&tfull[NH == 1 ? acc : 0], acc_phase, abort_flag, lim)) break;
-      tc_fence_after();
       const TileCoord tc = tile_coord(p, tile);
       const GemmJob& j = p.jobs[tc.job];
       const int m0 = tc.mb * kPairM + (int)rank * kBM;
       const int row = m0 + r_local;
       const bool row_ok = row < j.M;
+      // the row's target id, loaded while the tile's accumulator is still being computed
+      const int64_t tgt = (j.epi == kEpiLse && row_ok) ? __ldg(j.targets + row) : (int64_t)-1;
+      if (!mbar_wait(&tfull[NH == 1 ? acc : 0], acc_phase, abort_flag, lim)) break;
+      tc_fence_after();
 #pragma unroll 1
       for (int h = 0; h < NH; ++h) {
         // 256-column group h of the tile: TMEM columns [col_base, col_base + 256)
@@ -450,7 +455,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         } else if (j.epi == kEpiLse) {
           const T* bias = reinterpret_cast<const T*>(j.bias);
           T* logits = reinterpret_cast<T*>(j.logits);
-          const int64_t tgt_rel = row_ok ? (j.targets[row] - (int64_t)n0) : (int64_t)-1;
+          const int64_t tgt_rel = tgt >= 0 ? tgt - (int64_t)n0 : (int64_t)-1;
           float m_run = -INFINITY, s_run = 0.0f, ztv = 0.0f;
           bool got = false;
   #pragma unroll 1
@@ -509,7 +514,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             if (got) j.zt[row] = ztv;
           }
         } else {
-          const float sc = j.scale ? __ldg(j.scale) : 1.0f;
+          const float sc = tc.job ? job_scale1 : job_scale0;
   #pragma unroll 1
           for (int c = 0; c < kBN / 32; ++c) {
             float v[32];
@@ -526,7 +531,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           }
         }
         tc_fence_before();
-        mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[NH == 1 ? acc : h]), 0));
+        mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&tempty[NH == 1 ? acc : h]), 0));
       }  // groups
       if (NH == 1) {
         if (++acc == 2) {
