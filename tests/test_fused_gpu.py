@@ -208,3 +208,53 @@ def test_temperature(tau, chunk):
     assert abs(loss.item() - want["loss"]) <= 1e-3 * abs(want["loss"])
     for k, t in (("dX", dX), ("dW", dW), ("dbias", db)):
         assert rel_fro(t.cpu().double().numpy(), want[k]) <= 1e-2, k
+
+
+def test_empty_batch_gives_zero_loss_and_zero_weight_gradients():
+    # no rows: loss 0, n_valid 0, dW and dbias written as zeros (nothing to accumulate)
+    m = pl()
+    H, V = 128, 700
+    W = synth.normal((V, H), 11, std=0.02).to(torch.bfloat16).cuda()
+    b = synth.normal((V,), 12, std=0.01).to(torch.bfloat16).cuda()
+    dW = torch.full((V, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    db = torch.full((V,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    loss = torch.full((1,), float("nan"), device="cuda")
+    nv = torch.full((1,), -1, dtype=torch.int64, device="cuda")
+    empty16 = torch.empty(0, H, dtype=torch.bfloat16, device="cuda")
+    mode = m.PL_BF16 | m.PL_GRPO
+    wsb = m.pl_fused_linear_grpo_workspace_bytes(0, 64, H, V, mode, 1, 1)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    m.check(m.pl_fused_linear_grpo(empty16, W, b, torch.empty(0, dtype=torch.int64, device="cuda"), empty16, W,
+                                   torch.empty(0, device="cuda"), torch.empty(0, device="cuda"),
+                                   torch.empty(0, 64, dtype=torch.uint8, device="cuda"), 0, 64, H, V, EPS_LO,
+                                   EPS_HI, 0.04, mode, loss, None, dW, db, None, None, nv, ws, wsb))
+    torch.cuda.synchronize()
+    assert m.pl_device_status(ws) == 0
+    assert loss.item() == 0.0 and int(nv.item()) == 0
+    assert torch.all(dW == 0) and torch.all(db == 0)
+
+
+@pytest.mark.parametrize("red", [0, 1], ids=["bnpo", "grpo"])
+def test_all_masked_batch(red):
+    # every token masked: loss 0 through max(n, 1), every gradient exactly zero
+    inp = build_inputs(2, 64, 128, 640, torch.bfloat16, 4444, bias=True)
+    inp["mask"] = torch.zeros_like(inp["mask"])
+    got = run_fused(inp, torch.bfloat16, red, 0.04)
+    assert got["status"] == 0 and got["n_valid"] == 0
+    assert got["loss"] == 0.0
+    for k in ("dX", "dW", "dbias"):
+        assert np.all(got[k] == 0.0), k
+    want = oracle.fused_grpo(inp["X"], inp["W"], inp["bias"], inp["targets"], inp["Xref"], inp["Wref"],
+                             inp["old_lp"].reshape(2, 64), inp["adv"], inp["mask"], eps_lo=EPS_LO, eps_hi=EPS_HI,
+                             beta=0.04, reduction=red)
+    assert want["loss"] == 0.0
+    assert np.max(np.abs(got["logp"] - want["logp"])) <= 2e-3   # log-probs are still produced
+
+
+def test_repeat_calls_are_bit_identical():
+    inp = build_inputs(3, 100, 200, 1000, torch.bfloat16, 4545, bias=True)
+    a = run_fused(inp, torch.bfloat16, 1, 0.04, chunk=128)
+    b = run_fused(inp, torch.bfloat16, 1, 0.04, chunk=128)
+    assert a["loss"] == b["loss"]
+    for k in ("logp", "ref_logp", "dX", "dW", "dbias"):
+        assert np.array_equal(a[k], b[k]), k
