@@ -333,6 +333,20 @@ def loss_only(peaks, peak_kind):
         gbs = bytes_ / (per * 1e-3) / 1e9
         res[name] = {"bs": bs, "seq": seq, "us_per_call": per * 1e3, "GB_per_s": gbs,
                      "tokens_per_s": tokens / (per * 1e-3), "algorithmic_bytes": bytes_}
+        if name == "small":
+            # the launch-bound case again, 20 calls replayed as one CUDA graph
+            from rl_post_policy_b200.pipeline import GraphedCall
+            gc = GraphedCall(lambda: [call() for _ in range(20)])
+            for _ in range(3):
+                gc.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(10):
+                gc.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            res[name]["graph_us_per_call"] = e0.elapsed_time(e1) * 1e3 / 200
         del inp, g, ws
     peak = float(peaks["hbm_gbs"])
     sw = res["sweep"]
@@ -344,7 +358,8 @@ def loss_only(peaks, peak_kind):
                      "traffic": recorded_traffic("loss_kernel", LOSS_SOURCES)},
         "small_workload": {"workload": "bs=16 x seq=1024 (launch-latency bound)",
                            "us_per_call": res["small"]["us_per_call"],
-                           "tokens_per_s": res["small"]["tokens_per_s"]},
+                           "tokens_per_s": res["small"]["tokens_per_s"],
+                           "graph_us_per_call": res["small"]["graph_us_per_call"]},
     }
 
 

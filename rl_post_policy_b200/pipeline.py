@@ -1,5 +1,10 @@
-"""Host-to-device input staging that overlaps the next step's copy with this
-step's compute.
+"""Stream-level plumbing for the library's entry points: host-to-device input
+staging that overlaps the next step's copy with this step's compute
+(``InputPrefetcher``), and replay of a fixed call sequence as one CUDA graph
+(``GraphedCall``).
+
+Input staging
+-------------
 
 A training step reads a few per-step inputs from the host: hidden states,
 targets, behaviour log-probs, advantages and the mask.  Copied on the compute
@@ -79,3 +84,32 @@ class InputPrefetcher:
         """Makes the current stream wait for every copy still in flight."""
         for i in range(self.inflight):
             torch.cuda.current_stream().wait_event(self.copied[(self.tail + i) % len(self.slots)])
+
+
+class GraphedCall:
+    """Captures `fn` (a call sequence of the library's entry points on fixed
+    device buffers) into a CUDA graph and replays it with one launch.
+
+    The library's one-time host work (kernel attributes, occupancy queries) and
+    any workspace creation happen in the `warmup` eager calls before capture;
+    the captured calls then contain only kernel launches on the capturing
+    stream.  Replays read and write the same buffers as the captured call: copy
+    new inputs into them before ``replay()``.  This replaces per-call launch
+    overhead -- several kernels per fused step, one cooperative launch per loss
+    call -- for small, launch-bound batches.
+    """
+
+    def __init__(self, fn, warmup: int = 2):
+        stream = torch.cuda.Stream()
+        stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                fn()
+        torch.cuda.current_stream().wait_stream(stream)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            fn()
+
+    def replay(self) -> None:
+        self.graph.replay()
