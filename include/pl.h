@@ -103,10 +103,19 @@ typedef enum {
  * bs*seq == 0 writes loss 0.  Pointers that are not 16-byte aligned take a scalar
  * path; they never fail.
  * Scratch: pl_loss keeps one small zero-initialised buffer per (device, stream),
- * allocated on the first call on that pair (make that first call outside any
- * stream capture).  Calls on one stream are ordered; calls on different streams
- * use different scratch.
+ * allocated on the first call on that pair, or ahead of time by pl_init (make
+ * that first call, or pl_init, outside any stream capture).  Calls on one stream
+ * are ordered; calls on different streams use different scratch.
  */
+/* pl_init: creates, ahead of the first call, the library-owned scratch that
+ * pl_loss (and pl_reverse_kl with a NULL workspace) use on the current device
+ * and `stream`, sized for batches of up to max_bs sequences, so that later calls
+ * allocate nothing and may be captured into a CUDA graph.  It synchronises
+ * `stream` only when it has to grow an existing buffer.  max_bs < 0 is
+ * PL_ERR_ARG; a device that is not compute capability 10.0 is PL_ERR_ARCH.
+ */
+pl_status pl_init(int64_t max_bs, pl_stream_t stream);
+
 pl_status pl_loss(const void* policy_lp, const void* old_lp, const void* ref_lp,
                   const void* adv, const uint8_t* mask, int64_t bs, int64_t seq,
                   float eps_lo, float eps_hi, float beta, uint32_t mode,

@@ -68,6 +68,8 @@ _lib.pl_reverse_kl_workspace_bytes.argtypes = [_I64, _I64]
 _lib.pl_reverse_kl_workspace_bytes.restype = _SZ
 _lib.pl_count_ratio.argtypes = [_P, _P, _P, _P]
 _lib.pl_count_ratio.restype = _I
+_lib.pl_init.argtypes = [_I64, _P]
+_lib.pl_init.restype = _I
 _lib.pl_scale.argtypes = [_P, _I64, _U32, _P, _P]
 _lib.pl_scale.restype = _I
 _lib.pl_device_status.argtypes = [_P, _P]
@@ -93,7 +95,7 @@ _lib.pl_debug_set_rkl_cluster.restype = _I
 _lib.pl_debug_launch_count.argtypes = []
 _lib.pl_debug_launch_count.restype = _I64
 
-EXPORTED = ("pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_linear_grpo_temp", "pl_fused_selective_logprob",
+EXPORTED = ("pl_init", "pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_linear_grpo_temp", "pl_fused_selective_logprob",
             "pl_fused_selective_logprob_workspace_bytes", "pl_reverse_kl", "pl_reverse_kl_workspace_bytes", "pl_scale", "pl_count_ratio", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
             "pl_version", "pl_debug_gemm", "pl_debug_timing", "pl_debug_timing_read",
@@ -135,6 +137,10 @@ def check(status: int, where: str = "libpl") -> None:
 
 
 # ---- C entry points ---------------------------------------------------------------
+def pl_init(max_bs, stream=None) -> int:
+    return _lib.pl_init(max_bs, _stream(stream))
+
+
 def pl_loss(policy_lp, old_lp, ref_lp, adv, mask, bs, seq, eps_lo, eps_hi, beta, mode, loss_out,
             grad_out, stream=None) -> int:
     return _lib.pl_loss(_ptr(policy_lp), _ptr(old_lp), _ptr(ref_lp), _ptr(adv), _ptr(mask), bs, seq,

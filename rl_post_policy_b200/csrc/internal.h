@@ -126,4 +126,7 @@ pl_status check_arch();
 // synchronises the stream).  *out is NULL when none exists and !create.
 pl_status own_workspace(cudaStream_t stream, size_t need, void** out, bool create);
 
+// Bytes of a reverse-KL workspace (header + per-cluster loss partials).
+size_t reverse_kl_ws_bytes();
+
 }  // namespace pl

@@ -145,6 +145,15 @@ using namespace pl;
 
 extern "C" {
 
+pl_status pl_init(int64_t max_bs, pl_stream_t stream) {
+  if (max_bs < 0) return PL_ERR_ARG;
+  pl_status st = check_arch();
+  if (st != PL_OK) return st;
+  void* ws = nullptr;
+  const size_t need = std::max(loss_ws_bytes(max_bs), reverse_kl_ws_bytes());
+  return own_workspace(reinterpret_cast<cudaStream_t>(stream), need, &ws, true);
+}
+
 pl_status pl_loss(const void* policy_lp, const void* old_lp, const void* ref_lp, const void* adv,
                   const uint8_t* mask, int64_t bs, int64_t seq, float eps_lo, float eps_hi,
                   float beta, uint32_t mode, float* loss_out, void* grad_out, pl_stream_t stream) {

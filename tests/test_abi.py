@@ -165,3 +165,12 @@ def test_reverse_kl_rejects_invalid_arguments(over, code):
 def test_reverse_kl_valid_call_without_device():
     # element-aligned (not 16-byte aligned) pointers and a NULL workspace pass validation
     assert _rkl(student=FAKE + 2, workspace=None, ws_bytes=0) in (pl.PL_ERR_CUDA, pl.PL_ERR_ARCH)
+
+
+def test_init_rejects_negative_batch():
+    assert pl.pl_init(-1, stream=0) == pl.PL_ERR_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_init_without_device():
+    assert pl.pl_init(16, stream=0) in (pl.PL_ERR_CUDA, pl.PL_ERR_ARCH)

@@ -122,3 +122,31 @@ def test_graphed_loss_kernel_matches_eager_calls():
     torch.cuda.synchronize()
     assert pl.pl_device_status(ws) == 0
     assert torch.equal(loss, want_loss) and torch.equal(grad, want_grad)
+
+
+def test_pl_init_lets_the_first_library_scratch_call_be_captured():
+    # pl_init creates the per-stream scratch up front, so the very first pl_loss call
+    # on that stream allocates nothing and can be captured into a graph
+    import rl_post_policy_b200 as pl
+    import synth
+    s = torch.cuda.Stream()
+    assert pl.pl_init(16, s) == 0
+    inp = synth.loss_inputs(16, 512, torch.bfloat16, synth.seed_for(1, 3), len_lo=32, len_hi=512)
+    d = {k: inp[k].cuda() for k in ("policy_lp", "old_lp", "ref_lp", "adv", "mask")}
+    loss = torch.zeros(1, device="cuda")
+    grad = torch.empty_like(d["policy_lp"])
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        pl.check(pl.pl_loss(d["policy_lp"], d["old_lp"], d["ref_lp"], d["adv"], d["mask"], 16, 512, 0.2, 0.28,
+                            0.04, pl.PL_BF16 | pl.PL_GRPO, loss, grad))
+    g.replay()
+    torch.cuda.synchronize()
+    lossb = torch.zeros(1, device="cuda")
+    gradb = torch.empty_like(grad)
+    wsb = pl.pl_loss_workspace_bytes(16, 512)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    pl.check(pl.pl_loss_ex(d["policy_lp"], d["old_lp"], d["ref_lp"], d["adv"], d["mask"], 16, 512, 0.2, 0.28,
+                           0.04, pl.PL_BF16 | pl.PL_GRPO, lossb, gradb, None, None, ws, wsb))
+    torch.cuda.synchronize()
+    assert torch.equal(loss, lossb) and torch.equal(grad, gradb)
