@@ -26,6 +26,20 @@ pl_status pl_debug_gemm(const void* A, int a_mn, int64_t lda, const void* B, int
                         float* D, int64_t M, int64_t N, int64_t K, uint32_t mode, pl_stream_t stream);
 
 /*
+ * The same GEMM written to D[m*ldd + n] (ldd >= N) through one of the
+ * epilogue's three fp32 output paths:
+ *   out_path 0: per-thread row stores from registers      D  = A.B
+ *   out_path 1: staged in shared memory, TMA tile store   D  = A.B
+ *   out_path 2: staged in shared memory, TMA add          D += A.B
+ * Paths 1 and 2 need D 16-byte aligned and N and ldd multiples of 4 (else
+ * PL_ERR_ALIGN); no path writes D[m*ldd + n] for n >= N or m >= M.  Path 2 is what accumulates dW across the fused
+ * path's row chunks.  PL_ERR_ARG for another out_path.
+ */
+pl_status pl_debug_gemm_out(const void* A, int a_mn, int64_t lda, const void* B, int b_mn, int64_t ldb,
+                            float* D, int64_t ldd, int out_path, int64_t M, int64_t N, int64_t K,
+                            uint32_t mode, pl_stream_t stream);
+
+/*
  * Kernel timing for the benchmark.  While enabled, every kernel the library
  * launches is bracketed by a pair of CUDA events recorded on the launching
  * stream.  pl_debug_timing_read() waits for the recorded events, returns per

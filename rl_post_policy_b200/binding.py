@@ -80,6 +80,8 @@ _lib.pl_version.argtypes = []
 _lib.pl_version.restype = _I
 _lib.pl_debug_gemm.argtypes = [_P, _I, _I64, _P, _I, _I64, _P, _I64, _I64, _I64, _U32, _P]
 _lib.pl_debug_gemm.restype = _I
+_lib.pl_debug_gemm_out.argtypes = [_P, _I, _I64, _P, _I, _I64, _P, _I64, _I, _I64, _I64, _I64, _U32, _P]
+_lib.pl_debug_gemm_out.restype = _I
 _lib.pl_debug_timing.argtypes = [_I]
 _lib.pl_debug_timing.restype = None
 _lib.pl_debug_timing_read.argtypes = [_P, _P]
@@ -98,7 +100,7 @@ _lib.pl_debug_launch_count.restype = _I64
 EXPORTED = ("pl_init", "pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_linear_grpo_temp", "pl_fused_selective_logprob",
             "pl_fused_selective_logprob_workspace_bytes", "pl_reverse_kl", "pl_reverse_kl_workspace_bytes", "pl_scale", "pl_count_ratio", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
-            "pl_version", "pl_debug_gemm", "pl_debug_timing", "pl_debug_timing_read",
+            "pl_version", "pl_debug_gemm", "pl_debug_gemm_out", "pl_debug_timing", "pl_debug_timing_read",
             "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_set_gemm_tile", "pl_debug_pair_tiles")
 
 
@@ -240,6 +242,13 @@ def pl_debug_gemm(A, a_mn, lda, B, b_mn, ldb, D, M, N, K, mode, stream=None) -> 
     """Test hook (include/pl_debug.h): plain GEMM through the tcgen05 kernel."""
     return _lib.pl_debug_gemm(_ptr(A), int(a_mn), lda, _ptr(B), int(b_mn), ldb, _ptr(D), M, N, K,
                               mode, _stream(stream))
+
+
+def pl_debug_gemm_out(A, a_mn, lda, B, b_mn, ldb, D, ldd, out_path, M, N, K, mode, stream=None) -> int:
+    """Test hook (include/pl_debug.h): the same GEMM through a chosen fp32 output path
+    (0 row stores, 1 TMA store, 2 TMA add into D)."""
+    return _lib.pl_debug_gemm_out(_ptr(A), int(a_mn), lda, _ptr(B), int(b_mn), ldb, _ptr(D), ldd, int(out_path),
+                                  M, N, K, mode, _stream(stream))
 
 
 def pl_debug_timing(enable: bool) -> None:

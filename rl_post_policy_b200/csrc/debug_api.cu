@@ -4,15 +4,20 @@
 
 using namespace pl;
 
-extern "C" pl_status pl_debug_gemm(const void* A, int a_mn, int64_t lda, const void* B, int b_mn,
-                                   int64_t ldb, float* D, int64_t M, int64_t N, int64_t K, uint32_t mode,
-                                   pl_stream_t stream) {
+extern "C" pl_status pl_debug_gemm_out(const void* A, int a_mn, int64_t lda, const void* B, int b_mn,
+                                       int64_t ldb, float* D, int64_t ldd, int out_path, int64_t M, int64_t N,
+                                       int64_t K, uint32_t mode, pl_stream_t stream) {
   if (!A || !B || !D || M < 1 || N < 1 || K < 1) return PL_ERR_ARG;
-  if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return PL_ERR_ARG;
+  if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30) || ldd < N) return PL_ERR_ARG;
+  if (out_path < kOutDirect || out_path > kOutTmaReduce) return PL_ERR_ARG;
   const uint32_t dcode = (mode & PL_DTYPE_MASK) >> 4;
   if (dcode != 1 && dcode != 2) return PL_ERR_DTYPE;
   if (mode & ~PL_DTYPE_MASK) return PL_ERR_ARG;
   if ((lda % 8) || (ldb % 8) || (((uintptr_t)A) & 15) || (((uintptr_t)B) & 15)) return PL_ERR_ALIGN;
+  // The TMA paths need 16-byte rows: and N * 4 bytes a multiple of 16 as well,
+  // since a store was seen to write the whole 16-byte chunk that holds the
+  // last column of a row.
+  if (out_path != kOutDirect && ((ldd % 4) || (N % 4) || (((uintptr_t)D) & 15))) return PL_ERR_ALIGN;
   if (lda < (a_mn ? M : K) || ldb < (b_mn ? N : K)) return PL_ERR_ARG;
   pl_status st = check_arch();
   if (st != PL_OK) return st;
@@ -27,14 +32,22 @@ extern "C" pl_status pl_debug_gemm(const void* A, int a_mn, int64_t lda, const v
                  : make_tmap_2d(&p.maps[0], A, dt, K, M, lda * 2, kBK, kBM);
   ok = ok && (b_mn ? make_tmap_2d(&p.maps[1], B, dt, N, K, ldb * 2, 64, kBK)
                    : make_tmap_2d(&p.maps[1], B, dt, K, N, ldb * 2, kBK, kBNh));
+  if (out_path != kOutDirect) ok = ok && make_tmap_2d(&p.maps[4], D, DType::F32, N, M, ldd * 4, kOutBoxN, kOutBoxM);
   if (!ok) return PL_ERR_CUDA;
   GemmJob& j = p.jobs[0];
   j.a_map = 0; j.b_map = 1; j.a_mn = a_mn ? 1 : 0; j.b_mn = b_mn ? 1 : 0;
   j.M = (int)M; j.N = (int)N; j.K = (int)K; j.n_inner = 0; j.epi = kEpiStore;
-  j.out = D; j.out_f32 = 1; j.acc_in = nullptr; j.out_ld = N; j.scale = nullptr;
+  j.out = D; j.out_f32 = 1; j.acc_in = nullptr; j.out_ld = ldd; j.scale = nullptr;
+  j.out_path = out_path; j.out_map = 4;
   p.njobs = 1;
   gemm_finalize_jobs(&p);
   return launch_gemm(p, dt, s) == cudaSuccess ? PL_OK : PL_ERR_CUDA;
+}
+
+extern "C" pl_status pl_debug_gemm(const void* A, int a_mn, int64_t lda, const void* B, int b_mn,
+                                   int64_t ldb, float* D, int64_t M, int64_t N, int64_t K, uint32_t mode,
+                                   pl_stream_t stream) {
+  return pl_debug_gemm_out(A, a_mn, lda, B, b_mn, ldb, D, N, kOutDirect, M, N, K, mode, stream);
 }
 
 // pl_debug_pair_tiles: the GEMM's tile schedule for two jobs (t0 tiles of c0

@@ -83,6 +83,9 @@ cudaError_t launch_dlogits(const DlogitsArgs& a, DType dt, cudaStream_t s);
 cudaError_t launch_combine_ext(const CombineArgs& a, cudaStream_t s);
 // Zeroes the per-chunk max|g| slots (the count kernel does it in the loss form).
 cudaError_t launch_clear_gmax(unsigned char* ws, int nchunks, const FusedOffsets& off, cudaStream_t s);
+// out[0..n) = acc[0..n) rounded to the model dtype (n a multiple of 8; 16-byte
+// vectors when both pointers are 16-byte aligned, element stores otherwise).
+cudaError_t launch_convert(const float* acc, void* out, int64_t n, DType dt, cudaStream_t s);
 cudaError_t launch_finalize(const unsigned char* ws, const FusedOffsets& off, int nchunks, int part_stride,
                             int nblocks_last, float* loss, int64_t* n_valid_out, cudaStream_t s);
 

@@ -238,17 +238,26 @@ pl_status run_pipeline(const Pipe& q) {
       j.a_map = 2; j.b_map = 3; j.a_mn = 1; j.b_mn = 1;
       j.M = (int)V; j.N = (int)H; j.K = (int)rows; j.n_inner = 1; j.epi = kEpiStore;
       j.out_ld = H; j.scale = inv_scale;
+      // Several chunks: the first stores its fp32 contribution, every later one
+      // adds its own through the TMA unit (the memory system does the add, so
+      // the epilogue never waits on a load), and the sum is rounded to the
+      // model dtype once, after the last chunk.
       float* acc = reinterpret_cast<float*>(ws + plan.off.dw_acc);
-      switch (acc_mode(c, plan.nchunks)) {
-        case kAccStoreModel: j.out = dW; j.out_f32 = 0; j.acc_in = nullptr; break;
-        case kAccStoreF32: j.out = acc; j.out_f32 = 1; j.acc_in = nullptr; break;
-        case kAccAddF32: j.out = acc; j.out_f32 = 1; j.acc_in = acc; break;
-        default: j.out = dW; j.out_f32 = 0; j.acc_in = acc; break;
+      j.acc_in = nullptr;
+      if (plan.nchunks == 1) {
+        j.out = dW; j.out_f32 = 0; j.out_path = kOutDirect;
+      } else {
+        if (!make_tmap_2d(&bp.maps[4], acc, DType::F32, H, V, H * 4, kOutBoxN, kOutBoxM)) return PL_ERR_CUDA;
+        j.out = acc; j.out_f32 = 1; j.out_map = 4;
+        j.out_path = c == 0 ? kOutTmaStore : kOutTmaReduce;
       }
     }
     bp.njobs = nj;
     gemm_finalize_jobs(&bp);
     if (!ok(launch_gemm(bp, dt, s))) return PL_ERR_CUDA;
+    if (dW && plan.nchunks > 1 && c + 1 == plan.nchunks &&
+        !ok(launch_convert(reinterpret_cast<const float*>(ws + plan.off.dw_acc), dW, V * H, dt, s)))
+      return PL_ERR_CUDA;
   }
 
   if (q.ext_g) return PL_OK;

@@ -12,6 +12,8 @@
 //                      model dtype, and the column sums of dz (the bias gradient),
 //                      stored / accumulated in fp32 / converted like dW.
 //   finalize_kernel -- fixed-order sum of every chunk's loss partials.
+//   convert_kernel  -- the fp32 dW accumulator of a multi-chunk call, rounded
+//                      once to the model dtype after the last chunk's add.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -28,6 +30,15 @@ template <> __device__ __forceinline__ __nv_bfloat16 to_t<__nv_bfloat16>(float x
   return __float2bfloat16_rn(x);
 }
 template <> __device__ __forceinline__ __half to_t<__half>(float x) { return __float2half_rn(x); }
+template <typename T> __device__ __forceinline__ uint32_t pack_t(float a, float b);
+template <> __device__ __forceinline__ uint32_t pack_t<__nv_bfloat16>(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+template <> __device__ __forceinline__ uint32_t pack_t<__half>(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
 
 // ---------------------------------------------------------------- counts
 __global__ void count_kernel(const uint8_t* __restrict__ mask, int64_t bs, int64_t T,
@@ -387,6 +398,65 @@ cudaError_t launch_dlogits(const DlogitsArgs& a0, DType dt, cudaStream_t s) {
     { launch_begin(2, s); dlogits_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
   } else {
     { launch_begin(2, s); dlogits_kernel<__half><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
+  }
+  return cudaGetLastError();
+}
+
+namespace {
+// out[i] = round(acc[i]) for n = 8 * n8 elements; 8 per thread per step (two
+// 16-byte loads that bypass L1 and are marked read-once, one 16-byte store).
+template <typename T>
+__global__ void __launch_bounds__(256) convert_kernel(const float4* __restrict__ acc, uint4* __restrict__ out,
+                                                      int64_t n8) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const float4 a = __ldcs(acc + 2 * i), b = __ldcs(acc + 2 * i + 1);
+    uint4 o;
+    o.x = pack_t<T>(a.x, a.y);
+    o.y = pack_t<T>(a.z, a.w);
+    o.z = pack_t<T>(b.x, b.y);
+    o.w = pack_t<T>(b.z, b.w);
+    out[i] = o;
+  }
+}
+// The same for an output that is not 16-byte aligned (element stores).
+template <typename T>
+__global__ void __launch_bounds__(256) convert_kernel_unaligned(const float* __restrict__ acc, T* __restrict__ out,
+                                                                int64_t n) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) out[i] = to_t<T>(acc[i]);
+}
+}  // namespace
+
+cudaError_t launch_convert(const float* acc, void* out, int64_t n, DType dt, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  if (n % 8) return cudaErrorInvalidValue;
+  DevInfo di;
+  cudaError_t e = dev_info(&di);
+  if (e != cudaSuccess) return e;
+  const int64_t n8 = n / 8;
+  int64_t blocks = (n8 + 255) / 256;
+  const int64_t cap = (int64_t)di.sm_count * 8;  // 8 resident blocks of 256 threads per SM
+  if (blocks > cap) blocks = cap;
+  const unsigned g = (unsigned)blocks;
+  if ((reinterpret_cast<uintptr_t>(out) & 15) || (reinterpret_cast<uintptr_t>(acc) & 15)) {
+    if (dt == DType::BF16) {
+      launch_begin(2, s);
+      convert_kernel_unaligned<__nv_bfloat16><<<g, 256, 0, s>>>(acc, static_cast<__nv_bfloat16*>(out), n);
+      launch_end(2, s);
+    } else {
+      launch_begin(2, s);
+      convert_kernel_unaligned<__half><<<g, 256, 0, s>>>(acc, static_cast<__half*>(out), n);
+      launch_end(2, s);
+    }
+    return cudaGetLastError();
+  }
+  const float4* a = reinterpret_cast<const float4*>(acc);
+  uint4* o = reinterpret_cast<uint4*>(out);
+  if (dt == DType::BF16) {
+    { launch_begin(2, s); convert_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(a, o, n8); launch_end(2, s); }
+  } else {
+    { launch_begin(2, s); convert_kernel<__half><<<g, 256, 0, s>>>(a, o, n8); launch_end(2, s); }
   }
   return cudaGetLastError();
 }

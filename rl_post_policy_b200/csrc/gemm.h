@@ -24,6 +24,18 @@ enum EpiKind : int {
   kEpiStore = 1,  // acc * scale (+ fp32 acc_in) -> out (model dtype or fp32)
 };
 
+// How a kEpiStore job writes its fp32 result (out_f32 = 1 only).
+enum OutPath : int {
+  kOutDirect = 0,     // per-thread row stores (and acc_in loads) from registers
+  kOutTmaStore = 1,   // staged in shared memory, TMA tile store through maps[out_map]
+  kOutTmaReduce = 2,  // staged in shared memory, TMA element-wise add into maps[out_map]
+};
+
+// fp32 output tensor maps cover [M, out_ld] with {kOutBoxN, kOutBoxM} boxes,
+// 128-byte swizzle: one box is one epilogue warp's 32 rows x 32 columns.
+constexpr int kOutBoxN = 32;
+constexpr int kOutBoxM = 32;
+
 // One GEMM problem D[M,N] = sum_k A(m,k) B(n,k), tiled kPairM x kBN.
 //   A(m,k): K-major means A[m*lda + k]; MN-major means A[k*lda + m] (likewise B).
 struct GemmJob {
@@ -46,13 +58,15 @@ struct GemmJob {
   // kEpiStore
   void* out;
   int out_f32;
+  int out_path;            // OutPath; kOutTma* need out_f32 = 1, acc_in = null and out_map
+  int out_map;             // tensor-map index of `out` for the kOutTma* paths
   const float* acc_in;     // [M, out_ld] fp32 added before the store, or null
   int64_t out_ld;
   const float* scale;      // device scalar multiplier, or null for 1
 };
 
 struct __align__(64) GemmParams {
-  CUtensorMap maps[4];
+  CUtensorMap maps[5];
   GemmJob jobs[2];
   int njobs;
   int total_tiles;
@@ -70,9 +84,10 @@ struct __align__(64) GemmParams {
 
 // Tensor-map boxes: K-major operands load {kBK, kBM} (A) or {kBK, kBNh} (B)
 // boxes; MN-major operands load {64, kBK} boxes, two per 128 rows/columns.
-// Encodes a 2-D tensor map over a row-major [outer, inner] array of 16-bit
-// elements with a row pitch of `pitch_bytes`, box {box_inner, box_outer},
-// 128-byte swizzle, zero fill outside the extent.
+// Encodes a 2-D tensor map over a row-major [outer, inner] array of `dt`
+// elements (16-bit, or fp32 for the kOutTma* outputs) with a row pitch of
+// `pitch_bytes`, box {box_inner, box_outer}, 128-byte swizzle, zero fill
+// outside the extent.
 bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, uint64_t outer,
                   uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
 

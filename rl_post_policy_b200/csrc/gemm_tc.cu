@@ -50,6 +50,10 @@ using namespace sm100;
 constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t kBBytes = kBNh * kBK * 2;            // 16 KB: this CTA's 128 rows of B per MMA
 constexpr uint32_t kTmemCols = 512;
+// Epilogue staging for the TMA output paths: per epilogue warp, two buffers of
+// one 32 x 32 fp32 box (4 KB), so a warp fills one while the other drains.
+constexpr uint32_t kOutBoxBytes = kOutBoxM * kOutBoxN * 4;
+constexpr uint32_t kOutStageBytes = 4 * 2 * kOutBoxBytes;
 
 // Pair tile kPairM x (kBN * NH).  NH = 1: one N=256 MMA per K=16 step, two
 // accumulators alternating between tiles (the epilogue of tile t overlaps the
@@ -61,7 +65,12 @@ struct TileCfg {
   static constexpr int kTileN = kBN * NH;
   static constexpr int kStages = NH == 1 ? 6 : 4;
   static constexpr uint32_t kStageBytes = kABytes + NH * kBBytes;
-  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256;
+  // [alignment slack][operand ring][barriers, padded to 1 KB][output staging].
+  // Launches without a TMA output path leave the staging off the allocation,
+  // which keeps 32 KB more of the SM's unified L1 / shared memory as L1.
+  static constexpr size_t kSmemBase = 1024 + kStages * kStageBytes + 1024;
+  static constexpr size_t kSmem = kSmemBase + kOutStageBytes;
+  static_assert(kSmem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
 };
 
 __device__ __forceinline__ float cvt_in(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -215,6 +224,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* out_stage = smem + kStages * kStageBytes + 1024;  // 1024-byte aligned; only with a TMA output
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -244,6 +254,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     for (int q = 0; q < p.njobs; ++q) {
       prefetch_tmap(&p.maps[p.jobs[q].a_map]);
       prefetch_tmap(&p.maps[p.jobs[q].b_map]);
+      if (p.jobs[q].out_path != kOutDirect) prefetch_tmap(&p.maps[p.jobs[q].out_map]);
     }
   }
   if (warp == 1) {
@@ -432,6 +443,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     // the jobs' device scale factors, read once per launch rather than per tile
     const float job_scale0 = p.jobs[0].scale ? __ldg(p.jobs[0].scale) : 1.0f;
     const float job_scale1 = (p.njobs > 1 && p.jobs[1].scale) ? __ldg(p.jobs[1].scale) : 1.0f;
+    // this warp's two staging boxes for the TMA output paths
+    const uint32_t stage0 = smem_u32(out_stage) + (uint32_t)quarter * 2 * kOutBoxBytes;
+    int sbuf = 0;
     for (int it = 0;; ++it) {
       const int tile = pair_tile(p, pair, npairs, it);
       if (tile < 0) break;
@@ -513,6 +527,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             j.part[(int64_t)row * j.part_ld + grp] = make_float2(m_run, s_run);
             if (got) j.zt[row] = ztv;
           }
+        } else if (j.out_path != kOutDirect) {
+          // fp32 result through shared memory and the TMA unit: each warp
+          // stages its 32 rows x 32 columns in one 4 KB box (128-byte swizzle:
+          // 16-byte chunk q of row r sits at chunk q ^ (r % 8), so a warp's
+          // 16-byte stores hit every bank once per 8 lanes) and lane 0 issues
+          // the box's store or add.  Rows and columns past the output's extent
+          // are dropped by the TMA unit.
+          const float sc = tc.job ? job_scale1 : job_scale0;
+          const CUtensorMap* omap = &p.maps[j.out_map];
+          const int y = m0 + quarter * 32;
+  #pragma unroll 1
+          for (int c = 0; c < kBN / 32; ++c) {
+            float v[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, v);
+            const int col0 = n0 + c * 32;
+            if (col0 >= j.N || y >= j.M) continue;
+            // the box written two slices ago has been read out of shared memory
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            const uint32_t box = stage0 + (uint32_t)sbuf * kOutBoxBytes;
+            const uint32_t my_row = box + (uint32_t)lane * 128u;
+  #pragma unroll
+            for (int q = 0; q < 8; ++q)
+              st_shared_v4(my_row + ((uint32_t)(q ^ (lane & 7)) << 4), v[4 * q] * sc, v[4 * q + 1] * sc,
+                           v[4 * q + 2] * sc, v[4 * q + 3] * sc);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (j.out_path == kOutTmaReduce) tma_reduce_add_2d(omap, box, col0, y);
+              else tma_store_2d(omap, box, col0, y);
+              bulk_commit_group();
+            }
+            sbuf ^= 1;
+          }
         } else {
           const float sc = tc.job ? job_scale1 : job_scale0;
   #pragma unroll 1
@@ -542,6 +590,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         acc_phase ^= 1;
       }
     }
+    // every TMA store / add this warp issued has been performed before exit
+    if (lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();
@@ -647,7 +697,7 @@ cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (max_pairs == 0) {
+  if (max_pairs == 0) {  // one CTA per SM with or without the output staging
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel<T, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
     if (e != cudaSuccess) return e;
     DevInfo di;
@@ -658,6 +708,9 @@ cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     max_pairs = n > 0 ? n : 1;
   }
+  bool tma_out = false;
+  for (int i = 0; i < p.njobs; ++i) tma_out = tma_out || p.jobs[i].out_path != kOutDirect;
+  if (!tma_out) cfg.dynamicSmemBytes = TileCfg<NH>::kSmemBase;
   const int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
   cfg.gridDim = dim3(2 * pairs);
   GemmParams q = p;
@@ -718,8 +771,9 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, 
   const cuuint64_t strides[1] = {pitch_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapDataType t =
-      dt == DType::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapDataType t = dt == DType::BF16  ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                : dt == DType::F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   CUresult r = fn(map, t, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

@@ -1,5 +1,5 @@
 // Inline-PTX wrappers for the sm_100a features the GEMMs use: mbarriers with
-// bounded waits, TMA tile loads, tensor-memory allocation and loads, and the
+// bounded waits, TMA tile loads, stores and adds, tensor-memory allocation and loads, and the
 // 5th-generation tensor-core MMA (tcgen05) with its shared-memory operand
 // descriptors, in single-CTA and CTA-pair forms.  Only what the kernels here
 // need.  No load uses multicast: the one multicast is tcgen05.commit's
@@ -139,6 +139,41 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y)
       : "memory");
+}
+
+// 2-D tiled bulk tensor store from this CTA's shared memory, or an element-wise
+// add of the shared-memory tile into global memory performed by the memory
+// system (the tensor map's element type, here fp32).  Both join the issuing
+// thread's current bulk async-group.  Elements outside the tensor's extent are
+// not written.  x (elements) must be a multiple of 4 for 32-bit elements and
+// y must be non-negative; every caller passes x a multiple of 32 and y >= 0.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src_saddr, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src_saddr), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src_saddr, int32_t x,
+                                                  int32_t y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src_saddr), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Waits until every bulk group of this thread has completed (writes performed).
+__device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA) reads of the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t saddr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
 }
 
 // ---------------------------------------------------------------- tensor memory

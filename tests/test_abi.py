@@ -174,3 +174,18 @@ def test_init_rejects_negative_batch():
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
 def test_init_without_device():
     assert pl.pl_init(16, stream=0) in (pl.PL_ERR_CUDA, pl.PL_ERR_ARCH)
+
+
+def test_debug_gemm_out_rejects_invalid_arguments():
+    base = dict(A=FAKE, a_mn=0, lda=64, B=FAKE, b_mn=0, ldb=64, D=FAKE, ldd=256, out_path=2, M=128, N=256,
+                K=64, mode=pl.PL_BF16)
+    for over, code in [(dict(out_path=3), pl.PL_ERR_ARG), (dict(out_path=-1), pl.PL_ERR_ARG),
+                       (dict(ldd=255), pl.PL_ERR_ARG),           # ldd < N
+                       (dict(ldd=258), pl.PL_ERR_ALIGN),         # TMA rows must be 16-byte pitched
+                       (dict(N=254), pl.PL_ERR_ALIGN),           # and end on a 16-byte boundary
+                       (dict(N=254, out_path=0), pl.PL_ERR_CUDA),  # row stores take any N (no device here)
+                       (dict(D=FAKE + 4), pl.PL_ERR_ALIGN), (dict(mode=pl.PL_F32), pl.PL_ERR_DTYPE),
+                       (dict(D=None), pl.PL_ERR_ARG)]:
+        args = dict(base)
+        args.update(over)
+        assert pl.pl_debug_gemm_out(**args, stream=0) == code, over

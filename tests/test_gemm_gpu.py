@@ -60,3 +60,53 @@ def test_many_tiles_persistent():
     # more tiles than SMs: every CTA walks several tiles and both accumulators
     run(1024, 8192, 256, 0, 0, torch.bfloat16, seed=3)
     run(2048, 1024, 1024, 1, 1, torch.bfloat16, seed=4)
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (1, 1)])
+@pytest.mark.parametrize("shape", [(256, 512, 192), (333, 300, 136), (1, 4, 8), (700, 2052, 520)])
+def test_tma_output_paths(a_mn, b_mn, shape):
+    """The staged TMA store (path 1) and TMA add (path 2): D = A.B, then D += A.B
+    over a random start, on a pitched D whose pad rows and columns must stay
+    untouched (the TMA unit drops what lies past [M, N])."""
+    m = __import__("rl_post_policy_b200")
+    M, N, K = shape
+    g = torch.Generator().manual_seed(M * 7 + N + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    B = torch.randn(N, K, generator=g).to(torch.bfloat16)
+
+    def pitched(t, rows, cols):
+        ld = (cols + 7) // 8 * 8
+        out = torch.zeros(rows, ld, dtype=t.dtype)
+        out[:, :cols] = t
+        return out.cuda(), ld
+
+    Ad, lda = pitched(A.t(), K, M) if a_mn else pitched(A, M, K)
+    Bd, ldb = pitched(B.t(), K, N) if b_mn else pitched(B, N, K)
+    ldd = N + 8
+    sentinel = 12345.0
+    R = torch.randn(M, N, generator=g)
+    ref = A.double() @ B.double().t()
+    bound = A.double().abs() @ B.double().abs().t()
+    mode = m.dtype_mode(torch.bfloat16)
+
+    def fresh(start):
+        D = torch.full((M + 5, ldd), sentinel)
+        D[:M, :N] = start
+        return D.cuda()
+
+    def check(D, want, extra):
+        torch.cuda.synchronize()
+        m.check(m.pl_device_status(None), "device status")
+        D = D.cpu().double()
+        err = (D[:M, :N] - want).abs()
+        assert torch.all(err <= 1e-5 * (bound + extra) + 1e-6), float(err.max())
+        assert torch.all(D[:M, N:] == sentinel) and torch.all(D[M:] == sentinel)
+
+    D = fresh(float("nan"))
+    m.check(m.pl_debug_gemm_out(Ad, a_mn, lda, Bd, b_mn, ldb, D, ldd, 1, M, N, K, mode), "store")
+    check(D, ref, 0.0)
+    m.check(m.pl_debug_gemm_out(Ad, a_mn, lda, Bd, b_mn, ldb, D, ldd, 2, M, N, K, mode), "add")
+    check(D, 2 * ref, bound)
+    D = fresh(R)
+    m.check(m.pl_debug_gemm_out(Ad, a_mn, lda, Bd, b_mn, ldb, D, ldd, 2, M, N, K, mode), "add")
+    check(D, R.double() + ref, R.double().abs())
