@@ -80,6 +80,15 @@ int pl_debug_set_rkl_cluster(int cl);
 int pl_debug_set_gemm_tile(int nh);
 
 /*
+ * The GEMM launcher's tile-width choice (host logic, no device call): for
+ * njobs = 1 or 2 problems given as mnk = {M0, N0, K0[, M1, N1, K1]} on `pairs`
+ * CTA pairs, returns 1 (256-wide tiles) or 2 (512-wide), or -1 on bad input.
+ * The fused path's forward launch is {N, V, H} for the policy and reference;
+ * its backward launch is {N, H, V} (dX) and {V, H, N} (dW).
+ */
+int pl_debug_pick_tile(int njobs, const int64_t* mnk, int pairs);
+
+/*
  * The persistent GEMM's tile schedule, for a host-side check: two problems of
  * t0 tiles (c0 k-steps each) and t1 tiles (c1 k-steps each) over `pairs` CTA
  * pairs.  out_pair[t] (t0 + t1 entries) receives the pair that runs tile t.

@@ -90,6 +90,8 @@ _lib.pl_debug_set_wait.argtypes = [ctypes.c_ulonglong, ctypes.c_uint, ctypes.c_u
 _lib.pl_debug_set_wait.restype = None
 _lib.pl_debug_pair_tiles.argtypes = [_I, _I, _I, _I, _I, _P]
 _lib.pl_debug_pair_tiles.restype = _I
+_lib.pl_debug_pick_tile.argtypes = [_I, _P, _I]
+_lib.pl_debug_pick_tile.restype = _I
 _lib.pl_debug_set_gemm_tile.argtypes = [_I]
 _lib.pl_debug_set_gemm_tile.restype = _I
 _lib.pl_debug_set_rkl_cluster.argtypes = [_I]
@@ -101,7 +103,8 @@ EXPORTED = ("pl_init", "pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_line
             "pl_fused_selective_logprob_workspace_bytes", "pl_reverse_kl", "pl_reverse_kl_workspace_bytes", "pl_scale", "pl_count_ratio", "pl_loss_workspace_bytes", "pl_fused_linear_grpo",
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
             "pl_version", "pl_debug_gemm", "pl_debug_gemm_out", "pl_debug_timing", "pl_debug_timing_read",
-            "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_set_gemm_tile", "pl_debug_pair_tiles")
+            "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_set_gemm_tile", "pl_debug_pair_tiles",
+            "pl_debug_pick_tile")
 
 
 class PLError(RuntimeError):
@@ -285,3 +288,10 @@ def pl_debug_pair_tiles(t0: int, t1: int, c0: int, c1: int, pairs: int):
     out = (ctypes.c_int32 * max(t0 + t1, 1))()
     rc = _lib.pl_debug_pair_tiles(t0, t1, c0, c1, pairs, out)
     return int(rc), list(out)[: t0 + t1]
+
+
+def pl_debug_pick_tile(problems, pairs: int) -> int:
+    """Test hook: the GEMM launcher's tile width (1 or 2) for one or two (M, N, K) problems."""
+    flat = [int(x) for mnk in problems for x in mnk]
+    arr = (ctypes.c_int64 * max(len(flat), 1))(*flat)
+    return int(_lib.pl_debug_pick_tile(len(problems), arr, pairs))

@@ -50,6 +50,22 @@ extern "C" pl_status pl_debug_gemm(const void* A, int a_mn, int64_t lda, const v
   return pl_debug_gemm_out(A, a_mn, lda, B, b_mn, ldb, D, N, kOutDirect, M, N, K, mode, stream);
 }
 
+// pl_debug_pick_tile: the tile width the GEMM launcher picks for one or two
+// problems (M, N, K each) on `pairs` CTA pairs.
+extern "C" int pl_debug_pick_tile(int njobs, const int64_t* mnk, int pairs) {
+  if (njobs < 1 || njobs > 2 || !mnk || pairs < 1) return -1;
+  GemmParams p{};
+  p.njobs = njobs;
+  for (int i = 0; i < njobs; ++i) {
+    if (mnk[3 * i] < 1 || mnk[3 * i + 1] < 1 || mnk[3 * i + 2] < 1) return -1;
+    if (mnk[3 * i] > (1 << 30) || mnk[3 * i + 1] > (1 << 30) || mnk[3 * i + 2] > (1 << 30)) return -1;
+    p.jobs[i].M = (int)mnk[3 * i];
+    p.jobs[i].N = (int)mnk[3 * i + 1];
+    p.jobs[i].K = (int)mnk[3 * i + 2];
+  }
+  return pick_tile_width(p, pairs);
+}
+
 // pl_debug_pair_tiles: the GEMM's tile schedule for two jobs (t0 tiles of c0
 // k-steps, then t1 tiles of c1 k-steps) over `pairs` CTA pairs.  Writes, for
 // every tile, the pair that runs it (out_pair[t0 + t1]) and returns 0, or -1 if

@@ -229,6 +229,11 @@ pl_status run_pipeline(const Pipe& q) {
       j.M = (int)rows; j.N = (int)H; j.K = (int)V; j.n_inner = 0; j.epi = kEpiStore;
       j.out = static_cast<unsigned char*>(dX) + r0 * H * esz; j.out_f32 = 0; j.acc_in = nullptr;
       j.out_ld = H; j.scale = inv_scale;
+      // whole 128-byte lines through the TMA unit when dX is 16-byte aligned
+      if (aligned(dX, 16)) {
+        if (!make_tmap_2d(&bp.maps[5], j.out, dt, H, rows, H * esz, kOutBoxN16, kOutBoxM)) return PL_ERR_CUDA;
+        j.out_path = kOutTmaStore; j.out_map = 5;
+      }
     }
     if (dW) {
       if (!make_tmap_2d(&bp.maps[2], ws + plan.off.logits, dt, V, rows, plan.ld * esz, 64, kBK) ||
@@ -246,6 +251,10 @@ pl_status run_pipeline(const Pipe& q) {
       j.acc_in = nullptr;
       if (plan.nchunks == 1) {
         j.out = dW; j.out_f32 = 0; j.out_path = kOutDirect;
+        if (aligned(dW, 16)) {
+          if (!make_tmap_2d(&bp.maps[4], dW, dt, H, V, H * esz, kOutBoxN16, kOutBoxM)) return PL_ERR_CUDA;
+          j.out_path = kOutTmaStore; j.out_map = 4;
+        }
       } else {
         if (!make_tmap_2d(&bp.maps[4], acc, DType::F32, H, V, H * 4, kOutBoxN, kOutBoxM)) return PL_ERR_CUDA;
         j.out = acc; j.out_f32 = 1; j.out_map = 4;

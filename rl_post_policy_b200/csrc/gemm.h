@@ -24,16 +24,19 @@ enum EpiKind : int {
   kEpiStore = 1,  // acc * scale (+ fp32 acc_in) -> out (model dtype or fp32)
 };
 
-// How a kEpiStore job writes its fp32 result (out_f32 = 1 only).
+// How a kEpiStore job writes its result.
 enum OutPath : int {
   kOutDirect = 0,     // per-thread row stores (and acc_in loads) from registers
   kOutTmaStore = 1,   // staged in shared memory, TMA tile store through maps[out_map]
-  kOutTmaReduce = 2,  // staged in shared memory, TMA element-wise add into maps[out_map]
+  kOutTmaReduce = 2,  // fp32 only: staged, TMA element-wise add into maps[out_map]
 };
 
-// fp32 output tensor maps cover [M, out_ld] with {kOutBoxN, kOutBoxM} boxes,
-// 128-byte swizzle: one box is one epilogue warp's 32 rows x 32 columns.
+// Output tensor maps for the kOutTma* paths cover [M, N] (row pitch out_ld)
+// with boxes of kOutBoxM rows x 128 bytes -- kOutBoxN fp32 or kOutBoxN16
+// 16-bit columns -- and the 128-byte swizzle: one box is one epilogue warp's
+// 32 rows.  N * element size must be a multiple of 16 bytes.
 constexpr int kOutBoxN = 32;
+constexpr int kOutBoxN16 = 64;
 constexpr int kOutBoxM = 32;
 
 // One GEMM problem D[M,N] = sum_k A(m,k) B(n,k), tiled kPairM x kBN.
@@ -58,7 +61,7 @@ struct GemmJob {
   // kEpiStore
   void* out;
   int out_f32;
-  int out_path;            // OutPath; kOutTma* need out_f32 = 1, acc_in = null and out_map
+  int out_path;            // OutPath; kOutTma* need acc_in = null and out_map
   int out_map;             // tensor-map index of `out` for the kOutTma* paths
   const float* acc_in;     // [M, out_ld] fp32 added before the store, or null
   int64_t out_ld;
@@ -66,7 +69,7 @@ struct GemmJob {
 };
 
 struct __align__(64) GemmParams {
-  CUtensorMap maps[5];
+  CUtensorMap maps[6];
   GemmJob jobs[2];
   int njobs;
   int total_tiles;
@@ -96,6 +99,11 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, 
 void gemm_finalize_jobs(GemmParams* p);
 
 cudaError_t launch_gemm(const GemmParams& p, DType dt, cudaStream_t stream);
+
+// The tile width launch_gemm uses on P pairs (1: 256 wide, 2: 512 wide) unless
+// a test forces one, from the jobs' M, N, K.
+double launch_estimate(GemmParams p, int nh, int P);
+int pick_tile_width(const GemmParams& p, int P);
 
 // Tile schedule (host side of what the kernel runs): balance_schedule fills
 // sched/na/nb/rem for P pairs; pair_tile gives the i-th tile of a pair or -1.

@@ -528,30 +528,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             if (got) j.zt[row] = ztv;
           }
         } else if (j.out_path != kOutDirect) {
-          // fp32 result through shared memory and the TMA unit: each warp
-          // stages its 32 rows x 32 columns in one 4 KB box (128-byte swizzle:
-          // 16-byte chunk q of row r sits at chunk q ^ (r % 8), so a warp's
-          // 16-byte stores hit every bank once per 8 lanes) and lane 0 issues
-          // the box's store or add.  Rows and columns past the output's extent
-          // are dropped by the TMA unit.
+          // The result through shared memory and the TMA unit.  Each warp
+          // stages its 32 rows in one 4 KB box of 128-byte rows (32 fp32 or 64
+          // 16-bit columns) with the 128-byte swizzle: 16-byte chunk q of row r
+          // sits at chunk q ^ (r % 8), so a warp's 16-byte stores hit every
+          // bank once per 8 lanes.  Lane 0 then issues the box's store (or fp32
+          // add), which the TMA unit writes as whole 128-byte lines.  Rows and
+          // columns past the output's extent are dropped by the TMA unit.
           const float sc = tc.job ? job_scale1 : job_scale0;
           const CUtensorMap* omap = &p.maps[j.out_map];
           const int y = m0 + quarter * 32;
+          const int step = j.out_f32 ? 1 : 2;  // 32-column TMEM slices per box
   #pragma unroll 1
-          for (int c = 0; c < kBN / 32; ++c) {
+          for (int c = 0; c < kBN / 32; c += step) {
+            uint32_t w[32];
             float v[32];
             tmem_ld_32x32b_x32(taddr + c * 32, v);
+            if (j.out_f32) {
+  #pragma unroll
+              for (int q = 0; q < 32; ++q) w[q] = __float_as_uint(v[q] * sc);
+            } else {
+  #pragma unroll
+              for (int q = 0; q < 16; ++q) w[q] = pack2<T>(v[2 * q] * sc, v[2 * q + 1] * sc);
+              tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
+  #pragma unroll
+              for (int q = 0; q < 16; ++q) w[16 + q] = pack2<T>(v[2 * q] * sc, v[2 * q + 1] * sc);
+            }
             const int col0 = n0 + c * 32;
             if (col0 >= j.N || y >= j.M) continue;
-            // the box written two slices ago has been read out of shared memory
+            // the box written two boxes ago has been read out of shared memory
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
             const uint32_t box = stage0 + (uint32_t)sbuf * kOutBoxBytes;
             const uint32_t my_row = box + (uint32_t)lane * 128u;
   #pragma unroll
             for (int q = 0; q < 8; ++q)
-              st_shared_v4(my_row + ((uint32_t)(q ^ (lane & 7)) << 4), v[4 * q] * sc, v[4 * q + 1] * sc,
-                           v[4 * q + 2] * sc, v[4 * q + 3] * sc);
+              st_shared_v4(my_row + ((uint32_t)(q ^ (lane & 7)) << 4), w[4 * q], w[4 * q + 1], w[4 * q + 2],
+                           w[4 * q + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -648,18 +661,24 @@ void balance_schedule(GemmParams* p, int P) {
   p->rem = (int)(T1 - total());
 }
 
-namespace {
 // Estimated launch length, in N=256 MMA k-steps per pair, for pair tiles nh
 // MMAs wide on P pairs: the larger of the even share of all the work and the
 // longest single tile (a tile runs on one pair), or, for one problem of
 // equal-cost tiles, whole waves of tiles.
+// Cost of a launch in k-step units (one K=64 step of one N=256 MMA group): the
+// busiest pair's share.  Each tile also pays a fixed kTileOverhead for its
+// accumulator hand-off and pipeline turn; fitted to the backward launch of a
+// 1024-row chunk (V=128256, H=4096), whose 16-k-step dW tiles ran about 18%
+// slower at 256 wide than at 512 wide.
+constexpr double kTileOverhead = 8.0;
+
 double launch_estimate(GemmParams p, int nh, int P) {
   p.nh = nh;
   gemm_finalize_jobs(&p);
   double work = 0.0, longest = 0.0;
   for (int i = 0; i < p.njobs; ++i) {
     const GemmJob& j = p.jobs[i];
-    const double tile = (double)j.k_steps * nh;
+    const double tile = (double)j.k_steps * nh + kTileOverhead;
     work += (double)j.tiles_m * j.tiles_n * tile;
     if (j.tiles_m * j.tiles_n > 0 && tile > longest) longest = tile;
   }
@@ -671,16 +690,18 @@ double launch_estimate(GemmParams p, int nh, int P) {
   return share > longest ? share : longest;
 }
 
-// 256 x 512 tiles move 25% fewer operand bytes per flop and halve the barrier
-// round trips; measured on this kernel they run the same k-step work about 10%
-// faster when the launch stays balanced.  They need every problem to be at
-// least 512 wide.
+// 256 x 512 tiles move 25% fewer operand bytes per flop, halve the barrier
+// round trips and the tile count; measured on this kernel they run the same
+// k-step work about 10% faster when the launch stays balanced.  They need every
+// problem to be at least 512 wide.
 int pick_tile_width(const GemmParams& p, int P) {
   if (P <= 0) return 1;
   for (int i = 0; i < p.njobs; ++i)
     if (p.jobs[i].N < 2 * kBN) return 1;
   return 0.9 * launch_estimate(p, 2, P) < launch_estimate(p, 1, P) ? 2 : 1;
 }
+
+namespace {
 
 template <typename T, int NH>
 cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {

@@ -39,7 +39,7 @@ def build_inputs(bs, T, H, V, dtype, seed, bias=False, beta=0.04, len_lo=1, len_
 
 
 def run_fused(inp, dtype, red, beta, chunk=None, want=("dX", "dW", "dbias"), two_sided=False,
-              targets=None):
+              targets=None, out_offset=0):
     m = pl()
     dev = "cuda"
     bs, T = inp["mask"].shape
@@ -54,10 +54,18 @@ def run_fused(inp, dtype, red, beta, chunk=None, want=("dX", "dW", "dbias"), two
     adv = inp["adv"].float().to(dev)
     mask = inp["mask"].to(dev)
     loss = torch.full((1,), float("nan"), device=dev)
-    dX = torch.full((N, H), float("nan"), dtype=dtype, device=dev) if "dX" in want else None
-    dW = torch.full((V, H), float("nan"), dtype=dtype, device=dev) if "dW" in want else None
-    db = (torch.full((V,), float("nan"), dtype=dtype, device=dev)
-          if ("dbias" in want and b is not None) else None)
+    bufs = []
+
+    def out(shape):
+        # a NaN-filled view `out_offset` elements into a buffer 8 elements longer
+        n = int(np.prod(shape))
+        buf = torch.full((n + out_offset + 8,), float("nan"), dtype=dtype, device=dev)
+        bufs.append((buf, n))
+        return buf[out_offset:out_offset + n].view(shape)
+
+    dX = out((N, H)) if "dX" in want else None
+    dW = out((V, H)) if "dW" in want else None
+    db = out((V,)) if ("dbias" in want and b is not None) else None
     lp = torch.full((N,), float("nan"), device=dev)
     rlp = torch.full((N,), float("nan"), device=dev)
     nv = torch.full((1,), -1, dtype=torch.int64, device=dev)
@@ -71,11 +79,13 @@ def run_fused(inp, dtype, red, beta, chunk=None, want=("dX", "dW", "dbias"), two
     m.check(rc, "pl_fused_linear_grpo")
     torch.cuda.synchronize()
     status = m.pl_device_status(ws)
-    out = {"loss": loss.item(), "logp": lp.cpu().double().numpy(), "ref_logp": rlp.cpu().double().numpy(),
+    res = {"loss": loss.item(), "logp": lp.cpu().double().numpy(), "ref_logp": rlp.cpu().double().numpy(),
            "n_valid": int(nv.item()), "status": status}
+    for buf, n in bufs:   # nothing written outside the outputs
+        assert torch.isnan(buf[:out_offset]).all() and torch.isnan(buf[out_offset + n:]).all()
     for k, t in (("dX", dX), ("dW", dW), ("dbias", db)):
-        out[k] = None if t is None else t.cpu().double().numpy()
-    return out
+        res[k] = None if t is None else t.cpu().double().numpy()
+    return res
 
 
 def rel_fro(a, b):
@@ -169,6 +179,17 @@ def test_large_chunk_small_model(chunk):
     inp = build_inputs(36, 128, 64, 512, torch.float16, 77 + chunk, bias=True, len_lo=0, len_hi=128)
     got = run_fused(inp, torch.float16, 1, 0.04, chunk=chunk)
     check(inp, got, 1, 0.04)
+
+
+@pytest.mark.parametrize("offset", [0, 1, 4], ids=["aligned", "odd", "8byte"])
+@pytest.mark.parametrize("chunk", [None, 256], ids=["one_chunk", "chunks256"])
+def test_gradient_output_alignment(offset, chunk):
+    # dX, dW and dbias views 0, 2 or 8 bytes into their buffers: 16-byte aligned
+    # outputs take the TMA stores, the others per-thread stores; nothing is
+    # written before or after an output
+    inp = build_inputs(2, 300, 136, 1000, torch.bfloat16, 4242 + offset, bias=True, len_lo=0, len_hi=300)
+    got = run_fused(inp, torch.bfloat16, 0, 0.04, chunk=chunk, out_offset=offset)
+    check(inp, got, 0, 0.04)
 
 
 @pytest.mark.parametrize("tau", [0.7, 1.5])

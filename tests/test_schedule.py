@@ -43,3 +43,24 @@ def test_backward_schedule_is_balanced():
     for t in range(t0 + t1):
         rr[t % pairs] += c0 if t < t0 else c1
     assert max(per) < max(rr)
+
+
+@pytest.mark.parametrize("name,problems,want", [
+    ("forward, 1024 rows", [(1024, 128256, 4096)] * 2, 2),
+    ("backward, 1024-row chunk", [(1024, 4096, 128256), (128256, 4096, 1024)], 2),
+    ("backward, whole 8192-row batch", [(8192, 4096, 128256), (128256, 4096, 8192)], 2),
+    ("backward, 1024-row chunk, V=152064, H=4000", [(1024, 4000, 152064), (152064, 4000, 1024)], 2),
+    ("backward, 256-row chunk: 8 wide dX tiles would hold up the launch", [(256, 4096, 128256), (128256, 4096, 256)], 1),
+    ("dX alone: 32 wide tiles on 74 pairs", [(1024, 4096, 128256)], 1),
+    ("problem narrower than 512", [(1024, 256, 4096)], 1),
+    ("one of two problems narrower than 512", [(1024, 4096, 64), (4096, 448, 1024)], 1),
+])
+def test_tile_width_choice(name, problems, want):
+    assert pl.pl_debug_pick_tile(problems, 74) == want, name
+
+
+def test_pick_tile_rejects_bad_input():
+    assert pl.pl_debug_pick_tile([], 74) == -1
+    assert pl.pl_debug_pick_tile([(1, 1, 1)] * 3, 74) == -1
+    assert pl.pl_debug_pick_tile([(0, 512, 64)], 74) == -1
+    assert pl.pl_debug_pick_tile([(256, 512, 64)], 0) == -1
