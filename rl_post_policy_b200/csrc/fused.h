@@ -1,6 +1,7 @@
 // Workspace layout and kernel arguments of the fused linear path.
 #pragma once
 
+#include <cuda.h>
 #include <cstdint>
 
 #include "internal.h"
@@ -56,9 +57,14 @@ struct CombineArgs {
 };
 
 // The dlogits pass splits a chunk's rows into at most this many groups.
-constexpr int kDlMaxRowGroups = 16;
+constexpr int kDlMaxRowGroups = 4;
+
+// dlogits tiles: 32 rows x 256 columns of 16-bit logits.
+constexpr int kDlTileRows = 32;
+constexpr uint32_t kDlTileBytes = kDlTileRows * 256 * 2;
 
 struct DlogitsArgs {
+  CUtensorMap tmap;   // the chunk's logits, set by launch_dlogits
   unsigned char* ws;
   FusedOffsets off;
   const int64_t* targets;
@@ -73,6 +79,7 @@ struct DlogitsArgs {
   unsigned* db_cnt;
   int64_t rg_rows;    // set by launch_dlogits
   int n_rg;
+  unsigned long long wait_ns;  // bound of each wait for a tile (set by launch_dlogits)
 };
 
 cudaError_t launch_count(const uint8_t* mask, int64_t bs, int64_t T, unsigned char* ws, int nchunks,

@@ -18,7 +18,9 @@
 #include <cuda_fp16.h>
 
 #include "fused.h"
+#include "gemm.h"
 #include "policy_math.cuh"
+#include "sm100.cuh"
 
 namespace pl {
 namespace {
@@ -30,6 +32,16 @@ template <> __device__ __forceinline__ __nv_bfloat16 to_t<__nv_bfloat16>(float x
   return __float2bfloat16_rn(x);
 }
 template <> __device__ __forceinline__ __half to_t<__half>(float x) { return __float2half_rn(x); }
+template <typename T> __device__ __forceinline__ float2 unpack2(uint32_t u);
+template <> __device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t u) {
+  // a bf16 is the high half of the fp32 with the same value
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+template <> __device__ __forceinline__ float2 unpack2<__half>(uint32_t u) {
+  __half2 h;
+  *reinterpret_cast<uint32_t*>(&h) = u;
+  return __half22float2(h);
+}
 template <typename T> __device__ __forceinline__ uint32_t pack_t(float a, float b);
 template <> __device__ __forceinline__ uint32_t pack_t<__nv_bfloat16>(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -210,30 +222,26 @@ __global__ void clear_gmax_kernel(unsigned char* ws, int nchunks, FusedOffsets o
 
 // ---------------------------------------------------------------- dlogits
 // Block = 256 threads = 8 warps over one 256-column strip (blockIdx.x) and one
-// group of rows (blockIdx.y); lane l owns columns [8l, 8l+8) of the strip, warp
-// w rows w, w+8, ... of the group, kDlRows rows loaded before any is stored so
-// that each thread keeps kDlRows 16-byte loads in flight.  Many row groups per
-// strip fill the GPU several times over.  The bias gradient: each block writes
-// its strip's column sums for its row group; the strip's last block to finish
-// adds the row groups in order (deterministic) and stores / accumulates them.
-constexpr int kDlRows = 4;
-
-// 8 consecutive elements as raw 16 bytes (zeros past V on the ragged strip).
-template <typename T>
-__device__ __forceinline__ uint4 load8(const T* p, bool full8, int64_t col, int64_t V) {
-  if (full8) return *reinterpret_cast<const uint4*>(p);
-  uint4 u = make_uint4(0, 0, 0, 0);
-  T* e8 = reinterpret_cast<T*>(&u);
-#pragma unroll
-  for (int q = 0; q < 8; ++q)
-    if (col + q < V) e8[q] = p[q];
-  return u;
-}
+// group of rows (blockIdx.y).  The group's rows stream through shared memory in
+// tiles of 32 rows x 256 columns (16 KB of 16-bit logits): one thread issues the
+// TMA loads of a kDlStages-deep ring up front, every thread turns its part of a
+// landed tile into dz in place (lane l: columns [8l, 8l+8); warp w: rows w,
+// w+8, w+16, w+24), and the tile goes back to the same global rows by TMA
+// store, after which its slot takes the tile kDlStages further on.  The copies
+// need no registers, so a block keeps up to 64 KB of loads in flight.  Rows
+// past the chunk and columns past V are zero-filled on load and dropped on
+// store.  The bias gradient: each block writes its strip's column sums for its
+// row group; the strip's last block to finish adds the row groups in order
+// (deterministic) and stores / accumulates them.
+constexpr int kDlStages = 4;
 
 template <typename T>
-__global__ void __launch_bounds__(256, 3) dlogits_kernel(DlogitsArgs a) {
+__global__ void __launch_bounds__(256, 3) dlogits_kernel(const __grid_constant__ DlogitsArgs a) {
+  extern __shared__ __align__(128) uint8_t dl_ring[];  // kDlStages tiles of kDlTileBytes
+  __shared__ uint64_t full[kDlStages];
   __shared__ float s_col[8][256];
   __shared__ int s_last;
+  __shared__ int s_abort;
   const unsigned char* ws = a.ws;
   const float* row_lse = reinterpret_cast<const float*>(ws + a.off.lse);
   const float* row_g = reinterpret_cast<const float*>(ws + a.off.g);
@@ -250,61 +258,133 @@ __global__ void __launch_bounds__(256, 3) dlogits_kernel(DlogitsArgs a) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t col = (int64_t)blockIdx.x * 256 + lane * 8;
-  const bool full8 = col + 8 <= a.V;
+  const int32_t x0 = (int32_t)(blockIdx.x * 256);
   const int64_t r_begin = (int64_t)blockIdx.y * a.rg_rows;
   const int64_t r_end = min(a.rows, r_begin + a.rg_rows);
-  float csum[8];
+  const int ntiles = (int)((r_end - r_begin + kDlTileRows - 1) / kDlTileRows);
+  const uint32_t ring = sm100::smem_u32(dl_ring);
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kDlStages; ++st) sm100::mbar_init(&full[st], 1);
+    s_abort = 0;
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  int issued = 0;  // tiles whose load thread 0 has issued
+  if (threadIdx.x == 0) {
+    for (; issued < ntiles && issued < kDlStages; ++issued) {
+      sm100::mbar_arrive_expect_tx(&full[issued], kDlTileBytes);
+      sm100::tma_load_2d(dl_ring + issued * kDlTileBytes, &a.tmap, &full[issued], x0,
+                         (int32_t)(r_begin + (int64_t)issued * kDlTileRows));
+    }
+  }
+  float2 csum2[4];  // column sums of dz * 2^e (scaled back, exactly, at the end)
 #pragma unroll
-  for (int q = 0; q < 8; ++q) csum[q] = 0.0f;
-  T* L = reinterpret_cast<T*>(a.logits);
+  for (int h = 0; h < 4; ++h) csum2[h] = make_float2(0.0f, 0.0f);
   constexpr float kLog2e = 1.4426950408889634f;
-  if (col < a.V) {
-    for (int64_t i0 = r_begin + warp; i0 < r_end; i0 += 8 * kDlRows) {
-      uint4 raw[kDlRows];
-      float gi[kDlRows], lsei[kDlRows];
-      int ti[kDlRows];
+  // Per-row inputs of a tile (g, lse, target), loaded one tile ahead so that
+  // their latency hides behind the previous tile's work.
+  float gi[4], lsei[4];
+  int ti[4];
+  auto row_inputs = [&](int kt, float (&g4)[4], float (&l4)[4], int (&t4)[4]) {
 #pragma unroll
-      for (int u = 0; u < kDlRows; ++u) {
-        const int64_t i = i0 + 8 * u;
-        if (i < r_end) {
-          raw[u] = load8<T>(L + i * a.ld + col, full8, col, a.V);
-          gi[u] = __ldg(row_g + i);
-          lsei[u] = __ldg(row_lse + i) * kLog2e;
-          const int64_t tg = __ldg(a.targets + a.row0 + i);
-          ti[u] = (tg >= 0 && tg < a.V) ? (int)tg : -1;
-        }
+    for (int j = 0; j < 4; ++j) {
+      const int64_t i = r_begin + (int64_t)kt * kDlTileRows + warp + 8 * j;
+      g4[j] = 0.0f; l4[j] = 0.0f; t4[j] = -1;
+      if (i < r_end) {
+        g4[j] = __ldg(row_g + i);
+        l4[j] = __ldg(row_lse + i) * kLog2e;
+        const int64_t tg = __ldg(a.targets + a.row0 + i);
+        t4[j] = (tg >= 0 && tg < a.V) ? (int)tg : -1;
       }
+    }
+  };
+  if (ntiles > 0) row_inputs(0, gi, lsei, ti);
+  int k = 0;
+  for (; k < ntiles; ++k) {
+    const int slot = k % kDlStages;
+    bool rv[4];
 #pragma unroll
-      for (int u = 0; u < kDlRows; ++u) {
-        const int64_t i = i0 + 8 * u;
-        if (i >= r_end) break;
-        const T* z = reinterpret_cast<const T*>(&raw[u]);
-        float d[8];
+    for (int j = 0; j < 4; ++j) rv[j] = r_begin + (int64_t)k * kDlTileRows + warp + 8 * j < r_end;
+    float gn[4], ln[4];
+    int tn[4];
+    if (k + 1 < ntiles) row_inputs(k + 1, gn, ln, tn);
+    if (sm100::mbar_wait(&full[slot], (uint32_t)(k / kDlStages) & 1u, &s_abort, a.wait_ns)) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float pr = exp2f(fmaf(cvt(z[q]), kLog2e, -lsei[u]));
-          const float oh = (col + q == ti[u]) ? 1.0f : 0.0f;
-          d[q] = gi[u] * (oh - pr);
-          csum[q] += d[q];
+      for (int j = 0; j < 4; ++j) {
+        if (!rv[j]) continue;
+        uint4* p = reinterpret_cast<uint4*>(dl_ring + slot * kDlTileBytes + (warp + 8 * j) * 512 + lane * 16);
+        const uint4 raw = *p;
+        // dz * 2^e = -(g * 2^e) * p_v, plus g * 2^e at the target column; two
+        // columns per packed fp32 instruction
+        const float gs = gi[j] * sc;
+        const float2 nl2 = make_float2(-lsei[j], -lsei[j]);
+        const float2 ngs2 = make_float2(-gs, -gs);
+        const float2 l2e2 = make_float2(kLog2e, kLog2e);
+        const uint32_t r32[4] = {raw.x, raw.y, raw.z, raw.w};
+        float2 ds[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float2 x = __ffma2_rn(unpack2<T>(r32[h]), l2e2, nl2);
+          ds[h] = __fmul2_rn(make_float2(ex2_approx(x.x), ex2_approx(x.y)), ngs2);
         }
-        T* p = L + i * a.ld + col;
-        if (full8) {
-          uint4 w;
-          T* e8 = reinterpret_cast<T*>(&w);
+        const int rel = ti[j] - (int)col;  // the target's column within this thread's 8, if any
+        if ((unsigned)rel < 8u) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) e8[q] = to_t<T>(d[q] * sc);
-          *reinterpret_cast<uint4*>(p) = w;
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (col + q < a.V) p[q] = to_t<T>(d[q] * sc);
+          for (int h = 0; h < 4; ++h) {
+            if (rel == 2 * h) ds[h].x += gs;
+            if (rel == 2 * h + 1) ds[h].y += gs;
+          }
         }
+        uint4 w;
+        uint32_t* w32 = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          csum2[h] = __fadd2_rn(csum2[h], ds[h]);
+          w32[h] = pack_t<T>(ds[h].x, ds[h].y);
+        }
+        *p = w;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      gi[j] = gn[j];
+      lsei[j] = ln[j];
+      ti[j] = tn[j];
+    }
+    sm100::fence_proxy_async_smem();  // the tile's generic writes before the TMA store reads them
+    __syncthreads();
+    if (s_abort) break;
+    if (threadIdx.x == 0) {
+      sm100::tma_store_2d(&a.tmap, ring + slot * kDlTileBytes, x0, (int32_t)(r_begin + (int64_t)k * kDlTileRows));
+      sm100::bulk_commit_group();
+      if (issued < ntiles) {
+        // the slot is refilled once the store has read it out
+        sm100::bulk_wait_group_read<0>();
+        sm100::mbar_arrive_expect_tx(&full[slot], kDlTileBytes);
+        sm100::tma_load_2d(dl_ring + slot * kDlTileBytes, &a.tmap, &full[slot], x0,
+                           (int32_t)(r_begin + (int64_t)issued * kDlTileRows));
+        ++issued;
       }
     }
   }
+  if (threadIdx.x == 0) {
+    sm100::bulk_wait_group_all();
+    if (s_abort) {
+      // let the loads already issued land (bounded) before the block's shared memory goes away
+      volatile int no_abort = 0;
+      for (int t = k; t < issued; ++t)
+        sm100::mbar_wait(&full[t % kDlStages], (uint32_t)(t / kDlStages) & 1u, &no_abort, a.wait_ns);
+      atomicOr(reinterpret_cast<unsigned*>(a.ws), kDevErrTimeout);
+    }
+  }
+  if (s_abort) return;
   if (a.dbias_mode == kAccNone) return;
+  const float inv_sc = ldexpf(1.0f, -e);
 #pragma unroll
-  for (int q = 0; q < 8; ++q) s_col[warp][lane * 8 + q] = csum[q];
+  for (int h = 0; h < 4; ++h) {
+    s_col[warp][lane * 8 + 2 * h] = csum2[h].x * inv_sc;
+    s_col[warp][lane * 8 + 2 * h + 1] = csum2[h].y * inv_sc;
+  }
   __syncthreads();
   const int64_t v = (int64_t)blockIdx.x * 256 + threadIdx.x;
   float s = 0.0f;
@@ -388,16 +468,31 @@ cudaError_t launch_clear_gmax(unsigned char* ws, int nchunks, const FusedOffsets
 cudaError_t launch_dlogits(const DlogitsArgs& a0, DType dt, cudaStream_t s) {
   if (a0.rows <= 0) return cudaSuccess;
   DlogitsArgs a = a0;
-  // row groups of >= 128 rows (a multiple of the 32 rows one pass covers), at most kDlMaxRowGroups
+  // row groups of >= 128 rows (whole 32-row tiles), at most kDlMaxRowGroups
   int64_t rg = (a.rows + kDlMaxRowGroups - 1) / kDlMaxRowGroups;
-  rg = rg < 128 ? 128 : (rg + 31) / 32 * 32;
+  rg = rg < 128 ? 128 : (rg + kDlTileRows - 1) / kDlTileRows * kDlTileRows;
   a.rg_rows = rg;
   a.n_rg = (int)((a.rows + rg - 1) / rg);
+  a.wait_ns = debug_knobs().wait_ns;
+  // the chunk's [rows, V] logits, {256, 32} boxes, rows ld elements apart
+  if (!make_tmap_2d(&a.tmap, a.logits, dt, (uint64_t)a.V, (uint64_t)a.rows, (uint64_t)a.ld * 2, 256,
+                    kDlTileRows, false))
+    return cudaErrorInvalidValue;
   const dim3 grid((unsigned)((a.V + 255) / 256), (unsigned)a.n_rg);
+  const size_t smem = (size_t)kDlStages * kDlTileBytes;
+  static bool attr_set[2] = {false, false};
+  const int ti = dt == DType::BF16 ? 0 : 1;
+  if (!attr_set[ti]) {
+    const cudaError_t e = dt == DType::BF16
+        ? cudaFuncSetAttribute(dlogits_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+        : cudaFuncSetAttribute(dlogits_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set[ti] = true;
+  }
   if (dt == DType::BF16) {
-    { launch_begin(2, s); dlogits_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
+    { launch_begin(2, s); dlogits_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(a); launch_end(2, s); }
   } else {
-    { launch_begin(2, s); dlogits_kernel<__half><<<grid, 256, 0, s>>>(a); launch_end(2, s); }
+    { launch_begin(2, s); dlogits_kernel<__half><<<grid, 256, smem, s>>>(a); launch_end(2, s); }
   }
   return cudaGetLastError();
 }

@@ -89,10 +89,11 @@ struct __align__(64) GemmParams {
 // boxes; MN-major operands load {64, kBK} boxes, two per 128 rows/columns.
 // Encodes a 2-D tensor map over a row-major [outer, inner] array of `dt`
 // elements (16-bit, or fp32 for the kOutTma* outputs) with a row pitch of
-// `pitch_bytes`, box {box_inner, box_outer}, 128-byte swizzle, zero fill
-// outside the extent.
+// `pitch_bytes`, box {box_inner, box_outer}, zero fill outside the extent, and
+// the 128-byte swizzle (box rows of at most 128 bytes) or none (box rows of
+// up to 256 elements, laid out densely in shared memory).
 bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, uint64_t outer,
-                  uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
+                  uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128 = true);
 
 // Fills tiles_m/tiles_n/k_steps/tile_begin of each job and total_tiles, for
 // tiles nh * kBN wide.  launch_gemm picks nh and calls it again.

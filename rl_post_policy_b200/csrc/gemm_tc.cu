@@ -784,7 +784,7 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, uint64_t outer,
-                  uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+                  uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   if ((reinterpret_cast<uintptr_t>(base) & 15) || (pitch_bytes & 15)) return false;
@@ -796,7 +796,8 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, 
                                 : dt == DType::F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   CUresult r = fn(map, t, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
