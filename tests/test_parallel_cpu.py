@@ -96,3 +96,62 @@ def test_dp_step_matches_whole_batch_oracle(red):
         out, err = p.communicate(timeout=180)
         assert p.returncode == 0, err[-3000:]
         assert "RANK_OK" in out
+
+
+LOSS_SCRIPT = textwrap.dedent("""
+    import os, sys
+    sys.path.insert(0, {root!r})
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import oracle, synth
+    from rl_post_policy_b200 import parallel
+
+    rank, ws = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    red, two_sided = {red}, {two_sided}
+    bs, seq = 7, 40
+    inp = synth.loss_inputs(bs, seq, torch.float32, 99, len_lo=1, len_hi=seq)
+    inp["mask"][5] = 0                                  # a fully masked sequence
+    kw = dict(eps_lo=0.2, eps_hi=0.28, beta=0.04, reduction=red, two_sided=two_sided)
+    want = oracle.policy_loss(inp["policy_lp"], inp["old_lp"], inp["ref_lp"], inp["adv"], inp["mask"], **kw)
+    seqs = [[0, 1, 2], [3, 4, 5, 6]][rank]              # unequal shards; rank 1 holds the empty sequence
+
+    class OracleOps:
+        def local_loss(self, lp, old, ref, adv, mask, eps_lo, eps_hi, beta, reduction, two_sided=False,
+                       want_grad=True):
+            o = oracle.policy_loss(lp, old, ref, adv, mask, eps_lo=eps_lo, eps_hi=eps_hi, beta=beta,
+                                   reduction=reduction, two_sided=two_sided)
+            return {{"loss": torch.tensor([o["loss"]], dtype=torch.float64),
+                    "grad": torch.from_numpy(o["grad"]).double(),
+                    "n_valid": torch.tensor([o["n_valid"]], dtype=torch.int64)}}
+        def ratio(self, local, total):
+            return local.clamp(min=1).double() / total.clamp(min=1).double()
+        def scale(self, t, f):
+            t.mul_(f)
+
+    got = parallel.dp_policy_loss(inp["policy_lp"][seqs], inp["old_lp"][seqs], inp["ref_lp"][seqs],
+                                  inp["adv"][seqs], inp["mask"][seqs], ops=OracleOps(), **kw)
+    assert abs(got["loss"].item() - want["loss"]) <= 1e-12 * max(1.0, abs(want["loss"])), (got["loss"], want["loss"])
+    err = np.abs(got["grad"].numpy() - want["grad"][seqs]).max()
+    assert err <= 1e-15, err
+    assert int(got["count"].item()) == (want["n_valid"] if red == 0 else bs)
+    print("RANK_OK", rank, flush=True)
+    dist.destroy_process_group()
+""")
+
+
+@pytest.mark.parametrize("red,two_sided", [(0, False), (1, False), (1, True)], ids=["bnpo", "grpo", "grpo_two_sided"])
+def test_dp_loss_step_matches_whole_batch_oracle(red, two_sided):
+    script = LOSS_SCRIPT.format(root=ROOT, red=red, two_sided=two_sided)
+    port = _free_port()
+    procs = []
+    for r in range(2):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE="2", MASTER_ADDR="127.0.0.1",
+                   MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="")
+        procs.append(subprocess.Popen([sys.executable, "-c", script], env=env, stdout=subprocess.PIPE,
+                                      stderr=subprocess.PIPE, text=True))
+    for p in procs:
+        out, err = p.communicate(timeout=180)
+        assert p.returncode == 0, err[-3000:]
+        assert "RANK_OK" in out

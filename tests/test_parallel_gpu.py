@@ -51,6 +51,33 @@ def test_one_rank_equals_single_gpu_call(group, red):
     assert int(out["count"].item()) == (int(ref["n_valid"].item()) if red == pl.PL_BNPO else bs)
 
 
+@pytest.mark.parametrize("red", [0, 1], ids=["bnpo", "grpo"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+def test_one_rank_loss_step_equals_oracle(group, red, dtype):
+    # dp_policy_loss on one rank: the share is exactly 1, so loss and gradient
+    # are the loss kernel's own, and they match the oracle
+    import numpy as np
+    import oracle
+    from rl_post_policy_b200 import parallel
+    bs, seq = 6, 700
+    inp = synth.loss_inputs(bs, seq, dtype, 6061, len_lo=1, len_hi=seq)
+    g = {k: v.cuda() for k, v in inp.items()}
+    out = parallel.dp_policy_loss(g["policy_lp"], g["old_lp"], g["ref_lp"], g["adv"], g["mask"], eps_lo=0.2,
+                                  eps_hi=0.28, beta=0.04, reduction=red, group=group)
+    torch.cuda.synchronize()
+    want = oracle.policy_loss(inp["policy_lp"], inp["old_lp"], inp["ref_lp"], inp["adv"], inp["mask"],
+                              eps_lo=0.2, eps_hi=0.28, beta=0.04, reduction=red)
+    tol = 1e-5 if dtype == torch.float32 else 1e-3
+    assert abs(out["loss"].item() - want["loss"]) <= tol * max(abs(want["loss"]), 1e-3 * want["abs_sum"])
+    w = torch.from_numpy(want["grad"]).to(dtype).double().numpy()
+    err = np.abs(out["grad"].double().cpu().numpy() - w)
+    # fp32: the loss kernel's 1e-6; bf16: two units in the last place of the rounded oracle.
+    # At most one token within rounding of a clip bound may take the other side of the min.
+    bound = 1e-6 if dtype == torch.float32 else 2.0 ** -7 * np.abs(w) + 1e-9
+    assert np.count_nonzero(err > bound) <= 1, float(err.max())
+    assert int(out["count"].item()) == (want["n_valid"] if red == 0 else bs)
+
+
 def test_count_ratio_and_scale():
     import rl_post_policy_b200 as pl
     from rl_post_policy_b200 import parallel
