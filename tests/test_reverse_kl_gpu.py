@@ -90,6 +90,31 @@ def test_every_cluster_split(cl):
     check(got, want, inp["mask"], torch.bfloat16, 40, 5000)
 
 
+@pytest.mark.parametrize("cl", [1, 8])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+def test_many_rows_per_cluster_with_masked_runs(cl, dtype):
+    # Several rows per cluster, so a row's gradient pass runs inside the next
+    # valid row's statistics pass: masked rows first, in runs between valid
+    # rows, and last; one valid row alone at the end of a cluster's rows.
+    m = pl()
+    bs, seq, V = 3, 400, 2048
+    inp = synth.reverse_kl_inputs(bs, seq, V, dtype, synth.seed_for(47, cl))
+    mask = inp["mask"].reshape(-1).clone()
+    mask[:5] = 0
+    mask[100:160] = 0
+    mask[300:302] = 0
+    mask[-7:] = 0
+    mask[-9] = 1
+    mask = mask.reshape(bs, seq)
+    want = oracle.reverse_kl(inp["student"], inp["teacher"], mask)
+    assert m.pl_debug_set_rkl_cluster(cl) == 0
+    try:
+        got = run(inp["student"], inp["teacher"], mask)
+    finally:
+        m.pl_debug_set_rkl_cluster(0)
+    check(got, want, mask, dtype, bs * seq, V)
+
+
 def test_close_teacher_small_kl():
     # teacher = student + N(0, 0.05): kl ~ 1e-3, the cancellation-prone regime
     inp = synth.reverse_kl_inputs(4, 16, 32000, torch.bfloat16, synth.seed_for(42), teacher_std=0.05)
