@@ -177,6 +177,12 @@ pl_status run_pipeline(const Pipe& q) {
       j.zt = reinterpret_cast<float*>(ws + plan.off.zt);
       j.logits = need_bwd ? ws + plan.off.logits : nullptr; j.logits_ld = plan.ld;
       j.logit_scale = q.inv_temp;
+      if (j.logits) {
+        // the chunk's [rows, V] logits, written by TMA stores from the epilogue
+        if (!make_tmap_2d(&fp.maps[4], ws + plan.off.logits, dt, V, rows, plan.ld * esz, kOutBoxN16, kOutBoxM))
+          return PL_ERR_CUDA;
+        j.out_path = kOutTmaStore; j.out_map = 4;
+      }
     }
     fp.njobs = nj;
     gemm_finalize_jobs(&fp);

@@ -469,59 +469,90 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         } else if (j.epi == kEpiLse) {
           const T* bias = reinterpret_cast<const T*>(j.bias);
           T* logits = reinterpret_cast<T*>(j.logits);
+          // logits through shared memory and TMA stores (see the kEpiStore
+          // path below), 64 columns per box, or per-thread stores
+          const bool tma_logits = logits && j.out_path == kOutTmaStore;
+          const int y = m0 + quarter * 32;
           const int64_t tgt_rel = tgt >= 0 ? tgt - (int64_t)n0 : (int64_t)-1;
           float m_run = -INFINITY, s_run = 0.0f, ztv = 0.0f;
           bool got = false;
   #pragma unroll 1
-          for (int c = 0; c < kBN / 32; ++c) {
-            float v[32];
-            tmem_ld_32x32b_x32(taddr + c * 32, v);
-            const int col0 = n0 + c * 32;
-            const int nvalid = min(32, j.N - col0);
-            if (nvalid <= 0) continue;
-            if (bias) add_bias32<T>(bias + col0, v, nvalid);
-            if (j.logit_scale != 1.0f) {
+          for (int c = 0; c < kBN / 32; c += 2) {
+            uint32_t w[32];
   #pragma unroll
-              for (int q = 0; q < 32; ++q) v[q] *= j.logit_scale;
-            }
-            if (nvalid == 32) {
-              // full chunk: no per-column predicates; two columns per packed instruction
-              float cmax = v[0];
+            for (int h = 0; h < 2; ++h) {
+              float v[32];
+              tmem_ld_32x32b_x32(taddr + (c + h) * 32, v);
+              const int col0 = n0 + (c + h) * 32;
+              const int nvalid = min(32, j.N - col0);
+              if (nvalid > 0) {
+                if (bias) add_bias32<T>(bias + col0, v, nvalid);
+                if (j.logit_scale != 1.0f) {
   #pragma unroll
-              for (int q = 1; q < 32; ++q) cmax = fmaxf(cmax, v[q]);
-              const float m_new = fmaxf(m_run, cmax);
-              const float2 nmb = make_float2(-m_new * kLog2e, -m_new * kLog2e);
-              const float2 l2e = make_float2(kLog2e, kLog2e);
-              float2 s2 = make_float2(0.0f, 0.0f);
+                  for (int q = 0; q < 32; ++q) v[q] *= j.logit_scale;
+                }
+                if (nvalid == 32) {
+                  // full chunk: no per-column predicates; two columns per packed instruction
+                  float cmax = v[0];
   #pragma unroll
-              for (int q = 0; q < 32; q += 2) {
-                const float2 x = __ffma2_rn(make_float2(v[q], v[q + 1]), l2e, nmb);
-                s2 = __fadd2_rn(s2, make_float2(ex2_approx(x.x), ex2_approx(x.y)));
+                  for (int q = 1; q < 32; ++q) cmax = fmaxf(cmax, v[q]);
+                  const float m_new = fmaxf(m_run, cmax);
+                  const float2 nmb = make_float2(-m_new * kLog2e, -m_new * kLog2e);
+                  const float2 l2e = make_float2(kLog2e, kLog2e);
+                  float2 s2 = make_float2(0.0f, 0.0f);
+  #pragma unroll
+                  for (int q = 0; q < 32; q += 2) {
+                    const float2 x = __ffma2_rn(make_float2(v[q], v[q + 1]), l2e, nmb);
+                    s2 = __fadd2_rn(s2, make_float2(ex2_approx(x.x), ex2_approx(x.y)));
+                  }
+                  s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, nmb.x)) + (s2.x + s2.y);
+                  m_run = m_new;
+                } else {
+                  float cmax = -INFINITY;
+  #pragma unroll
+                  for (int q = 0; q < 32; ++q)
+                    if (q < nvalid) cmax = fmaxf(cmax, v[q]);
+                  const float m_new = fmaxf(m_run, cmax);
+                  const float mb = m_new * kLog2e;
+                  float s = 0.0f;
+  #pragma unroll
+                  for (int q = 0; q < 32; ++q)
+                    if (q < nvalid) s += ex2_approx(fmaf(v[q], kLog2e, -mb));
+                  s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, -mb)) + s;
+                  m_run = m_new;
+                }
+                const int64_t rel = tgt_rel - (c + h) * 32;
+                if (rel >= 0 && rel < 32) {
+  #pragma unroll
+                  for (int q = 0; q < 32; ++q)
+                    if (q == (int)rel) ztv = v[q];
+                  got = true;
+                }
+                if (logits && !tma_logits && row_ok)
+                  store_row32<T>(logits + (int64_t)row * j.logits_ld + col0, v, nvalid);
               }
-              s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, nmb.x)) + (s2.x + s2.y);
-              m_run = m_new;
-            } else {
-              float cmax = -INFINITY;
+              if (tma_logits) {
   #pragma unroll
-              for (int q = 0; q < 32; ++q)
-                if (q < nvalid) cmax = fmaxf(cmax, v[q]);
-              const float m_new = fmaxf(m_run, cmax);
-              const float mb = m_new * kLog2e;
-              float s = 0.0f;
-  #pragma unroll
-              for (int q = 0; q < 32; ++q)
-                if (q < nvalid) s += ex2_approx(fmaf(v[q], kLog2e, -mb));
-              s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, -mb)) + s;
-              m_run = m_new;
+                for (int q = 0; q < 16; ++q) w[16 * h + q] = pack2<T>(v[2 * q], v[2 * q + 1]);
+              }
             }
-            const int64_t rel = tgt_rel - c * 32;
-            if (rel >= 0 && rel < 32) {
+            if (tma_logits && n0 + c * 32 < j.N && y < j.M) {
+              if (lane == 0) bulk_wait_group_read<1>();
+              __syncwarp();
+              const uint32_t box = stage0 + (uint32_t)sbuf * kOutBoxBytes;
+              const uint32_t my_row = box + (uint32_t)lane * 128u;
   #pragma unroll
-              for (int q = 0; q < 32; ++q)
-                if (q == (int)rel) ztv = v[q];
-              got = true;
+              for (int q = 0; q < 8; ++q)
+                st_shared_v4(my_row + ((uint32_t)(q ^ (lane & 7)) << 4), w[4 * q], w[4 * q + 1], w[4 * q + 2],
+                             w[4 * q + 3]);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&p.maps[j.out_map], box, n0 + c * 32, y);
+                bulk_commit_group();
+              }
+              sbuf ^= 1;
             }
-            if (logits && row_ok) store_row32<T>(logits + (int64_t)row * j.logits_ld + col0, v, nvalid);
           }
           if (row_ok) {
             j.part[(int64_t)row * j.part_ld + grp] = make_float2(m_run, s_run);
