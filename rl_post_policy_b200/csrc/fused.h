@@ -48,7 +48,7 @@ struct CombineArgs {
   float* logp_out;
   float* ref_logp_out;
   int64_t row0, rows, bs, T, V;
-  int ntv;            // vocabulary tiles (partials per row)
+  int nparts;         // (max, sum exp) partials per row
   int chunk, part_stride;
   float lo, hi, beta;
   int grpo, adv_lp_dtype, bf16;

@@ -27,7 +27,7 @@ int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
   int64_t N = 0, C = 1024, Cbuf = 1, nchunks = 0, ld = 0;
-  int ntv = 0, part_stride = 1;
+  int ntv = 0, nparts = 0, part_stride = 1;  // 256-column vocabulary tiles; LSE partials per row
   FusedOffsets off{};
 };
 
@@ -42,6 +42,7 @@ Plan make_plan(int64_t bs, int64_t T, int64_t H, int64_t V, uint32_t mode, bool 
   p.Cbuf = p.N > 0 ? (p.N < p.C ? p.N : p.C) : 1;
   p.nchunks = p.N > 0 ? (p.N + p.C - 1) / p.C : 0;
   p.ntv = (int)((V + kBN - 1) / kBN);
+  p.nparts = p.ntv * kEpiColGroups;
   p.ld = align_up(V > 0 ? V : 1, 64);
   p.part_stride = (int)((p.Cbuf + 7) / 8);
   int64_t cur = (int64_t)kWsHeader;
@@ -60,8 +61,8 @@ Plan make_plan(int64_t bs, int64_t T, int64_t H, int64_t V, uint32_t mode, bool 
   p.off.g = region(4 * p.Cbuf);
   p.off.zt = region(4 * p.Cbuf);
   p.off.zt_ref = region(4 * p.Cbuf);
-  p.off.part = region(8 * p.Cbuf * (int64_t)p.ntv);
-  p.off.part_ref = region(8 * p.Cbuf * (int64_t)p.ntv);
+  p.off.part = region(8 * p.Cbuf * (int64_t)p.nparts);
+  p.off.part_ref = region(8 * p.Cbuf * (int64_t)p.nparts);
   p.off.logits = region(2 * p.Cbuf * p.ld);
   p.off.dw_acc = region((need_dW && p.nchunks > 1) ? 4 * V * H : 0);
   p.off.db_acc = region((need_dbias && p.nchunks > 1) ? 4 * V : 0);
@@ -161,7 +162,7 @@ pl_status run_pipeline(const Pipe& q) {
       j.a_map = 0; j.b_map = 1; j.a_mn = 0; j.b_mn = 0;
       j.M = (int)rows; j.N = (int)V; j.K = (int)H; j.n_inner = 0; j.epi = kEpiLse;
       j.bias = nullptr; j.targets = targets + r0;
-      j.part = reinterpret_cast<float2*>(ws + plan.off.part_ref); j.part_ld = plan.ntv;
+      j.part = reinterpret_cast<float2*>(ws + plan.off.part_ref); j.part_ld = plan.nparts;
       j.zt = reinterpret_cast<float*>(ws + plan.off.zt_ref); j.logits = nullptr;
       j.logit_scale = q.inv_temp;
     }
@@ -173,7 +174,7 @@ pl_status run_pipeline(const Pipe& q) {
       j.a_map = 2; j.b_map = 3; j.a_mn = 0; j.b_mn = 0;
       j.M = (int)rows; j.N = (int)V; j.K = (int)H; j.n_inner = 0; j.epi = kEpiLse;
       j.bias = bias; j.targets = targets + r0;
-      j.part = reinterpret_cast<float2*>(ws + plan.off.part); j.part_ld = plan.ntv;
+      j.part = reinterpret_cast<float2*>(ws + plan.off.part); j.part_ld = plan.nparts;
       j.zt = reinterpret_cast<float*>(ws + plan.off.zt);
       j.logits = need_bwd ? ws + plan.off.logits : nullptr; j.logits_ld = plan.ld;
       j.logit_scale = q.inv_temp;
@@ -192,7 +193,7 @@ pl_status run_pipeline(const Pipe& q) {
     CombineArgs ca{};
     ca.ws = ws; ca.off = plan.off; ca.targets = targets; ca.old_lp = old_lp; ca.adv = adv; ca.mask = mask;
     ca.logp_out = logp_out; ca.ref_logp_out = ref_logp_out;
-    ca.row0 = r0; ca.rows = rows; ca.bs = bs; ca.T = T; ca.V = V; ca.ntv = plan.ntv;
+    ca.row0 = r0; ca.rows = rows; ca.bs = bs; ca.T = T; ca.V = V; ca.nparts = plan.nparts;
     ca.chunk = (int)c; ca.part_stride = plan.part_stride;
     ca.lo = 1.0f - eps_lo; ca.hi = 1.0f + eps_hi; ca.beta = beta;
     ca.grpo = (mode & PL_REDUCTION_MASK) == PL_GRPO; ca.adv_lp_dtype = (mode & PL_ADV_LP_DTYPE) != 0;

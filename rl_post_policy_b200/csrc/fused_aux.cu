@@ -99,27 +99,27 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   if (i < a.rows) {
     const int64_t g = a.row0 + i;
     const unsigned char* ws = a.ws;
-    const float2* part = reinterpret_cast<const float2*>(ws + a.off.part) + i * a.ntv;
+    const float2* part = reinterpret_cast<const float2*>(ws + a.off.part) + i * a.nparts;
     const float* zt = reinterpret_cast<const float*>(ws + a.off.zt);
     // logsumexp over the vocabulary tiles: lse = M + log(sum_j s_j exp(m_j - M))
     float M = -INFINITY;
-    for (int j = lane; j < a.ntv; j += 32) M = fmaxf(M, part[j].x);
+    for (int j = lane; j < a.nparts; j += 32) M = fmaxf(M, part[j].x);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float S = 0.0f;
-    for (int j = lane; j < a.ntv; j += 32) S += part[j].y * expf(part[j].x - M);
+    for (int j = lane; j < a.nparts; j += 32) S += part[j].y * expf(part[j].x - M);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
     const float lse = M + logf(S);
     float ref_lp = 0.0f;
     if (HAS_KL) {
-      const float2* pr = reinterpret_cast<const float2*>(ws + a.off.part_ref) + i * a.ntv;
+      const float2* pr = reinterpret_cast<const float2*>(ws + a.off.part_ref) + i * a.nparts;
       float Mr = -INFINITY;
-      for (int j = lane; j < a.ntv; j += 32) Mr = fmaxf(Mr, pr[j].x);
+      for (int j = lane; j < a.nparts; j += 32) Mr = fmaxf(Mr, pr[j].x);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
       float Sr = 0.0f;
-      for (int j = lane; j < a.ntv; j += 32) Sr += pr[j].y * expf(pr[j].x - Mr);
+      for (int j = lane; j < a.nparts; j += 32) Sr += pr[j].y * expf(pr[j].x - Mr);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) Sr += __shfl_xor_sync(0xffffffffu, Sr, o);
       const float* ztr = reinterpret_cast<const float*>(ws + a.off.zt_ref);
@@ -184,13 +184,13 @@ __global__ void __launch_bounds__(256) combine_ext_kernel(CombineArgs a) {
   float gabs = 0.0f;
   if (i < a.rows) {
     const int64_t g = a.row0 + i;
-    const float2* part = reinterpret_cast<const float2*>(a.ws + a.off.part) + i * a.ntv;
+    const float2* part = reinterpret_cast<const float2*>(a.ws + a.off.part) + i * a.nparts;
     float M = -INFINITY;
-    for (int j = lane; j < a.ntv; j += 32) M = fmaxf(M, part[j].x);
+    for (int j = lane; j < a.nparts; j += 32) M = fmaxf(M, part[j].x);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float S = 0.0f;
-    for (int j = lane; j < a.ntv; j += 32) S += part[j].y * expf(part[j].x - M);
+    for (int j = lane; j < a.nparts; j += 32) S += part[j].y * expf(part[j].x - M);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
     if (lane == 0) {

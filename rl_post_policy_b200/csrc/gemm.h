@@ -17,7 +17,12 @@ constexpr int kPairM = 256;    // rows per CTA pair (the MMA's M)
 constexpr int kBN = 256;       // tile columns (tensor-memory columns per accumulator)
 constexpr int kBNh = 128;      // B rows (N) held by each CTA of the pair
 constexpr int kBK = 64;        // K per pipeline stage (one 128-byte swizzle row)
-constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+// Warp 0: TMA producer; warp 1: MMA issuer; then EW epilogue warps, EW = 8
+// (two per 32-lane quarter of tensor memory, splitting each 256-column group in
+// column halves) or 4 (one per quarter, two staging boxes each: launches with an
+// fp32 TMA output, whose 32-column boxes are too small to leave one box per warp).
+constexpr int kEpiColGroups = 2;   // LSE partials per row and 256-column group
+__host__ __device__ constexpr int gemm_threads(int ew) { return 64 + 32 * ew; }
 
 enum EpiKind : int {
   kEpiLse = 0,    // logits tile -> per-row (max, sum exp) + target logit (+ store logits)
@@ -52,7 +57,8 @@ struct GemmJob {
   // kEpiLse
   const void* bias;        // [N] model dtype or null
   const int64_t* targets;  // [M] (rows of this job)
-  float2* part;            // [M, part_ld] (max, sum exp) per (row, N tile)
+  float2* part;            // [M, part_ld] (max, sum exp) per row and 128-column half of each
+                           // 256-column group: entry grp * kEpiColGroups + column group
   int part_ld;
   float* zt;               // [M] target logit
   void* logits;            // [M, logits_ld] model dtype or null

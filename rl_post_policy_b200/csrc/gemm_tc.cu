@@ -50,10 +50,10 @@ using namespace sm100;
 constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t kBBytes = kBNh * kBK * 2;            // 16 KB: this CTA's 128 rows of B per MMA
 constexpr uint32_t kTmemCols = 512;
-// Epilogue staging for the TMA output paths: per epilogue warp, two buffers of
-// one 32 x 32 fp32 box (4 KB), so a warp fills one while the other drains.
+// Epilogue staging for the TMA output paths: 8 boxes of 4 KB (32 rows x 128
+// bytes), one per epilogue warp (8 warps) or two (4 warps).
 constexpr uint32_t kOutBoxBytes = kOutBoxM * kOutBoxN * 4;
-constexpr uint32_t kOutStageBytes = 4 * 2 * kOutBoxBytes;
+constexpr uint32_t kOutStageBytes = 8 * kOutBoxBytes;
 
 // Pair tile kPairM x (kBN * NH).  NH = 1: one N=256 MMA per K=16 step, two
 // accumulators alternating between tiles (the epilogue of tile t overlaps the
@@ -215,8 +215,9 @@ __device__ __forceinline__ void add_bias32(const T* bias, float (&v)[32], int nv
   }
 }
 
-template <typename T, int NH>
-__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+template <typename T, int NH, int EW>
+__global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  static_assert(EW == 4 || EW == 8, "4 or 8 epilogue warps");
   using Cfg = TileCfg<NH>;
   constexpr int kStages = Cfg::kStages;
   constexpr uint32_t kStageBytes = Cfg::kStageBytes;
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 2 * 128);  // both CTAs' epilogue threads release the leader's accumulator
+      mbar_init(&tempty[b], 2 * EW * 32);  // both CTAs' epilogue threads release the leader's accumulator
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -434,8 +435,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       mbar_wait(done, 0, &no_abort, lim);
     }
   } else {
-    // ---------------- epilogue (warps 2..5, both CTAs) ----------------
+    // ---------------- epilogue (warps 2 .. EW+1, both CTAs) ----------------
+    // A warp may only read the tensor-memory quarter warp % 4.  With 8 warps,
+    // warps 2-5 take columns [0, 128) of every 256-column group and warps 6-9
+    // columns [128, 256); with 4, each warp takes the whole group.
+    constexpr int kCG = EW / 4;    // column groups
+    constexpr int kBoxes = 8 / EW;  // staging boxes per warp
     const int quarter = warp & 3;  // tensor-memory lanes [32*quarter, 32*quarter+32)
+    const int colgrp = (warp - 2) / 4;
+    const int c_lo = colgrp * (kBN / 32 / kCG);  // first 32-column slice
+    const int c_hi = c_lo + kBN / 32 / kCG;
     const int r_local = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -444,7 +453,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     const float job_scale0 = p.jobs[0].scale ? __ldg(p.jobs[0].scale) : 1.0f;
     const float job_scale1 = (p.njobs > 1 && p.jobs[1].scale) ? __ldg(p.jobs[1].scale) : 1.0f;
     // this warp's two staging boxes for the TMA output paths
-    const uint32_t stage0 = smem_u32(out_stage) + (uint32_t)quarter * 2 * kOutBoxBytes;
+    const uint32_t box0 = smem_u32(out_stage) + (uint32_t)((warp - 2) * kBoxes) * kOutBoxBytes;
     int sbuf = 0;
     for (int it = 0;; ++it) {
       const int tile = pair_tile(p, pair, npairs, it);
@@ -477,7 +486,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           float m_run = -INFINITY, s_run = 0.0f, ztv = 0.0f;
           bool got = false;
   #pragma unroll 1
-          for (int c = 0; c < kBN / 32; c += 2) {
+          for (int c = c_lo; c < c_hi; c += 2) {
             uint32_t w[32];
   #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -537,9 +546,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
               }
             }
             if (tma_logits && n0 + c * 32 < j.N && y < j.M) {
-              if (lane == 0) bulk_wait_group_read<1>();
+              // the box's previous contents have been read out by the TMA unit
+              if (lane == 0) bulk_wait_group_read<kBoxes - 1>();
               __syncwarp();
-              const uint32_t box = stage0 + (uint32_t)sbuf * kOutBoxBytes;
+              const uint32_t box = box0 + (uint32_t)sbuf * kOutBoxBytes;
               const uint32_t my_row = box + (uint32_t)lane * 128u;
   #pragma unroll
               for (int q = 0; q < 8; ++q)
@@ -551,11 +561,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                 tma_store_2d(&p.maps[j.out_map], box, n0 + c * 32, y);
                 bulk_commit_group();
               }
-              sbuf ^= 1;
+              if (kBoxes > 1) sbuf ^= 1;
             }
           }
           if (row_ok) {
-            j.part[(int64_t)row * j.part_ld + grp] = make_float2(m_run, s_run);
+            // one partial per row, 256-column group and column group; (-inf, 0)
+            // for a column group wholly past N
+            j.part[(int64_t)row * j.part_ld + grp * kEpiColGroups + colgrp] = make_float2(m_run, s_run);
+            if (kCG == 1) j.part[(int64_t)row * j.part_ld + grp * kEpiColGroups + 1] = make_float2(-INFINITY, 0.0f);
             if (got) j.zt[row] = ztv;
           }
         } else if (j.out_path != kOutDirect) {
@@ -571,7 +584,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           const int y = m0 + quarter * 32;
           const int step = j.out_f32 ? 1 : 2;  // 32-column TMEM slices per box
   #pragma unroll 1
-          for (int c = 0; c < kBN / 32; c += step) {
+          for (int c = c_lo; c < c_hi; c += step) {
             uint32_t w[32];
             float v[32];
             tmem_ld_32x32b_x32(taddr + c * 32, v);
@@ -587,10 +600,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             }
             const int col0 = n0 + c * 32;
             if (col0 >= j.N || y >= j.M) continue;
-            // the box written two boxes ago has been read out of shared memory
-            if (lane == 0) bulk_wait_group_read<1>();
+            // the box's previous contents have been read out by the TMA unit
+            if (lane == 0) bulk_wait_group_read<kBoxes - 1>();
             __syncwarp();
-            const uint32_t box = stage0 + (uint32_t)sbuf * kOutBoxBytes;
+            const uint32_t box = box0 + (uint32_t)sbuf * kOutBoxBytes;
             const uint32_t my_row = box + (uint32_t)lane * 128u;
   #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -603,12 +616,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
               else tma_store_2d(omap, box, col0, y);
               bulk_commit_group();
             }
-            sbuf ^= 1;
+            if (kBoxes > 1) sbuf ^= 1;
           }
         } else {
           const float sc = tc.job ? job_scale1 : job_scale0;
   #pragma unroll 1
-          for (int c = 0; c < kBN / 32; ++c) {
+          for (int c = c_lo; c < c_hi; ++c) {
             float v[32];
             tmem_ld_32x32b_x32(taddr + c * 32, v);
             const int col0 = n0 + c * 32;
@@ -734,7 +747,7 @@ int pick_tile_width(const GemmParams& p, int P) {
 
 namespace {
 
-template <typename T, int NH>
+template <typename T, int NH, int EW>
 cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
   constexpr size_t kGemmSmem = TileCfg<NH>::kSmem;
   static int max_pairs = 0;
@@ -744,19 +757,19 @@ cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(gemm_threads(EW));
   cfg.dynamicSmemBytes = kGemmSmem;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (max_pairs == 0) {  // one CTA per SM with or without the output staging
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<T, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<T, NH, EW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
     if (e != cudaSuccess) return e;
     DevInfo di;
     if ((e = dev_info(&di)) != cudaSuccess) return e;
     cfg.gridDim = dim3(di.sm_count & ~1);
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<T, NH>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<T, NH, EW>, &cfg);
     if (e != cudaSuccess) return e;
     max_pairs = n > 0 ? n : 1;
   }
@@ -768,7 +781,7 @@ cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
   GemmParams q = p;
   balance_schedule(&q, pairs);
   launch_begin(0, stream);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<T, NH>, q);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<T, NH, EW>, q);
   launch_end(0, stream);
   return e;
 }
@@ -790,8 +803,18 @@ cudaError_t launch_gemm(const GemmParams& p0, DType dt, cudaStream_t stream) {
   p.nh = nh;
   gemm_finalize_jobs(&p);
   if (p.total_tiles <= 0) return cudaSuccess;
-  if (dt == DType::BF16) return nh == 2 ? launch_t<__nv_bfloat16, 2>(p, stream) : launch_t<__nv_bfloat16, 1>(p, stream);
-  if (dt == DType::F16) return nh == 2 ? launch_t<__half, 2>(p, stream) : launch_t<__half, 1>(p, stream);
+  // fp32 TMA outputs (chunked dW accumulation, the debug hook) move 32-column
+  // boxes: 4 epilogue warps with two boxes each drain them faster than 8 with one
+  bool f32_tma = false;
+  for (int i = 0; i < p.njobs; ++i) f32_tma = f32_tma || (p.jobs[i].out_path != kOutDirect && p.jobs[i].out_f32);
+  if (dt == DType::BF16) {
+    if (f32_tma) return nh == 2 ? launch_t<__nv_bfloat16, 2, 4>(p, stream) : launch_t<__nv_bfloat16, 1, 4>(p, stream);
+    return nh == 2 ? launch_t<__nv_bfloat16, 2, 8>(p, stream) : launch_t<__nv_bfloat16, 1, 8>(p, stream);
+  }
+  if (dt == DType::F16) {
+    if (f32_tma) return nh == 2 ? launch_t<__half, 2, 4>(p, stream) : launch_t<__half, 1, 4>(p, stream);
+    return nh == 2 ? launch_t<__half, 2, 8>(p, stream) : launch_t<__half, 1, 8>(p, stream);
+  }
   return cudaErrorInvalidValue;
 }
 
