@@ -304,7 +304,7 @@ def loss_only(peaks, peak_kind):
     import rl_post_policy_b200 as pl
     import synth
     res = {}
-    for name, (bs, seq, reps) in {"sweep": (16, 1 << 23, 10), "small": (16, 1024, 200)}.items():
+    for name, (bs, seq, reps) in {"sweep": (16, 1 << 23, 50), "small": (16, 1024, 200)}.items():
         inp = synth.loss_inputs(bs, seq, torch.bfloat16, synth.seed_for(1, 1), len_lo=min(64, seq),
                                 len_hi=seq, device="cuda")
         g = torch.empty_like(inp["policy_lp"])
@@ -317,7 +317,7 @@ def loss_only(peaks, peak_kind):
             pl.pl_loss_ex(inp["policy_lp"], inp["old_lp"], inp["ref_lp"], inp["adv"], inp["mask"], bs, seq,
                           EPS_LO, EPS_HI, 0.04, mode, loss, g, None, None, ws, wsb)
 
-        for _ in range(3):
+        for _ in range(10):
             call()
         torch.cuda.synchronize()
         pl.pl_debug_timing_read()

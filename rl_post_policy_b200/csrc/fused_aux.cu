@@ -480,14 +480,19 @@ cudaError_t launch_dlogits(const DlogitsArgs& a0, DType dt, cudaStream_t s) {
     return cudaErrorInvalidValue;
   const dim3 grid((unsigned)((a.V + 255) / 256), (unsigned)a.n_rg);
   const size_t smem = (size_t)kDlStages * kDlTileBytes;
-  static bool attr_set[2] = {false, false};
+  static bool attr_set[kMaxDevices][2] = {};
   const int ti = dt == DType::BF16 ? 0 : 1;
-  if (!attr_set[ti]) {
-    const cudaError_t e = dt == DType::BF16
-        ? cudaFuncSetAttribute(dlogits_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-        : cudaFuncSetAttribute(dlogits_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set[ti] = true;
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(setup_mutex());
+    if (!attr_set[dev][ti]) {
+      const cudaError_t e = dt == DType::BF16
+          ? cudaFuncSetAttribute(dlogits_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+          : cudaFuncSetAttribute(dlogits_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr_set[dev][ti] = true;
+    }
   }
   if (dt == DType::BF16) {
     { launch_begin(2, s); dlogits_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(a); launch_end(2, s); }

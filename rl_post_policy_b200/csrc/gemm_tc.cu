@@ -750,7 +750,9 @@ namespace {
 template <typename T, int NH, int EW>
 cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
   constexpr size_t kGemmSmem = TileCfg<NH>::kSmem;
-  static int max_pairs = 0;
+  static int max_pairs_dev[kMaxDevices] = {};  // resident CTA pairs, per device
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -762,16 +764,22 @@ cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (max_pairs == 0) {  // one CTA per SM with or without the output staging
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<T, NH, EW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
-    if (e != cudaSuccess) return e;
-    DevInfo di;
-    if ((e = dev_info(&di)) != cudaSuccess) return e;
-    cfg.gridDim = dim3(di.sm_count & ~1);
-    int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<T, NH, EW>, &cfg);
-    if (e != cudaSuccess) return e;
-    max_pairs = n > 0 ? n : 1;
+  int max_pairs;
+  {
+    std::lock_guard<std::mutex> lock(setup_mutex());
+    if (max_pairs_dev[dev] == 0) {  // one CTA per SM with or without the output staging
+      cudaError_t e = cudaFuncSetAttribute(gemm_kernel<T, NH, EW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)kGemmSmem);
+      if (e != cudaSuccess) return e;
+      DevInfo di;
+      if ((e = dev_info(&di)) != cudaSuccess) return e;
+      cfg.gridDim = dim3(di.sm_count & ~1);
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<T, NH, EW>, &cfg);
+      if (e != cudaSuccess) return e;
+      max_pairs_dev[dev] = n > 0 ? n : 1;
+    }
+    max_pairs = max_pairs_dev[dev];
   }
   bool tma_out = false;
   for (int i = 0; i < p.njobs; ++i) tma_out = tma_out || p.jobs[i].out_path != kOutDirect;

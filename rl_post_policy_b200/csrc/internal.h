@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "../../include/pl.h"
@@ -117,6 +118,13 @@ struct DevInfo {
   size_t smem_optin = 0;
 };
 cudaError_t dev_info(DevInfo* out);
+
+// Host-side caches of per-kernel launch setup (shared-memory attributes,
+// occupancy) are kept per device, under one mutex, for processes that drive
+// several GPUs or call from several threads.
+constexpr int kMaxDevices = 64;
+int current_device();  // the current device's index, or -1
+std::mutex& setup_mutex();
 
 // PL_OK when the current device is compute capability 10.0.
 pl_status check_arch();

@@ -447,14 +447,22 @@ template <typename T, bool HAS_KL, bool HAS_GRAD, bool TWO_SIDED, bool VEC>
 cudaError_t launch_t(const LossArgs& a0, cudaStream_t stream) {
   auto kern = loss_kernel<T, HAS_KL, HAS_GRAD, TWO_SIDED, VEC>;
   const size_t dyn = VEC ? kMaskBitsBytes : 0;
-  static int per_sm = -1;
-  if (per_sm < 0) {
-    cudaError_t e = cudaSuccess;
-    if (dyn > 48 * 1024)
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, dyn);
-    if (e != cudaSuccess) { per_sm = -1; return e; }
-    if (per_sm < 1) per_sm = 1;
+  static int per_sm_dev[kMaxDevices] = {};  // resident blocks per SM, per device (0: not yet known)
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  int per_sm;
+  {
+    std::lock_guard<std::mutex> lock(setup_mutex());
+    if (per_sm_dev[dev] == 0) {
+      cudaError_t e = cudaSuccess;
+      if (dyn > 48 * 1024)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+      int n = 0;
+      if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, dyn);
+      if (e != cudaSuccess) return e;
+      per_sm_dev[dev] = n < 1 ? 1 : n;
+    }
+    per_sm = per_sm_dev[dev];
   }
   DevInfo di;
   cudaError_t e = dev_info(&di);

@@ -34,6 +34,17 @@ cudaError_t dev_info(DevInfo* out) {
   return cudaSuccess;
 }
 
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+std::mutex& setup_mutex() {
+  static std::mutex mu;
+  return mu;
+}
+
 pl_status check_arch() {
   DevInfo di;
   if (dev_info(&di) != cudaSuccess) return PL_ERR_CUDA;
