@@ -8,6 +8,11 @@
 * ``reverse_kl_autograd`` -- the card's autograd-aware reverse-KL entry point:
   pl_reverse_kl's fused forward + student-logit gradient, scaled by the
   incoming gradient in the backward (pl_scale).
+* ``fused_linear_grpo_loss`` -- the fused linear GRPO / BNPO loss of "Add
+  SM100 CuTe DSL GRPO fast path" ("Summary"): the forward is one
+  pl_fused_linear_grpo_temp call that also produces dX, dW and dbias (the
+  chunked path computes them with the loss); the backward scales them by the
+  incoming gradient (pl_scale).
 * ``fused_selective_logprob`` -- the fused-linear selective log-prob autograd
   path of "Add SM100 CuTe DSL GRPO fast path" (Liger-Kernel PR #1363,
   "Summary"): forward = pl_fused_selective_logprob (log-probs), backward = the
@@ -106,6 +111,62 @@ def reverse_kl_autograd(student_logits, teacher_logits, completions_mask=None):
     """Masked mean over rows of KL(softmax(student) || softmax(teacher)), differentiable
     in the student logits (shape (..., V); mask of the leading shape, or None)."""
     return _ReverseKL.apply(student_logits, teacher_logits, completions_mask)
+
+
+class _FusedLinearGRPO(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, X, W, bias, targets, Xref, Wref, old_lp, adv, mask, eps_lo, eps_hi, beta, reduction,
+                two_sided, temperature, chunk_rows):
+        bs, T = mask.shape
+        N, H = X.shape
+        V = W.shape[0]
+        mode = (pl.dtype_mode(X.dtype) | reduction | (pl.PL_CLIP_TWO_SIDED if two_sided else 0) |
+                (pl.PL_CHUNK_ROWS(chunk_rows) if chunk_rows else 0))
+        Xc, Wc = X.detach().contiguous(), W.detach().contiguous()
+        bc = bias.detach().contiguous() if bias is not None else None
+        need_x, need_w, need_b = ctx.needs_input_grad[0], ctx.needs_input_grad[1], ctx.needs_input_grad[2]
+        dX = torch.empty_like(Xc) if need_x else None
+        dW = torch.empty_like(Wc) if need_w else None
+        db = torch.empty_like(bc) if (need_b and bc is not None) else None
+        loss = torch.empty(1, dtype=torch.float32, device=X.device)
+        ref_x = Xref.detach().contiguous() if beta != 0 else None
+        ref_w = Wref.detach().contiguous() if beta != 0 else None
+        wsb = pl.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, int(dW is not None), int(db is not None))
+        ws = _workspace(wsb, X.device)
+        pl.check(pl.pl_fused_linear_grpo_temp(Xc, Wc, bc, targets.detach().to(torch.int64).contiguous(), ref_x,
+                                              ref_w, old_lp.detach().to(torch.float32).contiguous(),
+                                              adv.detach().to(torch.float32).contiguous(),
+                                              mask.detach().contiguous(), bs, T, H, V, eps_lo, eps_hi, beta,
+                                              temperature, mode, loss, dX, dW, db, None, None, None, ws, wsb),
+                 "pl_fused_linear_grpo_temp")
+        ctx.save_for_backward(dX, dW, db)
+        return loss[0]
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        dX, dW, db = ctx.saved_tensors
+        scale = grad_out.detach().to(torch.float32).reshape(1).contiguous()
+        out = []
+        for g in (dX, dW, db):
+            if g is None:
+                out.append(None)
+                continue
+            g = g.clone()
+            pl.check(pl.pl_scale(g, g.numel(), pl.dtype_mode(g.dtype), scale), "pl_scale")
+            out.append(g)
+        return (*out, None, None, None, None, None, None, None, None, None, None, None, None, None)
+
+
+def fused_linear_grpo_loss(X, W, targets, old_lp, adv, mask, bias=None, Xref=None, Wref=None, epsilon=0.2,
+                           epsilon_high=0.2, beta=0.0, reduction="grpo", two_sided=False, temperature=1.0,
+                           chunk_rows=None):
+    """GRPO (or BNPO) loss of the sampled tokens' log-probs under log_softmax((X W^T + bias) / temperature),
+    with the reference model's (Xref Wref^T / temperature) in the KL term when beta != 0; differentiable
+    in X, W and bias.  X [N, H], W [V, H], targets [N], old_lp [N] (or [bs, T]), adv [bs], mask [bs, T]."""
+    red = {"grpo": pl.PL_GRPO, "bnpo": pl.PL_BNPO}[reduction] if isinstance(reduction, str) else int(reduction)
+    return _FusedLinearGRPO.apply(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, float(epsilon),
+                                  float(epsilon_high), float(beta), red, bool(two_sided), float(temperature),
+                                  chunk_rows)
 
 
 class _SelectiveLogprob(torch.autograd.Function):

@@ -10,6 +10,9 @@ Registered under ``torch.ops.rl_post_policy_b200``:
 * ``selective_logprob(X, W, bias?, targets, chunk_rows) -> logp`` and
   ``selective_logprob_backward(X, W, bias?, targets, grad_logp, chunk_rows,
   need_x, need_w, need_b) -> (dX, dW, dbias)`` -- pl_fused_selective_logprob;
+* ``fused_linear_grpo(X, W, bias?, targets, Xref?, Wref?, old_lp, adv, mask,
+  ..., need_x, need_w, need_b) -> (loss, dX, dW, dbias)`` --
+  pl_fused_linear_grpo_temp, loss and gradients in one call;
 * ``scale(x, factor) -> x * factor`` -- pl_scale, for the backward passes.
 
 Each operator has a shape function (so tracing with FakeTensors, as
@@ -17,11 +20,12 @@ Each operator has a shape function (so tracing with FakeTensors, as
 "Entry points" section of the "Geometric-AI Kernels" model card: the loss
 kernels return dLoss/dinput with the loss, and the backward scales it by the
 incoming gradient.  The functions at the bottom (``bnpo_loss``, ``grpo_loss``,
-``reverse_kl_loss``, ``selective_logprob``) are the user-facing forms.
+``reverse_kl_loss``, ``selective_logprob``, ``fused_linear_grpo_loss``) are the
+user-facing forms.
 
 Argument marshalling only: every arithmetic step runs in libpl.so.  Gradients
-that are not needed come back from ``selective_logprob_backward`` as empty
-tensors (an operator cannot return None).
+that are not needed come back from ``selective_logprob_backward`` and
+``fused_linear_grpo`` as empty tensors (an operator cannot return None).
 """
 from __future__ import annotations
 
@@ -197,7 +201,79 @@ def _sl_backward(ctx, grad_logp):
 selective_logprob_op.register_autograd(_sl_backward, setup_context=_sl_setup)
 
 
+# ------------------------------------------------------------------ fused linear GRPO / BNPO
+@torch.library.custom_op(f"{_NS}::fused_linear_grpo", mutates_args=())
+def fused_linear_grpo(X: Tensor, W: Tensor, bias: Optional[Tensor], targets: Tensor, Xref: Optional[Tensor],
+                      Wref: Optional[Tensor], old_lp: Tensor, adv: Tensor, mask: Tensor, eps_lo: float,
+                      eps_hi: float, beta: float, reduction: int, two_sided: bool, temperature: float,
+                      chunk_rows: int, need_x: bool, need_w: bool,
+                      need_b: bool) -> tuple[Tensor, Tensor, Tensor, Tensor]:
+    bs, T = mask.shape
+    N, H = X.shape
+    V = W.shape[0]
+    mode = (pl.dtype_mode(X.dtype) | int(reduction) | (pl.PL_CLIP_TWO_SIDED if two_sided else 0) |
+            (pl.PL_CHUNK_ROWS(chunk_rows) if chunk_rows else 0))
+    Xc, Wc = X.detach().contiguous(), W.detach().contiguous()
+    bc = bias.detach().contiguous() if bias is not None else None
+    nb = need_b and bc is not None
+    dX = torch.empty_like(Xc) if need_x else Xc.new_empty((0,))
+    dW = torch.empty_like(Wc) if need_w else Wc.new_empty((0,))
+    db = torch.empty_like(bc) if nb else Xc.new_empty((0,))
+    loss = torch.empty((), dtype=torch.float32, device=X.device)
+    ref_x = Xref.detach().contiguous() if (beta != 0.0 and Xref is not None) else None
+    ref_w = Wref.detach().contiguous() if (beta != 0.0 and Wref is not None) else None
+    wsb = pl.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, int(need_w), int(nb))
+    ws = _workspace(wsb, X.device)
+    pl.check(pl.pl_fused_linear_grpo_temp(Xc, Wc, bc, targets.detach().to(torch.int64).contiguous(), ref_x, ref_w,
+                                          old_lp.detach().to(torch.float32).contiguous(),
+                                          adv.detach().to(torch.float32).contiguous(), mask.detach().contiguous(),
+                                          bs, T, H, V, eps_lo, eps_hi, beta, temperature, mode, loss,
+                                          dX if need_x else None, dW if need_w else None, db if nb else None,
+                                          None, None, None, ws, wsb), "pl_fused_linear_grpo_temp")
+    return loss, dX, dW, db
+
+
+@fused_linear_grpo.register_fake
+def _(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, eps_lo, eps_hi, beta, reduction, two_sided,
+      temperature, chunk_rows, need_x, need_w, need_b):
+    dX = torch.empty_like(X, memory_format=torch.contiguous_format) if need_x else X.new_empty((0,))
+    dW = torch.empty_like(W, memory_format=torch.contiguous_format) if need_w else W.new_empty((0,))
+    db = (torch.empty_like(bias, memory_format=torch.contiguous_format) if (need_b and bias is not None)
+          else X.new_empty((0,)))
+    return X.new_empty((), dtype=torch.float32), dX, dW, db
+
+
+def _flg_setup(ctx, inputs, output):
+    _, dX, dW, db = output
+    ctx.save_for_backward(dX, dW, db)
+    ctx.need = (inputs[16], inputs[17], inputs[18] and inputs[2] is not None)
+
+
+def _flg_backward(ctx, grad_loss, g_dx, g_dw, g_db):
+    dX, dW, db = ctx.saved_tensors
+    out = [scale(g, grad_loss) if need else None for g, need in zip((dX, dW, db), ctx.need)]
+    return (out[0], out[1], out[2]) + (None,) * 16
+
+
+fused_linear_grpo.register_autograd(_flg_backward, setup_context=_flg_setup)
+
+
 # ------------------------------------------------------------------ user-facing forms
+def fused_linear_grpo_loss(X, W, targets, old_lp, adv, mask, bias=None, Xref=None, Wref=None, epsilon=0.2,
+                           epsilon_high=0.2, beta=0.0, reduction="grpo", two_sided=False, temperature=1.0,
+                           chunk_rows=0):
+    """The fused linear GRPO / BNPO loss through the custom operator; differentiable in X, W and bias
+    (see ``rl_post_policy_b200.autograd.fused_linear_grpo_loss`` for the arguments)."""
+    red = {"grpo": pl.PL_GRPO, "bnpo": pl.PL_BNPO}[reduction] if isinstance(reduction, str) else int(reduction)
+    grad_on = torch.is_grad_enabled()
+    loss, _, _, _ = fused_linear_grpo(X, W, bias, targets, Xref, Wref, old_lp, adv, mask, float(epsilon),
+                                      float(epsilon_high), float(beta), red, bool(two_sided), float(temperature),
+                                      int(chunk_rows or 0), grad_on and X.requires_grad,
+                                      grad_on and W.requires_grad,
+                                      grad_on and bias is not None and bias.requires_grad)
+    return loss
+
+
 def bnpo_loss(policy_lp, old_lp, ref_lp, adv, mask, epsilon=0.2, epsilon_high=0.2, beta=0.0, two_sided=False):
     """BNPO loss (global token mean) through the custom operator; differentiable in policy_lp."""
     return policy_lp_loss(policy_lp, old_lp, ref_lp, adv, mask, epsilon, epsilon_high, beta, pl.PL_BNPO, two_sided)

@@ -11,7 +11,8 @@ OPS = torch.ops.rl_post_policy_b200
 
 
 def test_operators_are_registered():
-    for name in ("policy_loss", "reverse_kl", "selective_logprob", "selective_logprob_backward", "scale"):
+    for name in ("policy_loss", "reverse_kl", "selective_logprob", "selective_logprob_backward", "scale",
+                 "fused_linear_grpo"):
         assert hasattr(OPS, name), name
 
 
@@ -36,6 +37,11 @@ def test_shapes_under_fake_tensors():
         assert logp.shape == (10,) and logp.dtype == torch.float32
         dX, dW, db = OPS.selective_logprob_backward(X, W, b, t, logp, 0, True, False, True)
         assert dX.shape == X.shape and dW.numel() == 0 and db.shape == b.shape
+
+        old = torch.empty(10, device="cuda")
+        loss, dX, dW, db = OPS.fused_linear_grpo(X, W, b, t, X, W, old, adv[:2], torch.empty(2, 5, dtype=torch.uint8, device="cuda"),
+                                                 0.2, 0.28, 0.04, 1, False, 1.0, 0, True, True, False)
+        assert loss.shape == () and dX.shape == X.shape and dW.shape == W.shape and db.numel() == 0
 
         y = OPS.scale(lp, adv[:1])
         assert y.shape == lp.shape and y.dtype == lp.dtype

@@ -111,3 +111,48 @@ def test_opcheck():
     x = torch.randn(4, 8, device="cuda", dtype=torch.bfloat16)
     torch.library.opcheck(ops.scale.default, (x, torch.tensor([0.5], device="cuda")),
                           test_utils=("test_schema", "test_faketensor"))
+
+
+@pytest.mark.parametrize("chunk", [0, 64], ids=["one_chunk", "chunks64"])
+def test_fused_linear_grpo_autograd_and_op(chunk):
+    # loss.backward() through the fused linear path: the gradients equal the
+    # direct entry point's scaled by the outer factor, for the autograd.Function
+    # and the custom operator alike, eager and compiled
+    import rl_post_policy_b200 as pl
+    from rl_post_policy_b200 import autograd as ag
+    from rl_post_policy_b200 import torch_ops as ops
+    bs, T, H, V = 2, 96, 64, 700
+    inp = synth.fused_inputs(bs, T, H, V, torch.bfloat16, 6262, bias=True, need_ref=True)
+    inp["old_lp"] = (inp["old_noise"] - 6.5).float()
+    g = {k: v.cuda() for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    kw = dict(bias=None, Xref=g["Xref"], Wref=g["Wref"], epsilon=0.2, epsilon_high=0.28, beta=0.04,
+              reduction="bnpo", temperature=0.9, chunk_rows=chunk)
+    outer = -0.75
+
+    def run(f):
+        x, w = g["X"].clone().requires_grad_(True), g["W"].clone().requires_grad_(True)
+        b = g["bias"].clone().requires_grad_(True)
+        loss = f(x, w, g["targets"], g["old_lp"], g["adv"], g["mask"], **dict(kw, bias=b))
+        (outer * loss).backward()
+        return loss.detach().reshape(1), x.grad, w.grad, b.grad
+
+    # the direct entry point, unscaled
+    N = bs * T
+    mode = pl.PL_BF16 | pl.PL_BNPO | (pl.PL_CHUNK_ROWS(chunk) if chunk else 0)
+    loss = torch.empty(1, device="cuda")
+    dX, dW, db = torch.empty_like(g["X"]), torch.empty_like(g["W"]), torch.empty_like(g["bias"])
+    wsb = pl.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, 1, 1)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    pl.check(pl.pl_fused_linear_grpo_temp(g["X"], g["W"], g["bias"], g["targets"], g["Xref"], g["Wref"],
+                                          g["old_lp"], g["adv"], g["mask"], bs, T, H, V, 0.2, 0.28, 0.04, 0.9, mode,
+                                          loss, dX, dW, db, None, None, None, ws, wsb))
+    want = (loss, (dX.float() * outer).to(dX.dtype), (dW.float() * outer).to(dW.dtype),
+            (db.float() * outer).to(db.dtype))
+    for f in (ag.fused_linear_grpo_loss, ops.fused_linear_grpo_loss):
+        got = run(f)
+        for a_, b_ in zip(got, want):
+            assert torch.equal(a_, b_)
+    torch._dynamo.reset()
+    got = run(torch.compile(ops.fused_linear_grpo_loss, backend="aot_eager", fullgraph=True))
+    for a_, b_ in zip(got, want):
+        assert torch.equal(a_, b_)
