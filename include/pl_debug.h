@@ -65,6 +65,16 @@ pl_status pl_debug_timing_read(double* ms, int64_t* launches);
 void pl_debug_set_wait(unsigned long long wait_ns, unsigned extra_arrivals, unsigned extra_tx);
 
 /*
+ * Chooses the loss-only kernel for later calls on this process: 1 = the
+ * small-batch kernel (no grid barrier; every block counts the whole mask),
+ * used when bs * seq <= 65536 and bs <= 1024, else the cooperative kernel;
+ * 2 = always the cooperative kernel; 0 restores the default (1).  A
+ * pl_debug_set_wait with extra arrivals also selects the cooperative kernel,
+ * whose grid barrier it targets.  Returns PL_ERR_ARG for any other value.
+ */
+int pl_debug_set_loss_path(int path);
+
+/*
  * Forces the reverse-KL kernel's cluster size (CTAs sharing one row: 1, 2, 4 or
  * 8) for later calls on this process, so tests reach every row split; 0
  * restores the host's choice.  Returns PL_ERR_ARG for any other value.

@@ -90,6 +90,8 @@ _lib.pl_debug_set_wait.argtypes = [ctypes.c_ulonglong, ctypes.c_uint, ctypes.c_u
 _lib.pl_debug_set_wait.restype = None
 _lib.pl_debug_pair_tiles.argtypes = [_I, _I, _I, _I, _I, _P]
 _lib.pl_debug_pair_tiles.restype = _I
+_lib.pl_debug_set_loss_path.argtypes = [_I]
+_lib.pl_debug_set_loss_path.restype = _I
 _lib.pl_debug_pick_tile.argtypes = [_I, _P, _I]
 _lib.pl_debug_pick_tile.restype = _I
 _lib.pl_debug_set_gemm_tile.argtypes = [_I]
@@ -104,7 +106,7 @@ EXPORTED = ("pl_init", "pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_line
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
             "pl_version", "pl_debug_gemm", "pl_debug_gemm_out", "pl_debug_timing", "pl_debug_timing_read",
             "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_set_gemm_tile", "pl_debug_pair_tiles",
-            "pl_debug_pick_tile")
+            "pl_debug_pick_tile", "pl_debug_set_loss_path")
 
 
 class PLError(RuntimeError):
@@ -295,3 +297,8 @@ def pl_debug_pick_tile(problems, pairs: int) -> int:
     flat = [int(x) for mnk in problems for x in mnk]
     arr = (ctypes.c_int64 * max(len(flat), 1))(*flat)
     return int(_lib.pl_debug_pick_tile(len(problems), arr, pairs))
+
+
+def pl_debug_set_loss_path(path: int) -> int:
+    """Test hook: 0 default, 1 small-batch loss kernel when eligible, 2 cooperative kernel."""
+    return int(_lib.pl_debug_set_loss_path(int(path)))

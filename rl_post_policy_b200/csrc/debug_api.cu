@@ -134,6 +134,12 @@ DebugKnobs& debug_knobs() {
 }
 }  // namespace pl
 
+extern "C" int pl_debug_set_loss_path(int path) {
+  if (path < 0 || path > 2) return PL_ERR_ARG;
+  debug_knobs().loss_path = path;
+  return PL_OK;
+}
+
 extern "C" void pl_debug_set_wait(unsigned long long wait_ns, unsigned extra_arrivals, unsigned extra_tx) {
   DebugKnobs& k = debug_knobs();
   k.wait_ns = wait_ns ? wait_ns : kWaitLimitNs;

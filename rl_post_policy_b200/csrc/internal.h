@@ -89,6 +89,13 @@ pl_status run_loss(const void* lp, const void* old, const void* ref, const void*
                    int64_t* n_valid_out, int64_t* row_valid_out, void* ws, cudaStream_t stream);
 
 // Launches the single-pass loss kernel; returns a CUDA error code.
+// Small batches (n <= kSmallMaxTokens tokens, bs <= kSmallMaxRows) can take a
+// kernel without the grid barrier, in which every block counts the whole mask.
+constexpr int64_t kSmallMaxTokens = 65536;
+constexpr int kSmallMaxRows = 1024;
+bool loss_small_eligible(int64_t bs, int64_t n);
+cudaError_t launch_loss_small(const LossArgs& a, DType dt, bool has_kl, bool has_grad, bool two_sided, bool vec,
+                              cudaStream_t stream);
 cudaError_t launch_loss(const LossArgs& a, DType dt, bool has_kl, bool has_grad, bool two_sided,
                         bool vec, cudaStream_t stream);
 
@@ -102,6 +109,8 @@ struct DebugKnobs {
   unsigned extra_tx = 0;
   int rkl_cluster = 0;   // reverse-KL CTAs per cluster (1, 2, 4 or 8; 0 = the host's choice)
   int gemm_nh = 0;       // GEMM tile width in N=256 MMAs (1 or 2; 0 = the host's choice)
+  int loss_path = 0;     // loss kernel: 0 = the host's choice, 1 = small-batch kernel when eligible,
+                         // 2 = the cooperative kernel
 };
 DebugKnobs& debug_knobs();
 

@@ -146,7 +146,12 @@ pl_status run_loss(const void* lp, const void* old, const void* ref, const void*
   const bool has_grad = grad_out != nullptr;
   const bool vec = aligned(lp, 16) && aligned(old, 16) && (!has_kl || aligned(ref, 16)) &&
                    (!has_grad || aligned(grad_out, 16)) && aligned(mask, 16);
-  cudaError_t e = launch_loss(a, dt, has_kl, has_grad, (mode & PL_CLIP_TWO_SIDED) != 0, vec, stream);
+  // Small batches skip the cooperative launch and its grid barrier, unless a
+  // test forces the cooperative kernel or makes its barrier wait run out.
+  const DebugKnobs& k = debug_knobs();
+  const bool small = loss_small_eligible(bs, a.n) && k.loss_path != 2 && k.extra_arrivals == 0;
+  cudaError_t e = small ? launch_loss_small(a, dt, has_kl, has_grad, (mode & PL_CLIP_TWO_SIDED) != 0, vec, stream)
+                        : launch_loss(a, dt, has_kl, has_grad, (mode & PL_CLIP_TWO_SIDED) != 0, vec, stream);
   return e == cudaSuccess ? PL_OK : PL_ERR_CUDA;
 }
 

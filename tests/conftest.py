@@ -30,3 +30,13 @@ def gemm_tile(request):
     assert pl.pl_debug_set_gemm_tile(request.param) == 0
     yield request.param
     pl.pl_debug_set_gemm_tile(0)
+
+
+@pytest.fixture(params=[1, 2], ids=["small_kernel", "cooperative"])
+def loss_path(request):
+    """Runs a GPU test once with each loss-only kernel: the small-batch kernel
+    (used whenever the batch is small enough) and the cooperative kernel."""
+    import rl_post_policy_b200 as pl
+    assert pl.pl_debug_set_loss_path(request.param) == 0
+    yield request.param
+    pl.pl_debug_set_loss_path(0)

@@ -189,3 +189,9 @@ def test_debug_gemm_out_rejects_invalid_arguments():
         args = dict(base)
         args.update(over)
         assert pl.pl_debug_gemm_out(**args, stream=0) == code, over
+
+
+def test_loss_path_knob_rejects_invalid_values():
+    assert pl.pl_debug_set_loss_path(3) == pl.PL_ERR_ARG
+    assert pl.pl_debug_set_loss_path(-1) == pl.PL_ERR_ARG
+    assert pl.pl_debug_set_loss_path(0) == pl.PL_OK

@@ -40,6 +40,8 @@ def _ulp(x, dtype):
 def test_loss_kernel_random_settings(bs, seq, dtype, red, beta, two_sided, eps_lo, eps_hi, adv_lp, offset, seed,
                                      keep):
     import rl_post_policy_b200 as pl
+    # alternate the two loss kernels (every drawn size here is small enough for either)
+    assert pl.pl_debug_set_loss_path(1 + (seed & 1)) == 0
     dev = torch.device("cuda")
     inp = synth.loss_inputs(bs, seq, torch.float32, seed, len_lo=1, len_hi=seq)
     g = torch.Generator().manual_seed(seed + 1)
@@ -89,6 +91,7 @@ def test_loss_kernel_random_settings(bs, seq, dtype, red, beta, two_sided, eps_l
         err, bound = np.abs(gg - wr) / _ulp(wr, dtype), 1.0
     bad = (err > bound) & ~kink
     assert not bad.any(), (int(bad.sum()), float(err[~kink].max()))
+    pl.pl_debug_set_loss_path(0)
 
 
 @settings(**SETTINGS)

@@ -16,7 +16,7 @@ import torch
 import oracle
 import synth
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("loss_path")]
 
 EPS_LO, EPS_HI = 0.2, 0.28
 DTYPES = [torch.bfloat16, torch.float16, torch.float32]
