@@ -57,8 +57,9 @@ def parse():
     ap.add_argument("--no-reverse-kl", action="store_true")
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip the temperature and selective log-prob measurements")
-    ap.add_argument("--only", choices=["reverse_kl", "loss_only"], default=None,
-                    help="run one side measurement alone and print its JSON (for profiling)")
+    ap.add_argument("--only", choices=["reverse_kl", "loss_only", "loss_matrix"], default=None,
+                    help="run one side measurement alone and print its JSON (for profiling); loss_matrix: "
+                         "the loss kernel's 24 variants at bs=16 x 1024 and its bandwidth sweep, L2 flushed")
     ap.add_argument("--reps", type=int, default=30, help="timed calls per side measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256, help="rows in the oracle's timed sample")
@@ -363,6 +364,71 @@ def loss_only(peaks, peak_kind):
     }
 
 
+def loss_matrix(peaks, peak_kind, reps=20):
+    """The loss kernel over its variants: BNPO/GRPO x beta in {0.04, 0} x fwd+bwd / fwd-only x
+    bf16/fp16/fp32 at bs=16 x seq=1024 (launch-latency bound: about 144 KB per call in bf16), and
+    a bandwidth sweep of bf16 BNPO fwd+bwd, beta=0.04, bs=16 x seq=2^18 ... 2^23.  A 256 MB buffer
+    is written between calls so every call starts with a cold L2; only the loss kernel's own
+    launches are timed (CUDA events around each)."""
+    import rl_post_policy_b200 as pl
+    import synth
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    peak = float(peaks["hbm_gbs"])
+
+    def time_call(call):
+        for _ in range(3):
+            flush.zero_()
+            call()
+        torch.cuda.synchronize()
+        pl.pl_debug_timing_read()
+        pl.pl_debug_timing(True)
+        for _ in range(reps):
+            flush.zero_()
+            call()
+        torch.cuda.synchronize()
+        pl.pl_debug_timing(False)
+        ms, n = pl.pl_debug_timing_read()
+        return ms[1] / max(n[1], 1)
+
+    def one(bs, seq, dt, red, beta, grad, inp32):
+        lp, old, ref = (inp32[k].to(dt) for k in ("policy_lp", "old_lp", "ref_lp"))
+        g = torch.empty_like(lp) if grad else None
+        loss = torch.zeros(1, device="cuda")
+        wsb = pl.pl_loss_workspace_bytes(bs, seq)
+        ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+        mode = pl.dtype_mode(dt) | red
+
+        def call():
+            pl.pl_loss_ex(lp, old, ref if beta else None, inp32["adv"], inp32["mask"], bs, seq, EPS_LO, EPS_HI,
+                          beta, mode, loss, g, None, None, ws, wsb)
+
+        per = time_call(call)
+        esz = lp.element_size()
+        tokens = bs * seq
+        bytes_ = tokens * ((2 + (1 if beta else 0) + (1 if grad else 0)) * esz + 1)
+        return {"bs": bs, "seq": seq, "dtype": str(dt).split(".")[-1], "reduction": "grpo" if red else "bnpo",
+                "beta": beta, "grad": grad, "us_per_call": per * 1e3, "tokens_per_s": tokens / (per * 1e-3),
+                "algorithmic_bytes": bytes_, "GB_per_s": bytes_ / (per * 1e-3) / 1e9,
+                "frac": bytes_ / (per * 1e-3) / 1e9 / peak}
+
+    variants = []
+    inp32 = synth.loss_inputs(16, 1024, torch.float32, synth.seed_for(1), device="cuda")
+    for dt in (torch.bfloat16, torch.float16, torch.float32):
+        for red in (pl.PL_BNPO, pl.PL_GRPO):
+            for beta in (0.04, 0.0):
+                for grad in (True, False):
+                    variants.append(one(16, 1024, dt, red, beta, grad, inp32))
+    sweep = []
+    for k in range(18, 24):
+        seq = 1 << k
+        inp = synth.loss_inputs(16, seq, torch.float32, synth.seed_for(1, 1), len_lo=64, len_hi=seq, device="cuda")
+        sweep.append(one(16, seq, torch.bfloat16, pl.PL_BNPO, 0.04, True, inp))
+        del inp
+    return {"metric": "loss kernel variants and bandwidth sweep", "peak_GB_per_s": peak,
+            "peak_source": f"{peak_kind} hbm_gbs", "l2": "256 MB written between calls",
+            "variants_bs16_seq1024": variants, "sweep_bf16_bnpo_beta0.04": sweep}
+
+
 # ------------------------------------------------------------------ temperature, selective log-prob
 def next_rows(d, inp, ws, wsb, mode, peak, reps=20):
     """The fused step at temperature 0.7 (pl_fused_linear_grpo_temp) and the fused
@@ -540,7 +606,12 @@ def run_ours(args):
     peaks, peak_kind = load_peaks()
     if args.only:
         if rank == 0:
-            out = reverse_kl(peaks, peak_kind, args.reps) if args.only == "reverse_kl" else loss_only(peaks, peak_kind)
+            if args.only == "reverse_kl":
+                out = reverse_kl(peaks, peak_kind, args.reps)
+            elif args.only == "loss_matrix":
+                out = loss_matrix(peaks, peak_kind)
+            else:
+                out = loss_only(peaks, peak_kind)
             print(json.dumps(out), flush=True)
         return
     d, inp, ws, wsb, mode = make_fused_inputs(args.workload, rank, args.chunk_rows)
@@ -617,10 +688,25 @@ def run_ours(args):
     e2e_val = total_tokens / args.steps / (e2e_ms * 1e-3)
 
     extra = {}
+
+    def side(fn, *fargs):
+        # The bandwidth-bound side measurements come after seconds of power-capped
+        # GEMM work, which leaves the SM clock low for a while; they get an idle
+        # pause first and carry the clocks sampled while they ran.
+        torch.cuda.synchronize()
+        time.sleep(2.0)
+        cs = ClockSampler(torch.cuda.current_device())
+        cs.start()
+        time.sleep(0.3)
+        out = fn(*fargs)
+        torch.cuda.synchronize()
+        out["clocks"] = cs.stop()
+        return out
+
     if rank == 0 and ws_world == 1 and not args.no_loss_only:
-        extra["loss_only"] = loss_only(peaks, peak_kind)
+        extra["loss_only"] = side(loss_only, peaks, peak_kind)
     if rank == 0 and ws_world == 1 and not args.no_reverse_kl:
-        extra["reverse_kl"] = reverse_kl(peaks, peak_kind, args.reps)
+        extra["reverse_kl"] = side(reverse_kl, peaks, peak_kind, args.reps)
     if rank == 0 and ws_world == 1 and not args.no_next_rows:
         extra.update(next_rows(d, inp, ws, wsb, mode, float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))))
     cpu = None
