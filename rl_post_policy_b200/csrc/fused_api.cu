@@ -7,6 +7,7 @@
 //                combine  (lse, logp, ref_logp, loss partials, g)
 //                dlogits  (in place, 2^e-scaled, + dbias)                       (if a gradient is wanted)
 //                GEMM  [dX rows of the chunk = dz W]  [dW (+)= dz^T X_chunk]     (if dX or dW)
+//          -> convert (the fp32 dW accumulator to the model dtype; several chunks only)
 //          -> finalize (fixed-order loss sum)
 //
 // following "Add SM100 CuTe DSL GRPO fast path" (Liger-Kernel PR #1363):

@@ -1,23 +1,27 @@
 // Persistent tcgen05 GEMM for sm_100a with the epilogues of the fused path.
 //
 // CTAs run in pairs (clusters of two, one CTA per SM); a pair owns a 256 x 256
-// output tile and the grid holds as many pairs as can be resident, each
-// walking the concatenated tile list of up to two GEMM problems round-robin.
+// or 256 x 512 output tile (NH = 1 or 2 N=256 MMAs per K step, picked per
+// launch by pick_tile_width) and the grid holds as many pairs as can be
+// resident, each walking its share of the tiles of up to two GEMM problems.
 // Per CTA:
 //   warp 0    one lane issues TMA tile loads (128-byte swizzle, no multicast)
-//             of this CTA's 128 rows of A and 128 rows (of the tile's 256
-//             columns) of B into a 6-stage ring (32 KB per stage); the pair
-//             leader's mbarrier counts both CTAs' bytes;
-//   warp 1    allocates 512 tensor-memory columns (two 128 x 256 fp32
-//             accumulators, cta_group::2); in the leader one lane issues
+//             of this CTA's 128 rows of A and its half of the tile's columns of
+//             B into the operand ring (6 stages of 32 KB at NH = 1, 4 of 48 KB
+//             at NH = 2); the pair leader's mbarrier counts both CTAs' bytes;
+//   warp 1    allocates 512 tensor-memory columns (two alternating 128 x 256
+//             fp32 accumulators at NH = 1, one 128 x 512 at NH = 2,
+//             cta_group::2); in the leader one lane issues
 //             tcgen05.mma.cta_group::2 (M=256, N=256, K=16), which reads the A
 //             and B halves from both CTAs' shared memory and writes each CTA's
 //             128 accumulator rows into its own tensor memory, and commits each
 //             stage back to both producers and each tile to both epilogues;
-//   warps 2-5 the epilogue: one accumulator row per thread (tcgen05.ld
-//             32x32b), 32 columns at a time, overlapping the next tile's
-//             mainloop thanks to the second accumulator; both CTAs release the
-//             accumulator on the leader's barrier.
+//   warps 2.. the epilogue, EW = 8 warps (or 4): one accumulator row per thread
+//             (tcgen05.ld 32x32b), 32 columns at a time, two warps per 32-lane
+//             quarter of tensor memory splitting each 256-column group; it
+//             overlaps the next tile's mainloop (second accumulator at NH = 1,
+//             the drained half at NH = 2); both CTAs release the accumulator on
+//             the leader's barrier.
 // Splitting B across the pair halves each SM's shared-memory operand traffic
 // compared with one CTA computing a 128 x 256 tile alone.
 // Operands may be K-major or MN-major (the backward GEMMs read the logits
@@ -25,12 +29,14 @@
 //
 // Epilogues ("Add SM100 CuTe DSL GRPO fast path", Liger-Kernel PR #1363,
 // "Summary": full logits are never materialised beyond a bounded workspace):
-//   kEpiLse   -- per (row, 256-column vocabulary tile): running max and sum of
-//                exp(z - max) over the valid columns, the target logit when the
-//                row's target falls in the tile, optional bias add and optional
-//                store of the logits in the model dtype;
-//   kEpiStore -- acc * scale (+ an fp32 accumulator) stored in the model dtype
-//                or in fp32 (dX; dW / dbias with fp32 accumulation across chunks).
+//   kEpiLse   -- per (row, 128-column half of a 256-column vocabulary tile):
+//                running max and sum of exp(z - max) over the valid columns,
+//                the target logit when the row's target falls in it, optional
+//                bias add, and the logits stored in the model dtype by TMA;
+//   kEpiStore -- acc * scale stored in the model dtype (dX, one-chunk dW) or
+//                fp32 (dW accumulated across chunks: a TMA store, then TMA adds),
+//                through shared-memory boxes and TMA, or per-thread stores for
+//                outputs that are not 16-byte aligned.
 //
 // Every wait is bounded (GemmParams::wait_ns); when one runs out the CTA sets a
 // shared abort flag, every role drains out, the leader waits (bounded) for its

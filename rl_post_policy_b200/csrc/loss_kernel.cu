@@ -17,6 +17,8 @@
 //   C. the last block to finish sums the partials in block order (fp64, so the
 //      result is deterministic), writes the loss and counts, and returns the
 //      workspace counters to zero.
+// Batches of up to 65536 tokens take the barrier-free kernel of loss_small.cu
+// instead, with the same per-token arithmetic (policy_math.cuh).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
