@@ -19,8 +19,8 @@
   same entry point with the incoming dL/dlogp (dX, dW, dbias).
 
 Argument marshalling only: every arithmetic step runs in libpl.so's kernels.
-Workspaces are cached per (device, size) and zero-filled once, as the C ABI
-requires; calls that share one must be ordered on one stream.
+Workspaces are cached per (entry point, device, size) and zero-filled once, as
+the C ABI requires; calls that share one must be ordered on one stream.
 """
 from __future__ import annotations
 
@@ -31,8 +31,10 @@ from . import binding as pl
 _ws_cache: dict = {}
 
 
-def _workspace(nbytes: int, device) -> torch.Tensor:
-    key = (torch.device(device).index, nbytes)
+def _workspace(kind: str, nbytes: int, device) -> torch.Tensor:
+    """A zero-filled workspace per entry point (`kind`), device and size: entry
+    points lay their workspaces out differently, so they never share one."""
+    key = (kind, torch.device(device).index, nbytes)
     ws = _ws_cache.get(key)
     if ws is None:
         ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
@@ -50,7 +52,7 @@ class _PolicyLoss(torch.autograd.Function):
         grad = torch.empty_like(lp)
         loss = torch.empty(1, dtype=torch.float32, device=lp.device)
         wsb = pl.pl_loss_workspace_bytes(bs, seq)
-        ws = _workspace(wsb, lp.device)
+        ws = _workspace("loss", wsb, lp.device)
         adv_c = adv.detach().to(torch.float32).contiguous()
         pl.check(pl.pl_loss_ex(lp, old_lp.detach().contiguous(), None if beta == 0 else ref_lp.detach().contiguous(),
                                adv_c, mask.detach().contiguous(), bs, seq, eps_lo, eps_hi, beta, mode, loss,
@@ -132,7 +134,7 @@ class _FusedLinearGRPO(torch.autograd.Function):
         ref_x = Xref.detach().contiguous() if beta != 0 else None
         ref_w = Wref.detach().contiguous() if beta != 0 else None
         wsb = pl.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, int(dW is not None), int(db is not None))
-        ws = _workspace(wsb, X.device)
+        ws = _workspace("fused", wsb, X.device)
         pl.check(pl.pl_fused_linear_grpo_temp(Xc, Wc, bc, targets.detach().to(torch.int64).contiguous(), ref_x,
                                               ref_w, old_lp.detach().to(torch.float32).contiguous(),
                                               adv.detach().to(torch.float32).contiguous(),
@@ -180,7 +182,7 @@ class _SelectiveLogprob(torch.autograd.Function):
         tg = targets.detach().to(torch.int64).contiguous()
         logp = torch.empty(N, dtype=torch.float32, device=X.device)
         wsb = pl.pl_fused_selective_logprob_workspace_bytes(N, H, V, mode, 1, int(bc is not None))
-        ws = _workspace(wsb, X.device)
+        ws = _workspace("selective", wsb, X.device)
         pl.check(pl.pl_fused_selective_logprob(Xc, Wc, bc, tg, N, H, V, mode, None, logp, None, None, None,
                                                ws, wsb), "pl_fused_selective_logprob")
         ctx.save_for_backward(Xc, Wc, bc, tg)
@@ -201,7 +203,7 @@ class _SelectiveLogprob(torch.autograd.Function):
         g = grad_logp.detach().to(torch.float32).contiguous()
         wsb = pl.pl_fused_selective_logprob_workspace_bytes(N, H, V, ctx.mode, int(dW is not None),
                                                             int(db is not None))
-        ws = _workspace(wsb, Xc.device)
+        ws = _workspace("selective", wsb, Xc.device)
         pl.check(pl.pl_fused_selective_logprob(Xc, Wc, bc, tg, N, H, V, ctx.mode, g, None, dX, dW, db, ws,
                                                wsb), "pl_fused_selective_logprob")
         return dX, dW, db, None, None

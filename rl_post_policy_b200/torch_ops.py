@@ -65,7 +65,7 @@ def policy_loss(policy_lp: Tensor, old_lp: Tensor, ref_lp: Optional[Tensor], adv
     grad = torch.empty_like(lp)
     loss = torch.empty((), dtype=torch.float32, device=lp.device)
     wsb = pl.pl_loss_workspace_bytes(bs, seq)
-    ws = _workspace(wsb, lp.device)
+    ws = _workspace("loss", wsb, lp.device)
     ref = None if beta == 0.0 or ref_lp is None else ref_lp.detach().contiguous()
     pl.check(pl.pl_loss_ex(lp, old_lp.detach().contiguous(), ref, adv.detach().to(torch.float32).contiguous(),
                            mask.detach().contiguous(), bs, seq, eps_lo, eps_hi, beta, mode, loss, grad, None,
@@ -138,7 +138,7 @@ def selective_logprob_op(X: Tensor, W: Tensor, bias: Optional[Tensor], targets: 
     bc = bias.detach().contiguous() if bias is not None else None
     logp = torch.empty(N, dtype=torch.float32, device=X.device)
     wsb = pl.pl_fused_selective_logprob_workspace_bytes(N, H, V, mode, 1, int(bc is not None))
-    ws = _workspace(wsb, X.device)
+    ws = _workspace("selective", wsb, X.device)
     pl.check(pl.pl_fused_selective_logprob(Xc, Wc, bc, targets.detach().to(torch.int64).contiguous(), N, H, V,
                                            mode, None, logp, None, None, None, ws, wsb),
              "pl_fused_selective_logprob")
@@ -166,7 +166,7 @@ def selective_logprob_backward(X: Tensor, W: Tensor, bias: Optional[Tensor], tar
         g = grad_logp.detach().to(torch.float32).contiguous()
         wsb = pl.pl_fused_selective_logprob_workspace_bytes(N, H, V, mode, int(need_w),
                                                             int(need_b and bc is not None))
-        ws = _workspace(wsb, X.device)
+        ws = _workspace("selective", wsb, X.device)
         pl.check(pl.pl_fused_selective_logprob(Xc, Wc, bc, targets.detach().to(torch.int64).contiguous(), N, H,
                                                V, mode, g, None, dX if need_x else None,
                                                dW if need_w else None,
@@ -223,7 +223,7 @@ def fused_linear_grpo(X: Tensor, W: Tensor, bias: Optional[Tensor], targets: Ten
     ref_x = Xref.detach().contiguous() if (beta != 0.0 and Xref is not None) else None
     ref_w = Wref.detach().contiguous() if (beta != 0.0 and Wref is not None) else None
     wsb = pl.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, int(need_w), int(nb))
-    ws = _workspace(wsb, X.device)
+    ws = _workspace("fused", wsb, X.device)
     pl.check(pl.pl_fused_linear_grpo_temp(Xc, Wc, bc, targets.detach().to(torch.int64).contiguous(), ref_x, ref_w,
                                           old_lp.detach().to(torch.float32).contiguous(),
                                           adv.detach().to(torch.float32).contiguous(), mask.detach().contiguous(),
