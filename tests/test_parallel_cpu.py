@@ -1,6 +1,8 @@
-"""The data-parallel step (rl_post_policy_b200.parallel) on two `gloo` CPU ranks.
+"""The data-parallel steps (rl_post_policy_b200.parallel) on two and three
+`gloo` CPU ranks.
 
-Each rank takes its share of the sequences of one seeded batch (2 and 3 of 5).  The per-rank
+Each rank takes its share of the sequences of one seeded batch (2 + 3, or
+2 + 1 + 2, of 5 for the fused step).  The per-rank
 operations are the CPU oracle (the fused loss and gradients of the rank's
 shard, normalised by the shard's own count) and plain tensor arithmetic for
 the ratio and the scale, so what is under test is the host-side sequence: the
@@ -49,7 +51,7 @@ SCRIPT = textwrap.dedent("""
     want = oracle.fused_grpo(inp["X"], inp["W"], inp["bias"], inp["targets"], inp["Xref"], inp["Wref"],
                              inp["old_lp"].reshape(bs, T), inp["adv"], inp["mask"], eps_lo=0.2, eps_hi=0.28,
                              beta=0.04, reduction=red)
-    seqs = [range(0, 2), range(2, 5)][rank]          # unequal shards; rank 1 holds the empty sequence
+    seqs = {shards}[rank]                               # unequal shards; the last holds the empty sequence
     rows = [r * T + t for r in seqs for t in range(T)]
 
     class OracleOps:
@@ -82,13 +84,17 @@ SCRIPT = textwrap.dedent("""
 """)
 
 
+SHARDS = {2: "[range(0, 2), range(2, 5)]", 3: "[range(0, 2), range(2, 3), range(3, 5)]"}
+
+
+@pytest.mark.parametrize("world", [2, 3], ids=["2ranks", "3ranks"])
 @pytest.mark.parametrize("red", [0, 1], ids=["bnpo", "grpo"])
-def test_dp_step_matches_whole_batch_oracle(red):
-    script = SCRIPT.format(root=ROOT, red=red)
+def test_dp_step_matches_whole_batch_oracle(red, world):
+    script = SCRIPT.format(root=ROOT, red=red, shards=SHARDS[world])
     port = _free_port()
     procs = []
-    for r in range(2):
-        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE="2", MASTER_ADDR="127.0.0.1",
+    for r in range(world):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
                    MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="")
         procs.append(subprocess.Popen([sys.executable, "-c", script], env=env, stdout=subprocess.PIPE,
                                       stderr=subprocess.PIPE, text=True))
@@ -115,7 +121,7 @@ LOSS_SCRIPT = textwrap.dedent("""
     inp["mask"][5] = 0                                  # a fully masked sequence
     kw = dict(eps_lo=0.2, eps_hi=0.28, beta=0.04, reduction=red, two_sided=two_sided)
     want = oracle.policy_loss(inp["policy_lp"], inp["old_lp"], inp["ref_lp"], inp["adv"], inp["mask"], **kw)
-    seqs = [[0, 1, 2], [3, 4, 5, 6]][rank]              # unequal shards; rank 1 holds the empty sequence
+    seqs = {shards}[rank]                               # unequal shards; the last holds the empty sequence
 
     class OracleOps:
         def local_loss(self, lp, old, ref, adv, mask, eps_lo, eps_hi, beta, reduction, two_sided=False,
@@ -141,13 +147,17 @@ LOSS_SCRIPT = textwrap.dedent("""
 """)
 
 
+LOSS_SHARDS = {2: "[[0, 1, 2], [3, 4, 5, 6]]", 3: "[[0, 1], [2, 3, 4], [5, 6]]"}
+
+
+@pytest.mark.parametrize("world", [2, 3], ids=["2ranks", "3ranks"])
 @pytest.mark.parametrize("red,two_sided", [(0, False), (1, False), (1, True)], ids=["bnpo", "grpo", "grpo_two_sided"])
-def test_dp_loss_step_matches_whole_batch_oracle(red, two_sided):
-    script = LOSS_SCRIPT.format(root=ROOT, red=red, two_sided=two_sided)
+def test_dp_loss_step_matches_whole_batch_oracle(red, two_sided, world):
+    script = LOSS_SCRIPT.format(root=ROOT, red=red, two_sided=two_sided, shards=LOSS_SHARDS[world])
     port = _free_port()
     procs = []
-    for r in range(2):
-        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE="2", MASTER_ADDR="127.0.0.1",
+    for r in range(world):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
                    MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="")
         procs.append(subprocess.Popen([sys.executable, "-c", script], env=env, stdout=subprocess.PIPE,
                                       stderr=subprocess.PIPE, text=True))
