@@ -88,9 +88,11 @@ typedef enum {
  * pl_loss: fused forward + backward (grad_out != NULL) or forward-only
  * (grad_out == NULL) of the BNPO/GRPO loss above, as ONE kernel launch: the
  * valid-token counts (global for BNPO, per sequence for GRPO) are taken on the
- * device in a first phase, a bounded grid barrier orders them before the
- * scaling phase, and the last block to finish reduces the per-block partial sums
- * in a fixed order (deterministic).  No host synchronisation.
+ * device before any gradient is scaled -- in a first phase ordered by a bounded
+ * grid barrier, or, for batches of up to 65536 tokens and 1024 sequences, by
+ * every block counting the whole mask itself -- and the last block to finish
+ * reduces the per-block partial sums in a fixed order (deterministic for a
+ * given size).  No host synchronisation.
  *
  *   policy_lp, old_lp, ref_lp : [bs, seq] in the mode's dtype.  ref_lp may be NULL
  *                               only when beta == 0 (the KL branch is then compiled
@@ -127,7 +129,9 @@ pl_status pl_loss(const void* policy_lp, const void* old_lp, const void* ref_lp,
  *   workspace     : device buffer of at least pl_loss_workspace_bytes(bs, seq) bytes,
  *                   256-byte aligned, zero-filled by the caller ONCE after allocation; the kernel
  *                   returns its counters to zero, so it stays reusable.  Calls that
- *                   share a workspace must be ordered on one stream.
+ *                   share a workspace must be ordered on one stream.  After
+ *                   pl_device_status has reported a device error, zero-fill the
+ *                   workspace again before reusing it.
  */
 pl_status pl_loss_ex(const void* policy_lp, const void* old_lp, const void* ref_lp,
                      const void* adv, const uint8_t* mask, int64_t bs, int64_t seq,
