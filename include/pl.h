@@ -33,7 +33,9 @@
  *     return an error code before any launch and before any output is written.
  *   - Problems only the device can see (a bounded wait that ran out, a target id
  *     outside [0, V)) set a sticky flag in the workspace; outputs are then
- *     undefined.  Read and clear it with pl_device_status().
+ *     undefined.  Read and clear it with pl_device_status().  After a wait that
+ *     ran out, zero-fill a caller-owned workspace again before reusing it (a
+ *     call cut short may leave its counters set).
  *   - No exception crosses this boundary.
  */
 #ifndef PL_H_
@@ -129,9 +131,7 @@ pl_status pl_loss(const void* policy_lp, const void* old_lp, const void* ref_lp,
  *   workspace     : device buffer of at least pl_loss_workspace_bytes(bs, seq) bytes,
  *                   256-byte aligned, zero-filled by the caller ONCE after allocation; the kernel
  *                   returns its counters to zero, so it stays reusable.  Calls that
- *                   share a workspace must be ordered on one stream.  After
- *                   pl_device_status has reported a device error, zero-fill the
- *                   workspace again before reusing it.
+ *                   share a workspace must be ordered on one stream.
  */
 pl_status pl_loss_ex(const void* policy_lp, const void* old_lp, const void* ref_lp,
                      const void* adv, const uint8_t* mask, int64_t bs, int64_t seq,
