@@ -90,7 +90,7 @@ def fused_inputs(bs: int, T: int, H: int, V: int, dtype: torch.dtype, seed: int,
         out["Xref"] = (X32 + normal((N, H), s + 3, std=0.01, device=device)).to(dtype)
     del X32
     W32 = normal((V, H), s + 2, std=0.02, device=device)
-    out["W"] = W32.to(dtype)
+    out["W"] = W32.to(dtype, copy=True)  # a copy even for fp32: W32 becomes Wref below
     if need_ref:
         W32.add_(normal((V, H), s + 4, std=0.002, device=device))
         out["Wref"] = W32.to(dtype)
