@@ -11,7 +11,14 @@ module only marshals arrays and composes the three steps the pages describe:
 2. the PPO-clipped loss with the k3 KL penalty, reduced BNPO- or GRPO-style
    ("Geometric-AI Kernels" model card, "BNPO Loss" and "GRPO Loss"),
 3. the backward pass to dX, dW and dbias (chain rule through log-softmax and
-   the linear layer).
+   the linear layer);
+
+with the logits divided by a sampling temperature where one is given, and,
+separately, the reverse-KL self-distillation loss and its student gradient
+("Geometric-AI Kernels" model card, "Reverse KL").  Every function is pinned
+by tests/test_oracle_pins.py and tests/test_oracle_reverse_kl.py against
+closed forms, invariants, brute force, library routines and finite
+differences.
 """
 from __future__ import annotations
 
