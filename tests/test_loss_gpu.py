@@ -1,4 +1,7 @@
-"""Parity of the loss-only CUDA kernel (pl_loss / pl_loss_ex) with the CPU oracle.
+"""Parity of the loss-only CUDA kernels (pl_loss / pl_loss_ex) with the CPU oracle.
+Every test runs twice through the loss_path fixture: with the small-batch kernel
+(taken whenever the batch has at most 65536 tokens and 1024 sequences) and with
+the cooperative kernel.
 
 Tolerances: loss relative error <= 1e-5 (fp32 inputs) and <= 1e-3 (bf16/fp16);
 fp32 grad max abs error <= 1e-6; bf16/fp16 grad within one unit in the last
