@@ -20,6 +20,8 @@ def loads(t0, t1, c0, c1, pairs):
 
 @pytest.mark.parametrize("t0,t1,c0,c1,pairs", [
     (64, 8016, 2004, 16, 74),   # batch-1 backward: 64 dX tiles (K=128256), 8016 dW tiles (K=1024)
+    (32, 4008, 4008, 32, 74),   # the same at 512-wide tiles (k-steps counted per N=256 MMA group)
+    (32, 4752, 4752, 32, 74),   # V=152064, H=4000 at 512 wide
     (64, 9504, 2376, 16, 74),   # V=152064, H=4000
     (64, 8016, 2004, 16, 70),   # fewer resident pairs than SM pairs
     (4, 9504, 2376, 4, 74),     # 256-row chunk
@@ -64,3 +66,17 @@ def test_pick_tile_rejects_bad_input():
     assert pl.pl_debug_pick_tile([(1, 1, 1)] * 3, 74) == -1
     assert pl.pl_debug_pick_tile([(0, 512, 64)], 74) == -1
     assert pl.pl_debug_pick_tile([(256, 512, 64)], 0) == -1
+
+
+def test_wide_backward_schedule_is_within_one_short_tile_of_its_longest_tile():
+    # at 512-wide tiles a dX tile (4008 units) exceeds the fair share (about 3466): the
+    # makespan cannot go below one dX tile, and the schedule stays within one dW tile of it
+    t0, t1, c0, c1, pairs = 32, 4008, 4008, 32, 74
+    rc, owner = pl.pl_debug_pair_tiles(t0, t1, c0, c1, pairs)
+    assert rc == 0
+    per = [0] * pairs
+    for t, q in enumerate(owner):
+        per[q] += c0 if t < t0 else c1
+    assert max(per) <= c0 + c1
+    rest = per[t0:]
+    assert max(rest) - min(rest) <= c1
