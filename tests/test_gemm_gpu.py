@@ -5,7 +5,6 @@ and ragged shapes (M, N, K not multiples of the 128 x 256 x 64 tiling).
 Tolerance: |D - ref| <= 1e-5 * sum_k |A(m,k) B(n,k)| + 1e-6 (fp32 accumulation
 of exactly representable 16-bit products).
 """
-import numpy as np
 import pytest
 import torch
 

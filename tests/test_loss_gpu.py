@@ -10,8 +10,6 @@ A token whose oracle ratio lies within 8 fp32 ulps of the clip bound 1+eps_hi ma
 take either side of the min() in fp32 (both sides are correct), so its gradient
 is left out of the element-wise comparison.
 """
-import math
-
 import numpy as np
 import pytest
 import torch

@@ -50,7 +50,6 @@ def test_prefetcher_guards():
 
 def test_graphed_fused_step_matches_eager_calls():
     # the tiny fused workload: count, two GEMM launches, combine, dlogits, finalize in one graph
-    import numpy as np
     import rl_post_policy_b200 as pl
     from rl_post_policy_b200.pipeline import GraphedCall
     import synth
