@@ -44,8 +44,10 @@ pl_status pl_debug_gemm_out(const void* A, int a_mn, int64_t lda, const void* B,
  * launches is bracketed by a pair of CUDA events recorded on the launching
  * stream.  pl_debug_timing_read() waits for the recorded events, returns per
  * kind the summed device milliseconds and launch counts, and clears them.
- * Kinds: 0 = GEMM (tcgen05 kernel), 1 = loss-only kernel, 2 = other kernels of
- * the fused path (counts, combine, dlogits, finalize).  Arrays have 3 entries.
+ * Kinds: 0 = GEMM (tcgen05 kernel), 1 = loss-only kernels (cooperative and
+ * small-batch), 2 = every other kernel (the fused path's counts, combine,
+ * dlogits, convert and finalize; reverse KL; scale and count ratio).  Arrays
+ * have 3 entries.
  * Not thread-safe; meant for one benchmarking thread.
  */
 void pl_debug_timing(int enable);
