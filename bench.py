@@ -36,8 +36,12 @@ METRIC = "fused GRPO fwd+bwd tokens/s and % of B200 BF16 tensor peak; loss-only 
 # Published CuTe-DSL latency at batch 1, T=1024, H=4096, V=128256, BF16 on B200
 # ("Add SM100 CuTe DSL GRPO fast path", "B200 results" table).
 PUBLISHED_MS = {1: 6.69, 2: 12.09, 4: 23.07, 8: 43.79}
+# Used only when MEASURED_PEAKS.json is absent: an earlier measurement on B200s of
+# this kind -- copy bandwidth 6.65 TB/s, bf16 GEMM 1.59 PFLOP/s in a burst, settling
+# near 1.4 PFLOP/s (at about 1.3 GHz) when run for seconds under the 1 kW power cap.
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 EPS_LO, EPS_HI = 0.2, 0.28
+GRPO = 1  # the reduction bit of the library's mode word
 GEMM_SOURCES = ["rl_post_policy_b200/csrc/gemm_tc.cu", "rl_post_policy_b200/csrc/sm100.cuh",
                 "rl_post_policy_b200/csrc/gemm.h"]
 LOSS_SOURCES = ["rl_post_policy_b200/csrc/loss_kernel.cu", "rl_post_policy_b200/csrc/policy_math.cuh"]
@@ -51,15 +55,20 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5])
-    ap.add_argument("--chunk-rows", type=int, default=-1,
-                    help="rows per chunk (multiple of 128); -1: the whole batch in one chunk")
+    ap.add_argument("--chunk-rows", type=int, default=1024,
+                    help="rows per chunk (multiple of 128; the pages' 1024 by default); -1: the whole "
+                         "batch in one chunk")
     ap.add_argument("--no-loss-only", action="store_true")
     ap.add_argument("--no-reverse-kl", action="store_true")
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip the temperature and selective log-prob measurements")
-    ap.add_argument("--only", choices=["reverse_kl", "loss_only", "loss_matrix"], default=None,
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other fused workloads (3, 4a, 4b) and the loss-only variants")
+    ap.add_argument("--config-steps", type=int, default=10, help="timed steps per other fused workload")
+    ap.add_argument("--only", choices=["reverse_kl", "loss_only", "loss_matrix", "configs"], default=None,
                     help="run one side measurement alone and print its JSON (for profiling); loss_matrix: "
-                         "the loss kernel's 24 variants at bs=16 x 1024 and its bandwidth sweep, L2 flushed")
+                         "the loss kernel's 24 variants at bs=16 x 1024 and its bandwidth sweep, L2 flushed; "
+                         "configs: the other fused workloads and the loss-only variants")
     ap.add_argument("--reps", type=int, default=30, help="timed calls per side measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256, help="rows in the oracle's timed sample")
@@ -104,6 +113,11 @@ def dist_init(args):
     if ws > 1:
         import datetime
         import torch.distributed as dist
+        # NCCL's communicator set-up lines (rank count, devices, channels) on stderr,
+        # so a run's log shows how many ranks took part
+        os.environ.setdefault("NCCL_DEBUG", "INFO")
+        os.environ.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
+        os.environ.setdefault("NCCL_DEBUG_FILE", "/dev/stderr")
         backend = "nccl" if torch.cuda.is_available() else "gloo"
         if torch.cuda.is_available():
             torch.cuda.set_device(local)
@@ -139,19 +153,39 @@ def sum_over_ranks(x: float, ws: int) -> float:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi sampling every 100 ms; stop() keeps the samples whose
-    timestamps fall inside the timed window (mark_start / mark_end)."""
-    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """The SM clock and the active clock-event reasons, read through NVML every
+    2 ms on a background thread while the GPU works (nvidia-smi every 100 ms
+    where NVML is not available).  stop() keeps the samples taken between
+    mark_start() and mark_end(), so a timed region of tens of milliseconds still
+    gets a median of many readings."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+    SMI_FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device: int):
-        self.proc = None
+    def __init__(self, device: int, period_s: float = 0.002):
+        self.period = period_s
+        self.samples = []  # (time.time(), sm MHz, reason bits)
+        self.t0 = self.t1 = None
+        self.thread = self.proc = self.nvml = None
+        self.max_mhz = None
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
-            self.sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         except Exception:
-            self.sel = None
+            self.uuid = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = (pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid
+                           else pynvml.nvmlDeviceGetHandleByIndex(device))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            get = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+            self.get_reasons = get or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:
+            self.nvml = None
 
     def mark_start(self):
         self.t0 = time.time()
@@ -159,19 +193,35 @@ class ClockSampler:
     def mark_end(self):
         self.t1 = time.time()
 
+    def _loop(self):
+        import threading  # noqa: F401
+        nv, h = self.nvml, self.handle
+        while not self._stop:
+            try:
+                self.samples.append((time.time(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                     int(self.get_reasons(h))))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
     def start(self):
         self.t0 = self.t1 = None
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
-        if self.sel:
-            cmd += ["-i", self.sel]
+        self.samples = []
+        if self.nvml is not None:
+            import threading
+            self._stop = False
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+            return
+        cmd = ["nvidia-smi", f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
 
-    def stop(self) -> dict:
-        if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+    def _smi_samples(self):
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
@@ -179,30 +229,59 @@ class ClockSampler:
             self.proc.kill()
             out, _ = self.proc.communicate()
         import datetime
-        sm, mx, reasons, total = [], None, set(), 0
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
-            total += 1
             try:
                 ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-            except ValueError:
-                ts = None
-            if self.t0 is not None and ts is not None and not (self.t0 <= ts <= (self.t1 or ts)):
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                mhz = float(f[1])
+                self.max_mhz = float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            bits = 0
+            for (name, bit), v in zip(self.REASONS, f[5:9]):
                 if v.lower().startswith("active"):
-                    reasons.add(n)
-        load = [x for x in sm if mx and x > 0.3 * mx] or sm
-        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm), "samples_total": total}
+                    bits |= bit
+            self.samples.append((ts, mhz, bits))
+
+    def stop(self) -> dict:
+        if self.thread is not None:
+            self._stop = True
+            self.thread.join(timeout=5)
+            self.thread = None
+            source = f"NVML every {self.period * 1e3:.0f} ms"
+        elif self.proc is not None:
+            self._smi_samples()
+            self.proc = None
+            source = "nvidia-smi every 100 ms"
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"], "samples": 0}
+        total = len(self.samples)
+        win = [x for x in self.samples
+               if (self.t0 is None or x[0] >= self.t0) and (self.t1 is None or x[0] <= self.t1)]
+        sm = [x[1] for x in win]
+        bits = 0
+        for x in win:
+            bits |= x[2]
+        reasons = sorted(name for name, bit in self.REASONS if bits & bit)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(sm) if sm else None, "reasons": reasons, "samples": len(sm),
+                "samples_total": total, "source": source}
+
+
+def peak_for(peaks, peak_kind, timed_s, dtype):
+    """The dense tensor peak a GEMM is held to: the measured burst figure for a
+    timed region shorter than 2 s (the clock has not yet settled under the power
+    cap), the sustained one for longer regions.  fp16 takes the bf16 figure
+    (nominal ratio 1:1)."""
+    sustained = timed_s >= 2.0
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    peak = float(peaks.get(key, peaks["bf16_tflops"]))
+    regime = (f"{'sustained' if sustained else 'burst'}: timed region {timed_s:.2f} s "
+              f"({'>=' if sustained else '<'} 2 s)")
+    note = f"{peak_kind} {key}" + (" x 1.0 (fp16 nominal ratio 1:1)" if dtype == torch.float16 else "")
+    return peak, f"{note}; {regime}"
 
 
 # ------------------------------------------------------------------ workload
@@ -230,19 +309,23 @@ def chunk_mode(N: int, chunk_rows: int) -> int:
 def arm_config(d: dict, chunk_rows: int, ws_world: int) -> dict:
     """The workload named in both arms' JSON lines."""
     N = d["bs"] * d["T"]
+    par = (f"dp{ws_world}: one batch of {ws_world} x {N} rows sharded by sequences, dW/dbias/loss all-reduced"
+           if ws_world > 1 else "dp1")
     return {"workload": f"fused GRPO fwd+bwd, bs={d['bs']} x T={d['T']} (N={N}), H={d['H']}, V={d['V']}, "
                         f"beta={d['beta']}, GRPO, eps=0.2/0.28",
             "per_gpu_rows": N, "chunk_rows": chunk_rows,
             "l2": "inputs larger than L2 (W and Wref are 1 GB each); no flush",
-            "parallelism": f"dp{ws_world} (independent batches)"}
+            "parallelism": par}
 
 
-def make_fused_inputs(w: int, rank: int, chunk_rows: int = -1):
+def make_fused_inputs(w: int, rank: int, chunk_rows: int = -1, beta=None):
     """Synthetic inputs on the GPU; old_lp = policy log-prob (from a forward-only
-    call of the same entry point) + N(0, 0.1)."""
+    call of the same entry point) + N(0, 0.1).  `beta` overrides the workload's."""
     import rl_post_policy_b200 as pl
     import synth
     d = workload_desc(w)
+    if beta is not None:
+        d["beta"] = beta
     inp = synth.fused_inputs(d["bs"], d["T"], d["H"], d["V"], d["dtype"], synth.seed_for(w, rank),
                              bias=d.get("bias", False), len_lo=d["len_lo"], len_hi=d["len_hi"],
                              fully_masked_last=d.get("fully_masked_last", False), device="cuda")
@@ -282,6 +365,40 @@ class FusedStep:
             None, self.ws, self.wsb)
         if rc != 0:
             raise RuntimeError(f"pl_fused_linear_grpo: {self.pl.pl_status_string(rc)}")
+
+
+class DataParallelStep:
+    """One data-parallel step of the fused path (the multi-GPU partitioning the
+    path has): this rank's sequences of one global batch through
+    parallel.dp_fused_linear_grpo -- the rank's fused forward + backward
+    normalised by its own count, the all-reduce of the count, the rank's share
+    applied on the device, and the all-reduce of the loss, dW and dbias.  `ops`
+    replaces the library's per-rank operations (CPU tests)."""
+
+    def __init__(self, d, inp, chunk_rows=None, ops=None, group=None):
+        from rl_post_policy_b200 import parallel
+        self.parallel, self.d, self.inp, self.ops, self.group = parallel, d, inp, ops, group
+        self.chunk_rows = chunk_rows
+        self.out = None
+
+    def __call__(self):
+        i, d = self.inp, self.d
+        self.out = self.parallel.dp_fused_linear_grpo(
+            i["X"], i["W"], i["bias"], i["targets"], i["Xref"] if d["beta"] else None,
+            i["Wref"] if d["beta"] else None, i["old_lp"], i["adv"], i["mask"], eps_lo=EPS_LO, eps_hi=EPS_HI,
+            beta=d["beta"], reduction=GRPO, chunk_rows=self.chunk_rows, group=self.group, ops=self.ops)
+        return self.out
+
+
+def broadcast_weights(inp, ws_world):
+    """Rank 0's W, Wref and bias on every rank: the data-parallel step holds one
+    replica of the weights per rank (each rank draws its own rows)."""
+    if ws_world == 1:
+        return
+    import torch.distributed as dist
+    for k in ("W", "Wref", "bias"):
+        if inp.get(k) is not None:
+            dist.broadcast(inp[k], src=0)
 
 
 def time_steps(fn, steps, ws_world):
@@ -364,7 +481,7 @@ def loss_only(peaks, peak_kind):
     }
 
 
-def loss_matrix(peaks, peak_kind, reps=20):
+def loss_matrix(peaks, peak_kind, reps=20, sweep=True):
     """The loss kernel over its variants: BNPO/GRPO x beta in {0.04, 0} x fwd+bwd / fwd-only x
     bf16/fp16/fp32 at bs=16 x seq=1024 (launch-latency bound: about 144 KB per call in bf16), and
     a bandwidth sweep of bf16 BNPO fwd+bwd, beta=0.04, bs=16 x seq=2^18 ... 2^23.  A 256 MB buffer
@@ -418,19 +535,22 @@ def loss_matrix(peaks, peak_kind, reps=20):
             for beta in (0.04, 0.0):
                 for grad in (True, False):
                     variants.append(one(16, 1024, dt, red, beta, grad, inp32))
-    sweep = []
-    for k in range(18, 24):
+    sweep_pts = []
+    for k in (range(18, 24) if sweep else ()):
         seq = 1 << k
         inp = synth.loss_inputs(16, seq, torch.float32, synth.seed_for(1, 1), len_lo=64, len_hi=seq, device="cuda")
-        sweep.append(one(16, seq, torch.bfloat16, pl.PL_BNPO, 0.04, True, inp))
+        sweep_pts.append(one(16, seq, torch.bfloat16, pl.PL_BNPO, 0.04, True, inp))
         del inp
-    return {"metric": "loss kernel variants and bandwidth sweep", "peak_GB_per_s": peak,
-            "peak_source": f"{peak_kind} hbm_gbs", "l2": "256 MB written between calls",
-            "variants_bs16_seq1024": variants, "sweep_bf16_bnpo_beta0.04": sweep}
+    out = {"metric": "loss kernel variants and bandwidth sweep", "peak_GB_per_s": peak,
+           "peak_source": f"{peak_kind} hbm_gbs", "l2": "256 MB written between calls",
+           "variants_bs16_seq1024": variants}
+    if sweep:
+        out["sweep_bf16_bnpo_beta0.04"] = sweep_pts
+    return out
 
 
 # ------------------------------------------------------------------ temperature, selective log-prob
-def next_rows(d, inp, ws, wsb, mode, peak, reps=20):
+def next_rows(d, inp, ws, wsb, mode, peaks, peak_kind, reps=20):
     """The fused step at temperature 0.7 (pl_fused_linear_grpo_temp) and the fused
     selective log-prob forward + backward with an external dL/dlogp
     (pl_fused_selective_logprob), on the benchmarked workload's tensors, CUDA
@@ -451,12 +571,14 @@ def next_rows(d, inp, ws, wsb, mode, peak, reps=20):
         torch.cuda.synchronize()
         pl.pl_debug_timing_read()
         pl.pl_debug_timing(True)
+        t0 = time.perf_counter()
         for _ in range(reps):
             call()
         torch.cuda.synchronize()
+        span = time.perf_counter() - t0
         pl.pl_debug_timing(False)
         ms, _ = pl.pl_debug_timing_read()
-        return sum(ms) / reps
+        return sum(ms) / reps, span
 
     def temp_call():
         pl.check(pl.pl_fused_linear_grpo_temp(inp["X"], inp["W"], inp["bias"], inp["targets"], inp["Xref"],
@@ -464,7 +586,7 @@ def next_rows(d, inp, ws, wsb, mode, peak, reps=20):
                                               EPS_LO, EPS_HI, d["beta"], 0.7, mode, loss, dX, dW, db, None, None,
                                               None, ws, wsb), "pl_fused_linear_grpo_temp")
 
-    t_ms = timed(temp_call)
+    t_ms, t_span = timed(temp_call)
     smode = pl.dtype_mode(dt) | (mode & (0xFF << pl.PL_CHUNK_SHIFT))
     swsb = pl.pl_fused_selective_logprob_workspace_bytes(N, H, V, smode, 1, int(db is not None))
     sws = torch.zeros(swsb, dtype=torch.uint8, device="cuda")
@@ -474,16 +596,20 @@ def next_rows(d, inp, ws, wsb, mode, peak, reps=20):
         pl.check(pl.pl_fused_selective_logprob(inp["X"], inp["W"], inp["bias"], inp["targets"], N, H, V, smode, g,
                                                lp, dX, dW, db, sws, swsb), "pl_fused_selective_logprob")
 
-    s_ms = timed(sel_call)
+    s_ms, s_span = timed(sel_call)
     del sws, dX, dW
     f_temp, f_sel = 8.0 * N * H * V, 6.0 * N * H * V
+    t_peak, t_src = peak_for(peaks, peak_kind, t_span, dt)
+    s_peak, s_src = peak_for(peaks, peak_kind, s_span, dt)
     return {
         "temperature": {"workload": f"fused GRPO fwd+bwd at temperature 0.7, N={N}, H={H}, V={V}",
                         "ms": t_ms, "tokens_per_s": N / (t_ms * 1e-3), "tflops": f_temp / (t_ms * 1e-3) / 1e12,
-                        "frac_of_peak": f_temp / (t_ms * 1e-3) / 1e12 / peak},
+                        "frac_of_peak": f_temp / (t_ms * 1e-3) / 1e12 / t_peak, "peak": t_peak,
+                        "peak_source": t_src},
         "selective_logprob": {"workload": f"fused selective log-prob fwd + bwd (dX, dW), N={N}, H={H}, V={V}",
                               "ms": s_ms, "tokens_per_s": N / (s_ms * 1e-3), "tflops": f_sel / (s_ms * 1e-3) / 1e12,
-                              "frac_of_peak": f_sel / (s_ms * 1e-3) / 1e12 / peak},
+                              "frac_of_peak": f_sel / (s_ms * 1e-3) / 1e12 / s_peak, "peak": s_peak,
+                              "peak_source": s_src},
     }
 
 
@@ -600,6 +726,98 @@ def run_reference(args):
     }), flush=True)
 
 
+def fused_roofline(d, steps, kms, kn, ms_per_step, timed_s, peaks, peak_kind):
+    """Roofline of the dominant kernel (the tcgen05 GEMM) over a timed region:
+    algorithmic flops per GEMM launch over the mean launch time (CUDA events on
+    the launching stream), against the dense tensor peak for the region's length,
+    with the fractions of both measured peaks beside it."""
+    N, H, V = d["N"], d["H"], d["V"]
+    flops_step = (8 if d["beta"] != 0 else 6) * N * H * V
+    gemm_ms = kms[0] / max(kn[0], 1)
+    gemm_flops_launch = flops_step * steps / max(kn[0], 1)
+    achieved = gemm_flops_launch / (gemm_ms * 1e-3) / 1e12
+    peak, src = peak_for(peaks, peak_kind, timed_s, d["dtype"])
+    step_tflops = flops_step / (ms_per_step * 1e-3) / 1e12
+    burst = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained", burst))
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": src, "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
+            "kernel": "gemm_kernel (tcgen05 persistent GEMM)", "launch_ms": gemm_ms, "launches": kn[0],
+            "flops_per_step": flops_step, "share_of_step": kms[0] / max(sum(kms), 1e-9),
+            "step_tflops": step_tflops, "step_frac_of_peak": step_tflops / peak,
+            "step_frac_of_burst": step_tflops / burst, "step_frac_of_sustained": step_tflops / sustained}
+
+
+def measure_fused(w, chunk_rows, steps, warmup, peaks, peak_kind, beta=None):
+    """One fused workload at one chunk size: `warmup` untimed steps, then `steps`
+    timed with CUDA events (and the GEMM launches with their own events), with
+    the SM clock sampled inside the timed region."""
+    import rl_post_policy_b200 as pl
+    d, inp, ws, wsb, mode = make_fused_inputs(w, 0, chunk_rows, beta)
+    step = FusedStep(d, inp, ws, wsb, mode)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    pl.check(pl.pl_device_status(ws), "device status after warm-up")
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    pl.pl_debug_timing_read()
+    pl.pl_debug_timing(True)
+    clocks.mark_start()
+    t0 = time.perf_counter()
+    elapsed = time_steps(step, steps, 1)
+    span = time.perf_counter() - t0
+    clocks.mark_end()
+    pl.pl_debug_timing(False)
+    clk = clocks.stop()
+    kms, kn = pl.pl_debug_timing_read()
+    pl.check(pl.pl_device_status(ws), "device status after timing")
+    ms = elapsed / steps
+    N = d["N"]
+    rl = fused_roofline(d, steps, kms, kn, ms, span, peaks, peak_kind)
+    out = {"chunk_rows": d["chunk_rows"], "chunks": (N + d["chunk_rows"] - 1) // d["chunk_rows"],
+           "steps": steps, "ms": ms, "tokens_per_s": N / (ms * 1e-3), "tflops": rl["step_tflops"],
+           "frac_of_burst": rl["step_frac_of_burst"], "frac_of_sustained": rl["step_frac_of_sustained"],
+           "gemm_tflops": rl["achieved"], "gemm_frac_of_burst": rl["frac_of_burst"],
+           "gemm_ms_per_step": kms[0] / steps, "other_kernels_ms_per_step": (kms[1] + kms[2]) / steps,
+           "clocks": clk}
+    if clk.get("sm_mhz"):
+        out["ms_x_sm_ghz"] = ms * clk["sm_mhz"] / 1e3
+    del step, inp, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+# The other fused workloads: name -> (workload number, beta).  Numbers as in synth.WORKLOADS.
+OTHER_CONFIGS = {
+    "w3_fp16_bias_bs4_T1024_H4096_V128256_beta0.04": (3, 0.04),
+    "w4a_bf16_bs8_T1024_H4096_V128256_beta0.04": (4, 0.04),
+    "w4a_bf16_bs8_T1024_H4096_V128256_beta0": (4, 0.0),
+    "w4b_bf16_bs8_T1024_H4000_V152064_beta0.04": (5, 0.04),
+    "w4b_bf16_bs8_T1024_H4000_V152064_beta0": (5, 0.0),
+}
+
+
+def other_configs(peaks, peak_kind, steps):
+    """Every other fused workload at the pages' 1024-row chunks and with one
+    chunk spanning the batch, plus the loss-only kernel's 24 variants at
+    bs=16 x 1024 (the launch-bound loss workload)."""
+    import synth
+    out = {}
+    for name, (w, beta) in OTHER_CONFIGS.items():
+        d = synth.WORKLOADS[w]
+        N = d["bs"] * d["T"]
+        out[name] = {"workload": f"fused GRPO fwd+bwd, bs={d['bs']} x T={d['T']} (N={N}), H={d['H']}, "
+                                 f"V={d['V']}, {str(d['dtype']).split('.')[-1]}, beta={beta}"
+                                 + (", policy bias" if d.get("bias") else "")
+                                 + (", last sequence fully masked" if d.get("fully_masked_last") else ""),
+                     "flops_per_step": (8 if beta else 6) * N * d["H"] * d["V"],
+                     "chunked_1024": measure_fused(w, 1024, steps, 2, peaks, peak_kind, beta),
+                     "whole_batch": measure_fused(w, -1, steps, 2, peaks, peak_kind, beta)}
+    out["w1_loss_only_variants_bs16_seq1024"] = loss_matrix(peaks, peak_kind, sweep=False)
+    return out
+
+
 def run_ours(args):
     ws_world, rank = dist_init(args)
     import rl_post_policy_b200 as pl
@@ -610,13 +828,21 @@ def run_ours(args):
                 out = reverse_kl(peaks, peak_kind, args.reps)
             elif args.only == "loss_matrix":
                 out = loss_matrix(peaks, peak_kind)
+            elif args.only == "configs":
+                out = other_configs(peaks, peak_kind, args.config_steps)
             else:
                 out = loss_only(peaks, peak_kind)
             print(json.dumps(out), flush=True)
         return
     d, inp, ws, wsb, mode = make_fused_inputs(args.workload, rank, args.chunk_rows)
-    step = FusedStep(d, inp, ws, wsb, mode)
     N, H, V = d["N"], d["H"], d["V"]
+    single = FusedStep(d, inp, ws, wsb, mode)
+    if ws_world > 1:
+        # one global batch sharded by sequences: the same weights on every rank
+        broadcast_weights(inp, ws_world)
+        step = DataParallelStep(d, inp, chunk_rows=d["chunk_rows"])
+    else:
+        step = single
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -627,40 +853,30 @@ def run_ours(args):
     pl.pl_debug_timing_read()
     launches0 = pl.pl_debug_launch_count()
     clocks.start()
-    for _ in range(max(1, args.warmup)):  # keep the GPU busy while the sampler starts
-        step()
-    time.sleep(0.3)
     pl.pl_debug_timing(True)
     clocks.mark_start()
+    t0 = time.perf_counter()
     elapsed = time_steps(step, args.steps, ws_world)
+    span = time.perf_counter() - t0
     clocks.mark_end()
     pl.pl_debug_timing(False)
     clk = clocks.stop()
     launches = pl.pl_debug_launch_count() - launches0
     kms, kn = pl.pl_debug_timing_read()
     pl.check(pl.pl_device_status(ws), "device status after timing")
+    if ws_world > 1:
+        from rl_post_policy_b200 import parallel
+        for w in parallel._default_ops()._ws.values():
+            pl.check(pl.pl_device_status(w), "device status of the data-parallel step")
     t_max = max_over_ranks(elapsed, ws_world)
     ms_per_step = t_max / args.steps
     total_tokens = sum_over_ranks(float(N * args.steps), ws_world)
     value = total_tokens / (t_max * 1e-3)
-
-    # ---- roofline of the dominant kernel (the tcgen05 GEMM) ----
-    flops_step = (8 if d["beta"] != 0 else 6) * N * H * V
-    gemm_ms = kms[0] / max(kn[0], 1)
-    gemm_flops_launch = flops_step * args.steps / max(kn[0], 1)
-    achieved = gemm_flops_launch / (gemm_ms * 1e-3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-    if d["dtype"] == torch.float16:
-        peak_note = f"{peak_kind} bf16 sustained x 1.0 (fp16 nominal ratio 1:1)"
-    else:
-        peak_note = f"{peak_kind} bf16 sustained (the GEMMs run back to back for seconds)"
-    step_tflops = flops_step / (ms_per_step * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": recorded_traffic("gemm_kernel", GEMM_SOURCES),
-                "kernel": "gemm_kernel (tcgen05 persistent GEMM)", "peak_source": peak_note,
-                "launch_ms": gemm_ms, "launches": kn[0],
-                "share_of_step": kms[0] / max(sum(kms), 1e-9),
-                "step_tflops": step_tflops, "step_frac_of_peak": step_tflops / peak}
+    roofline = fused_roofline(d, args.steps, kms, kn, ms_per_step, max_over_ranks(span, ws_world), peaks,
+                              peak_kind)
+    roofline["traffic"] = recorded_traffic("gemm_kernel", GEMM_SOURCES)
+    if clk.get("sm_mhz"):
+        roofline["gemm_ms_x_sm_ghz"] = roofline["launch_ms"] * clk["sm_mhz"] / 1e3
 
     # ---- end to end through the C ABI from pinned host buffers ----
     # Every step copies its inputs from pinned host memory (on a copy stream, one
@@ -678,16 +894,31 @@ def run_ours(args):
             dev = pf.next()
             if i + 1 < steps:
                 pf.prefetch(host)
-            step(**dev)
-            loss_host.copy_(step.loss, non_blocking=True)
+            if ws_world > 1:
+                step.inp = dict(inp, **dev)
+                step()
+                loss_host.copy_(step.out["loss"], non_blocking=True)
+            else:
+                step(**dev)
+                loss_host.copy_(step.loss, non_blocking=True)
             pf.release()
         pf.finish()
 
     e2e_run(2)
     e2e_ms = max_over_ranks(time_steps(lambda: e2e_run(args.steps), 1, ws_world), ws_world) / args.steps
     e2e_val = total_tokens / args.steps / (e2e_ms * 1e-3)
+    if ws_world > 1:
+        step.inp = inp
 
     extra = {}
+    if ws_world > 1:
+        # the same step with no collective: each rank's own batch (weak scaling, independent batches)
+        for _ in range(2):
+            single()
+        ind = max_over_ranks(time_steps(single, args.steps, ws_world), ws_world)
+        extra["independent_batches"] = {
+            "what": "each rank runs its own batch, no collective", "ms_per_step": ind / args.steps,
+            "value": total_tokens / (ind * 1e-3), "unit": "tokens/s"}
 
     def side(fn, *fargs):
         # The bandwidth-bound side measurements come after seconds of power-capped
@@ -697,7 +928,6 @@ def run_ours(args):
         time.sleep(2.0)
         cs = ClockSampler(torch.cuda.current_device())
         cs.start()
-        time.sleep(0.3)
         out = fn(*fargs)
         torch.cuda.synchronize()
         out["clocks"] = cs.stop()
@@ -708,7 +938,7 @@ def run_ours(args):
     if rank == 0 and ws_world == 1 and not args.no_reverse_kl:
         extra["reverse_kl"] = side(reverse_kl, peaks, peak_kind, args.reps)
     if rank == 0 and ws_world == 1 and not args.no_next_rows:
-        extra.update(next_rows(d, inp, ws, wsb, mode, float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))))
+        extra.update(next_rows(d, inp, ws, wsb, mode, peaks, peak_kind))
     cpu = None
     if rank == 0 and ws_world == 1 and not args.no_cpu_baseline:
         rows = max(1, min(args.cpu_rows, N))
@@ -716,6 +946,10 @@ def run_ours(args):
         cpu = {"value": rows / secs, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"first {rows} rows of the batch as one sequence: policy+reference forward over "
                          f"V={V}, GRPO loss, dX/dW/dbias, fp64 ({secs:.1f} s)"}
+    if rank == 0 and ws_world == 1 and not args.no_configs:
+        del single, step, ws
+        torch.cuda.empty_cache()
+        extra["configs"] = other_configs(peaks, peak_kind, args.config_steps)
 
     if rank == 0:
         bsz = d["bs"]

@@ -158,9 +158,11 @@ size_t pl_loss_workspace_bytes(int64_t bs, int64_t seq);
  *                (0 = none, 1 = a bounded wait ran out) and clears them.  With
  *                NULL, the bits accumulate until a call passes status_out.
  * The first call on each device looks up the array's device address (with that
- * device current), so make it before any stream capture.  Every call shares the
- * one array and resets the counters it needs on `stream` before its kernel:
- * calls whose work overlaps on the GPU race, so order them on one stream.
+ * device current), so make it before any stream capture.  The address is cached
+ * per device and context; after a cudaDeviceReset the next call looks it up
+ * again (and should again come before any capture).  Every call shares the one
+ * array and resets the counters it needs on `stream` before its kernel: calls
+ * whose work overlaps on the GPU race, so order them on one stream.
  */
 pl_status pl_loss_static(const void* policy_lp, const void* old_lp, const void* ref_lp,
                          const void* adv, const uint8_t* mask, int64_t bs, int64_t seq,

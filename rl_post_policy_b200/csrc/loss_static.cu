@@ -7,10 +7,15 @@
 // kStaticMaxBs.  Every GPU that loads libpl.so holds this array until the
 // process exits.  Host code cannot use the array's name as a device address,
 // so the first call on each device looks the address up with
-// cudaGetSymbolAddress (with that device current) and caches it; that first
-// call should therefore come before any stream capture.  All calls share the
+// cudaGetSymbolAddress (with that device current) and caches it, keyed by the
+// device and its current context; that first call should therefore come before
+// any stream capture.  A device reset (cudaDeviceReset) gives the device a new
+// context in which the module is loaded again, so the next call after it looks
+// the address up again rather than reusing the old one.  All calls share the
 // one array: calls whose work overlaps on the GPU race with each other, so
 // issue them on one stream (or otherwise order them).
+#include <cuda.h>
+
 #include <mutex>
 
 #include "internal.h"
@@ -27,17 +32,40 @@ static __device__ __align__(256) unsigned char g_loss_scratch[kStaticScratchByte
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_addr[kMaxDevices] = {};
+CUcontext g_ctx[kMaxDevices] = {};
 
-// Device address of g_loss_scratch on the current device (looked up once per device).
+// The current context through the driver entry point the runtime hands out
+// (the library does not link the driver library itself).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  }
+  return fn;
+}
+
+// Device address of g_loss_scratch on the current device, looked up once per
+// device and context.
 pl_status scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return PL_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return PL_ERR_CUDA;
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  CUcontext ctx = nullptr;
+  if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) return PL_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
+  if (!ctx || !g_addr[dev] || g_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_loss_scratch) != cudaSuccess || !p) return PL_ERR_CUDA;
+    // the lookup makes the device's primary context current if nothing had yet
+    if (!ctx && (get_ctx(&ctx) != CUDA_SUCCESS || !ctx)) return PL_ERR_CUDA;
     g_addr[dev] = p;
+    g_ctx[dev] = ctx;
   }
   *out = g_addr[dev];
   return PL_OK;

@@ -60,27 +60,41 @@ def _rel(a, b):
     return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
 
 
-@pytest.mark.parametrize("workload", [2, 3, 4, 5])
-def test_full_size(workload):
-    d = dict(synth.WORKLOADS[workload])
-    if workload == 5:
-        d["beta"] = 0.0  # the batch-8 shapes are run at beta=0.04 (H=4096) and beta=0 (H=4000)
-    bs, T, H, V = d["bs"], d["T"], d["H"], d["V"]
-    N = bs * T
-    inp = synth.fused_inputs(bs, T, H, V, d["dtype"], synth.seed_for(workload), bias=d.get("bias", False),
-                             len_lo=d["len_lo"], len_hi=d["len_hi"],
-                             fully_masked_last=d.get("fully_masked_last", False), need_ref=d["beta"] != 0)
-    lse, logp, _ = oracle.lm_head_logprob(inp["X"], inp["W"], inp["bias"], inp["targets"])
-    inp["old_lp"] = (torch.from_numpy(logp) + inp["old_noise"].double()).float()
-    ref_logp = None
-    if d["beta"] != 0:
-        _, ref_logp, _ = oracle.lm_head_logprob(inp["Xref"], inp["Wref"], None, inp["targets"])
+_ORACLE_CACHE = {}
 
-    runs = [_run(inp, d)]
+
+def _inputs(workload, need_ref):
+    """The workload's inputs and the oracle's policy (and, on request, reference)
+    log-probs, computed once per workload and shared by its beta variants."""
+    if workload not in _ORACLE_CACHE:
+        d = synth.WORKLOADS[workload]
+        inp = synth.fused_inputs(d["bs"], d["T"], d["H"], d["V"], d["dtype"], synth.seed_for(workload),
+                                 bias=d.get("bias", False), len_lo=d["len_lo"], len_hi=d["len_hi"],
+                                 fully_masked_last=d.get("fully_masked_last", False), need_ref=True)
+        lse, logp, _ = oracle.lm_head_logprob(inp["X"], inp["W"], inp["bias"], inp["targets"])
+        inp["old_lp"] = (torch.from_numpy(logp) + inp["old_noise"].double()).float()
+        _ORACLE_CACHE.clear()  # one workload's tensors at a time
+        _ORACLE_CACHE[workload] = {"inp": inp, "lse": lse, "logp": logp, "ref_logp": None}
+    c = _ORACLE_CACHE[workload]
+    if need_ref and c["ref_logp"] is None:
+        _, c["ref_logp"], _ = oracle.lm_head_logprob(c["inp"]["Xref"], c["inp"]["Wref"], None,
+                                                     c["inp"]["targets"])
+    return c
+
+
+# Every fused workload at beta = 0.04; the batch-8 shapes (H=4096 / V=128256 and
+# H=4000 / V=152064) at beta = 0 as well, where the reference GEMM is skipped.
+@pytest.mark.parametrize("workload,beta", [(2, 0.04), (3, 0.04), (4, 0.04), (4, 0.0), (5, 0.04), (5, 0.0)])
+def test_full_size(workload, beta):
+    d = dict(synth.WORKLOADS[workload])
+    d["beta"] = beta
+    N = d["bs"] * d["T"]
+    c = _inputs(workload, beta != 0)
+    runs = [_run(c["inp"], d)]
     if N > 1024:  # also one chunk spanning the whole batch: dW as a single K = N GEMM
-        runs.append(_run(inp, d, chunk=N))
+        runs.append(_run(c["inp"], d, chunk=N))
     for got in runs:
-        _check(inp, d, got, workload, lse, logp, ref_logp)
+        _check(c["inp"], d, got, workload, c["lse"], c["logp"], c["ref_logp"] if beta != 0 else None)
 
 
 def _check(inp, d, got, workload, lse, logp, ref_logp):

@@ -368,3 +368,107 @@ def test_tempered_gradients_match_finite_differences(tau):
         m[v] -= h
         fdb[v] = (loss_with(bias=p) - loss_with(bias=m)) / (2 * h)
     np.testing.assert_allclose(base["dbias"], fdb, atol=1e-8, rtol=1e-5)
+
+
+# ---- row groups of at most four rows ----
+# The oracle's contractions take 32 rows per pass over a weight row and a short
+# branch for a group of at most 4 rows: every N <= 4, and the remainder group of
+# N = 33 and N = 36.  These pins reach that branch in the forward and in both
+# halves of the backward.
+SMALL_GROUP_N = [1, 2, 3, 4, 33, 36]
+
+
+def _longdouble_logits(X, W, b):
+    Xl = X.numpy().astype(np.longdouble)
+    Wl = W.numpy().astype(np.longdouble)
+    z = np.einsum("ih,vh->iv", Xl, Wl)  # a plain sum per element, no BLAS, in long double
+    return z + b.numpy().astype(np.longdouble)
+
+
+@pytest.mark.parametrize("N", SMALL_GROUP_N)
+def test_small_row_groups_logprob_against_brute_force(N):
+    g = torch.Generator().manual_seed(100 + N)
+    H, V = 24, 300
+    X = torch.randn(N, H, generator=g, dtype=torch.float64)
+    W = 0.3 * torch.randn(V, H, generator=g, dtype=torch.float64)
+    b = 0.1 * torch.randn(V, generator=g, dtype=torch.float64)
+    tg = torch.randint(0, V, (N,), generator=g)
+    lse, logp, zt = oracle.lm_head_logprob(X, W, b, tg)
+    z = _longdouble_logits(X, W, b)
+    brute = np.log(np.exp(z).sum(axis=1))
+    rows = np.arange(N)
+    np.testing.assert_allclose(lse, brute.astype(np.float64), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(zt, z[rows, tg.numpy()].astype(np.float64), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(logp, (z[rows, tg.numpy()] - brute).astype(np.float64), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("N", SMALL_GROUP_N)
+def test_small_row_groups_backward_against_brute_force(N):
+    # dz = g (onehot - softmax), dX = dz W, dW = dz^T X, dbias = column sums of dz,
+    # each written out element by element in long double
+    g = torch.Generator().manual_seed(200 + N)
+    H, V = 16, 90
+    X = torch.randn(N, H, generator=g, dtype=torch.float64)
+    W = 0.3 * torch.randn(V, H, generator=g, dtype=torch.float64)
+    b = 0.1 * torch.randn(V, generator=g, dtype=torch.float64)
+    tg = torch.randint(0, V, (N,), generator=g)
+    gv = torch.randn(N, generator=g, dtype=torch.float64).numpy()
+    if N > 2:
+        gv[N // 2] = 0.0  # a row with no gradient
+    z = _longdouble_logits(X, W, b)
+    lse = np.log(np.exp(z).sum(axis=1))
+    onehot = np.zeros((N, V), dtype=np.longdouble)
+    onehot[np.arange(N), tg.numpy()] = 1
+    dz = gv.astype(np.longdouble)[:, None] * (onehot - np.exp(z - lse[:, None]))
+    want_dX = np.einsum("iv,vh->ih", dz, W.numpy().astype(np.longdouble))
+    want_dW = np.einsum("iv,ih->vh", dz, X.numpy().astype(np.longdouble))
+    want_db = dz.sum(axis=0)
+    dx_rows = np.arange(N)[::-1].copy()  # any order: rows are gathered by index
+    dw_rows = np.array([0, 5, V - 1] + [int(t) for t in tg[:3]])
+    dX, dW, db = oracle.lm_head_backward(X, W, b, tg, lse.astype(np.float64), gv, dx_rows, dw_rows)
+    np.testing.assert_allclose(dX, want_dX[dx_rows].astype(np.float64), rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(dW, want_dW[dw_rows].astype(np.float64), rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(db, want_db[dw_rows].astype(np.float64), rtol=1e-11, atol=1e-14)
+
+
+@pytest.mark.parametrize("N", SMALL_GROUP_N)
+def test_small_row_groups_fused_gradients_match_finite_differences(N):
+    bs = {1: 1, 2: 1, 3: 1, 4: 2, 33: 3, 36: 4}[N]
+    T = N // bs
+    g = torch.Generator().manual_seed(300 + N)
+    H, V = 4, 6
+    X = torch.randn(N, H, generator=g, dtype=torch.float64)
+    W = 0.5 * torch.randn(V, H, generator=g, dtype=torch.float64)
+    bvec = 0.1 * torch.randn(V, generator=g, dtype=torch.float64)
+    Xr = X + 0.05 * torch.randn(N, H, generator=g, dtype=torch.float64)
+    Wr = W + 0.05 * torch.randn(V, H, generator=g, dtype=torch.float64)
+    tg = torch.randint(0, V, (N,), generator=g)
+    adv = torch.randn(bs, generator=g, dtype=torch.float64)
+    mask = torch.ones(bs, T, dtype=torch.int8)
+    if T > 1:
+        mask[0, T - 1] = 0
+    _, logp, _ = oracle.lm_head_logprob(X, W, bvec, tg)
+    old = torch.from_numpy(logp) + 0.2 * torch.randn(N, generator=g, dtype=torch.float64)
+    # keep every ratio clear of the kink at 1 + eps_hi (finite differences straddle it otherwise)
+    ln_hi = math.log(float(np.float32(1.0) + np.float32(EPS_HI)))
+    d = torch.from_numpy(logp) - old - ln_hi
+    old[d.abs() < 1e-3] -= 2e-3
+    inp = dict(X=X, W=W, bias=bvec, targets=tg, Xref=Xr, Wref=Wr, old_lp=old.reshape(bs, T), adv=adv, mask=mask)
+    kw = dict(eps_lo=EPS_LO, eps_hi=EPS_HI, beta=0.04, reduction=GRPO)
+    base = oracle.fused_grpo(**inp, **kw)
+
+    def loss_with(**over):
+        dd = dict(inp)
+        dd.update(over)
+        return oracle.fused_grpo(**dd, **kw, dx_rows=[], dw_rows=[])["loss"]
+
+    h = 1e-6
+    for name, grad in (("X", base["dX"]), ("W", base["dW"]), ("bias", base["dbias"])):
+        t = inp[name]
+        fd = np.zeros(tuple(t.shape))
+        for idx in np.ndindex(*t.shape):
+            p, m = t.clone(), t.clone()
+            p[idx] += h
+            m[idx] -= h
+            fd[idx] = (loss_with(**{name: p}) - loss_with(**{name: m})) / (2 * h)
+        np.testing.assert_allclose(grad, fd, atol=1e-8, rtol=1e-5, err_msg=name)

@@ -68,13 +68,26 @@ def test_one_rank_loss_step_equals_oracle(group, red, dtype):
     want = oracle.policy_loss(inp["policy_lp"], inp["old_lp"], inp["ref_lp"], inp["adv"], inp["mask"],
                               eps_lo=0.2, eps_hi=0.28, beta=0.04, reduction=red)
     tol = 1e-5 if dtype == torch.float32 else 1e-3
-    assert abs(out["loss"].item() - want["loss"]) <= tol * max(abs(want["loss"]), 1e-3 * want["abs_sum"])
-    w = torch.from_numpy(want["grad"]).to(dtype).double().numpy()
-    err = np.abs(out["grad"].double().cpu().numpy() - w)
-    # fp32: the loss kernel's 1e-6; bf16: two units in the last place of the rounded oracle.
-    # At most one token within rounding of a clip bound may take the other side of the min.
-    bound = 1e-6 if dtype == torch.float32 else 2.0 ** -7 * np.abs(w) + 1e-9
-    assert np.count_nonzero(err > bound) <= 1, float(err.max())
+    # these inputs keep the loss well away from a +/-A cancellation (|loss| > 0.5 sum|terms|)
+    assert abs(want["loss"]) > 0.5 * want["abs_sum"]
+    assert abs(out["loss"].item() - want["loss"]) <= tol * abs(want["loss"])
+    w = want["grad"]
+    # fp32: max abs 1e-6; bf16: one unit in the last place of the rounded oracle value.
+    # A token whose ratio lies within 8 fp32 ulps of 1 + eps_hi may take either side of
+    # the min() in fp32 (both are correct), so it is left out, as in the loss-kernel tests.
+    lp_d, old_d = oracle.decode(inp["policy_lp"]), oracle.decode(inp["old_lp"])
+    hi = np.float32(1.0) + np.float32(0.28)
+    kink = np.abs(np.exp(lp_d - old_d) - float(hi)) <= 8 * float(np.spacing(hi))
+    got = out["grad"].double().cpu().numpy()
+    if dtype == torch.float32:
+        err, bound = np.abs(got - w), 1e-6
+    else:
+        wr = torch.from_numpy(w).to(dtype).double().numpy()
+        ax = np.abs(wr)
+        ulp = np.exp2(np.maximum(np.floor(np.log2(np.where(ax > 0, ax, 1.0))), -126) - 7)
+        err, bound = np.abs(got - wr) / ulp, 1.0
+    bad = (err > bound) & ~kink
+    assert not bad.any(), (int(bad.sum()), float(err[~kink].max()))
     assert int(out["count"].item()) == (want["n_valid"] if red == 0 else bs)
 
 
