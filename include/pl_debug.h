@@ -84,6 +84,17 @@ int pl_debug_set_loss_path(int path);
 int pl_debug_set_rkl_cluster(int cl);
 
 /*
+ * Chooses the reverse-KL kernel for later calls with a gradient on this
+ * process: 1 = the streaming kernel (pass 2 re-reads each slice from L2);
+ * 2 = the register-resident kernel (each slice read from HBM once) wherever it
+ * applies -- 16-bit logits, V a multiple of 8, 16-byte aligned student,
+ * teacher and gradient, and a row slice that fits its shared-memory slots --
+ * and the streaming kernel otherwise; 0 restores the default (the streaming
+ * kernel, measured faster).  Returns PL_ERR_ARG for another value.
+ */
+int pl_debug_set_rkl_path(int path);
+
+/*
  * Forces the GEMM's pair tile for later launches on this process: 1 = 256 x 256
  * (one N=256 MMA per K step, double-buffered accumulators), 2 = 256 x 512 (two
  * MMAs sharing the A stage); 0 restores the host's choice (256 x 512 when every
@@ -104,9 +115,28 @@ int pl_debug_pick_tile(int njobs, const int64_t* mnk, int pairs);
  * The persistent GEMM's tile schedule, for a host-side check: two problems of
  * t0 tiles (c0 k-steps each) and t1 tiles (c1 k-steps each) over `pairs` CTA
  * pairs.  out_pair[t] (t0 + t1 entries) receives the pair that runs tile t.
+ * The schedule balances per-pair loads counting each tile as its k-steps plus
+ * a fixed hand-off cost of 8 k-steps.
  * Returns 0, or -1 when some tile would run on no pair or on two.
  */
 int pl_debug_pair_tiles(int t0, int t1, int c0, int c1, int pairs, int32_t* out_pair);
+
+/*
+ * The backward launch's K-split choice (host logic, no device call): for the two
+ * problems mnk = {M0, N0, K0, M1, N1, K1} (dX, then dW) on `pairs` CTA pairs,
+ * returns 2 when the dX problem is computed in two K halves (each half's tiles
+ * add their fp32 results into a zeroed buffer, which is then rounded to the
+ * model dtype), else 1, or -1 on bad input; *nh_out (if not NULL) receives the
+ * tile width that goes with it (1: 256 wide, 2: 512 wide).
+ */
+int pl_debug_pick_split(const int64_t* mnk, int pairs, int* nh_out);
+
+/*
+ * Forces the K split of the fused path's backward dX problem for later calls on
+ * this process: 1 = never, 2 = always (when its K has at least two 64-wide
+ * steps); 0 restores the host's choice.  Returns PL_ERR_ARG for another value.
+ */
+int pl_debug_set_gemm_split(int mode);
 
 /* Number of kernels this library has launched in this process. */
 int64_t pl_debug_launch_count(void);

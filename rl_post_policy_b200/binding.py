@@ -98,6 +98,12 @@ _lib.pl_debug_set_gemm_tile.argtypes = [_I]
 _lib.pl_debug_set_gemm_tile.restype = _I
 _lib.pl_debug_set_rkl_cluster.argtypes = [_I]
 _lib.pl_debug_set_rkl_cluster.restype = _I
+_lib.pl_debug_set_rkl_path.argtypes = [_I]
+_lib.pl_debug_set_rkl_path.restype = _I
+_lib.pl_debug_pick_split.argtypes = [_P, _I, _P]
+_lib.pl_debug_pick_split.restype = _I
+_lib.pl_debug_set_gemm_split.argtypes = [_I]
+_lib.pl_debug_set_gemm_split.restype = _I
 _lib.pl_debug_launch_count.argtypes = []
 _lib.pl_debug_launch_count.restype = _I64
 
@@ -106,7 +112,8 @@ EXPORTED = ("pl_init", "pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_line
             "pl_fused_linear_grpo_workspace_bytes", "pl_device_status", "pl_status_string",
             "pl_version", "pl_debug_gemm", "pl_debug_gemm_out", "pl_debug_timing", "pl_debug_timing_read",
             "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_set_gemm_tile", "pl_debug_pair_tiles",
-            "pl_debug_pick_tile", "pl_debug_set_loss_path")
+            "pl_debug_pick_tile", "pl_debug_set_loss_path", "pl_debug_pick_split", "pl_debug_set_gemm_split",
+            "pl_debug_set_rkl_path")
 
 
 class PLError(RuntimeError):
@@ -297,6 +304,29 @@ def pl_debug_pick_tile(problems, pairs: int) -> int:
     flat = [int(x) for mnk in problems for x in mnk]
     arr = (ctypes.c_int64 * max(len(flat), 1))(*flat)
     return int(_lib.pl_debug_pick_tile(len(problems), arr, pairs))
+
+
+def pl_debug_pick_split(problems, pairs: int):
+    """Test hook: the backward launch's K split of its dX problem (1 or 2) and the
+    tile width that goes with it, for the (M, N, K) of dX and dW."""
+    flat = [int(x) for mnk in problems for x in mnk]
+    if len(flat) != 6:
+        return -1, 0
+    arr = (ctypes.c_int64 * 6)(*flat)
+    nh = ctypes.c_int(0)
+    split = int(_lib.pl_debug_pick_split(arr, pairs, ctypes.byref(nh)))
+    return split, int(nh.value)
+
+
+def pl_debug_set_rkl_path(path: int) -> int:
+    """Test hook: reverse KL with a gradient -- 0 the default (the streaming kernel), 1 the
+    streaming kernel, 2 the register-resident kernel where it applies."""
+    return int(_lib.pl_debug_set_rkl_path(int(path)))
+
+
+def pl_debug_set_gemm_split(mode: int) -> int:
+    """Test hook: K split of the backward dX problem -- 0 the host's choice, 1 never, 2 always."""
+    return int(_lib.pl_debug_set_gemm_split(int(mode)))
 
 
 def pl_debug_set_loss_path(path: int) -> int:

@@ -66,6 +66,30 @@ extern "C" int pl_debug_pick_tile(int njobs, const int64_t* mnk, int pairs) {
   return pick_tile_width(p, pairs);
 }
 
+// pl_debug_pick_split: the K-split choice for the dX problem (job 0) of a
+// two-problem backward launch, and the tile width that goes with it.
+extern "C" int pl_debug_pick_split(const int64_t* mnk, int pairs, int* nh_out) {
+  if (!mnk || pairs < 1) return -1;
+  GemmParams p{};
+  p.njobs = 2;
+  for (int i = 0; i < 2; ++i) {
+    if (mnk[3 * i] < 1 || mnk[3 * i + 1] < 1 || mnk[3 * i + 2] < 1) return -1;
+    if (mnk[3 * i] > (1 << 30) || mnk[3 * i + 1] > (1 << 30) || mnk[3 * i + 2] > (1 << 30)) return -1;
+    p.jobs[i].M = (int)mnk[3 * i];
+    p.jobs[i].N = (int)mnk[3 * i + 1];
+    p.jobs[i].K = (int)mnk[3 * i + 2];
+  }
+  const int split = gemm_choose_k_split(&p, 0, pairs);
+  if (nh_out) *nh_out = p.nh;
+  return split;
+}
+
+extern "C" int pl_debug_set_gemm_split(int mode) {
+  if (mode < 0 || mode > 2) return PL_ERR_ARG;
+  debug_knobs().gemm_split = mode;
+  return PL_OK;
+}
+
 // pl_debug_pair_tiles: the GEMM's tile schedule for two jobs (t0 tiles of c0
 // k-steps, then t1 tiles of c1 k-steps) over `pairs` CTA pairs.  Writes, for
 // every tile, the pair that runs it (out_pair[t0 + t1]) and returns 0, or -1 if
@@ -150,6 +174,12 @@ extern "C" void pl_debug_set_wait(unsigned long long wait_ns, unsigned extra_arr
 extern "C" int pl_debug_set_gemm_tile(int nh) {
   if (nh < 0 || nh > 2) return PL_ERR_ARG;
   debug_knobs().gemm_nh = nh;
+  return PL_OK;
+}
+
+extern "C" int pl_debug_set_rkl_path(int path) {
+  if (path < 0 || path > 2) return PL_ERR_ARG;
+  debug_knobs().rkl_path = path;
   return PL_OK;
 }
 

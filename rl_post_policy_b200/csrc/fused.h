@@ -23,6 +23,7 @@ struct FusedOffsets {
   int64_t part_ref;   // float2 [C, ntv]     reference ditto
   int64_t logits;     // T [C, ld]           logits, then dlogits (if a gradient is wanted)
   int64_t dw_acc;     // f32 [V, H]          dW accumulator (multi-chunk only)
+  int64_t dx_acc;     // f32 [C, H]          the chunk's dX when the backward splits its K (zeroed per chunk)
   int64_t db_acc;     // f32 [V]             dbias accumulator (multi-chunk only)
   int64_t db_part;    // f32 [kDlMaxRowGroups, V]  dbias column sums per dlogits row group
   int64_t db_cnt;     // u32 [ceil(V/256)]   finished row groups per 256-column strip (self-resetting)

@@ -7,6 +7,7 @@
 //                combine  (lse, logp, ref_logp, loss partials, g)
 //                dlogits  (in place, 2^e-scaled, + dbias)                       (if a gradient is wanted)
 //                GEMM  [dX rows of the chunk = dz W]  [dW (+)= dz^T X_chunk]     (if dX or dW)
+//                (convert: dX from its fp32 buffer, when the GEMM split dX's K in two)
 //          -> convert (the fp32 dW accumulator to the model dtype; several chunks only)
 //          -> finalize (fixed-order loss sum)
 //
@@ -66,6 +67,7 @@ Plan make_plan(int64_t bs, int64_t T, int64_t H, int64_t V, uint32_t mode, bool 
   p.off.part_ref = region(8 * p.Cbuf * (int64_t)p.nparts);
   p.off.logits = region(2 * p.Cbuf * p.ld);
   p.off.dw_acc = region((need_dW && p.nchunks > 1) ? 4 * V * H : 0);
+  p.off.dx_acc = region(4 * p.Cbuf * (H > 0 ? H : 0));
   p.off.db_acc = region((need_dbias && p.nchunks > 1) ? 4 * V : 0);
   p.off.db_part = region(need_dbias ? 4 * (int64_t)kDlMaxRowGroups * V : 0);
   p.off.db_cnt = region(need_dbias ? 4 * (int64_t)p.ntv : 0);
@@ -271,7 +273,28 @@ pl_status run_pipeline(const Pipe& q) {
     }
     bp.njobs = nj;
     gemm_finalize_jobs(&bp);
+    // dX has K = V: its few long tiles would finish last next to the many short
+    // dW tiles.  When the schedule estimate says so, each dX tile is computed as
+    // two tiles over the halves of the vocabulary, both adding their fp32 result
+    // into a zeroed buffer through the TMA unit (two addends onto zero: the sum
+    // does not depend on their order), which one pass then rounds into dX.
+    int dx_split = 1;
+    float* dx_acc = reinterpret_cast<float*>(ws + plan.off.dx_acc);
+    if (dX) {
+      DevInfo di;
+      if (dev_info(&di) != cudaSuccess) return PL_ERR_CUDA;
+      dx_split = gemm_choose_k_split(&bp, 0, di.sm_count / 2);
+    }
+    if (dx_split == 2) {
+      GemmJob& j = bp.jobs[0];
+      if (!make_tmap_2d(&bp.maps[5], dx_acc, DType::F32, H, rows, H * 4, kOutBoxN, kOutBoxM)) return PL_ERR_CUDA;
+      j.out = dx_acc; j.out_f32 = 1; j.out_path = kOutTmaReduce; j.out_map = 5; j.out_ld = H;
+      if (!ok(cudaMemsetAsync(dx_acc, 0, (size_t)rows * H * 4, s))) return PL_ERR_CUDA;
+    }
     if (!ok(launch_gemm(bp, dt, s))) return PL_ERR_CUDA;
+    if (dx_split == 2 &&
+        !ok(launch_convert(dx_acc, static_cast<unsigned char*>(dX) + r0 * H * esz, rows * H, dt, s)))
+      return PL_ERR_CUDA;
     if (dW && plan.nchunks > 1 && c + 1 == plan.nchunks &&
         !ok(launch_convert(reinterpret_cast<const float*>(ws + plan.off.dw_acc), dW, V * H, dt, s)))
       return PL_ERR_CUDA;

@@ -51,6 +51,14 @@ struct GemmJob {
   int a_mn, b_mn;          // 0 = K-major, 1 = MN-major
   int M, N, K;
   int tiles_m, tiles_n, k_steps;
+  // K split: 1, or 2 -- every output tile is then computed as two tiles, one per
+  // half of the k-steps, and each adds its fp32 result into `out` through the TMA
+  // unit (out_path kOutTmaReduce, out_f32, onto a zeroed buffer; with exactly two
+  // addends onto zero the sum does not depend on their order).  Halving the
+  // length of a problem's longest tiles lets the schedule balance a launch whose
+  // long tiles would otherwise finish last.
+  int k_split;
+  int k_per;               // k-steps per split (set by gemm_finalize_jobs)
   int n_inner;             // 1: consecutive tiles walk N first (share the A rows)
   int tile_begin;          // first global tile index of this job
   int epi;
@@ -101,16 +109,25 @@ struct __align__(64) GemmParams {
 bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, uint64_t outer,
                   uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128 = true);
 
-// Fills tiles_m/tiles_n/k_steps/tile_begin of each job and total_tiles, for
-// tiles nh * kBN wide.  launch_gemm picks nh and calls it again.
+// Fills tiles_m/tiles_n/k_steps/k_per/tile_begin of each job and total_tiles, for
+// tiles nh * kBN wide.  launch_gemm picks nh (unless p->nh is set) and calls it again.
 void gemm_finalize_jobs(GemmParams* p);
+
+// Tiles of a job (output tiles times its K split).
+inline int job_tiles(const GemmJob& j) { return j.tiles_m * j.tiles_n * (j.k_split > 1 ? j.k_split : 1); }
 
 cudaError_t launch_gemm(const GemmParams& p, DType dt, cudaStream_t stream);
 
 // The tile width launch_gemm uses on P pairs (1: 256 wide, 2: 512 wide) unless
-// a test forces one, from the jobs' M, N, K.
+// a test forces one or p.nh is set, from the jobs' M, N, K and K splits.
 double launch_estimate(GemmParams p, int nh, int P);
 int pick_tile_width(const GemmParams& p, int P);
+
+// Decides whether job `job` of a two-problem launch is computed in two K halves
+// (see GemmJob::k_split) and with which tile width, on P pairs: sets
+// p->jobs[job].k_split and p->nh.  A debug knob can force the split on or off.
+// Returns the chosen k_split.
+int gemm_choose_k_split(GemmParams* p, int job, int P);
 
 // Tile schedule (host side of what the kernel runs): balance_schedule fills
 // sched/na/nb/rem for P pairs; pair_tile gives the i-th tile of a pair or -1.

@@ -103,13 +103,25 @@ template <> struct AbFormat<__nv_bfloat16> { static constexpr uint32_t v = 1; };
 
 struct TileCoord {
   int job, mb, nb;
+  int kb, nk;  // first k-step and number of k-steps of this tile (all of K unless the job is split)
 };
 
+// Tile `tile` of the launch: its job, row block, column block and K range.  A
+// split job lists all tiles of its first K half, then all of the second.
 __device__ __forceinline__ TileCoord tile_coord(const GemmParams& p, int tile) {
   TileCoord c;
   c.job = (p.njobs > 1 && tile >= p.jobs[1].tile_begin) ? 1 : 0;
   const GemmJob& j = p.jobs[c.job];
-  const int local = tile - j.tile_begin;
+  int local = tile - j.tile_begin;
+  c.kb = 0;
+  c.nk = j.k_steps;
+  if (j.k_split > 1) {
+    const int per = j.tiles_m * j.tiles_n;
+    const int ks = local / per;
+    local -= ks * per;
+    c.kb = ks * j.k_per;
+    c.nk = min(j.k_per, j.k_steps - c.kb);
+  }
   if (j.n_inner) {
     c.mb = local / j.tiles_n;
     c.nb = local - c.mb * j.tiles_n;
@@ -289,13 +301,13 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
         const int nt0 = tc.nb * Cfg::kTileN + (int)rank * kBNh;
         const CUtensorMap* amap = &p.maps[j.a_map];
         const CUtensorMap* bmap = &p.maps[j.b_map];
-        for (int k = 0; k < j.k_steps; ++k) {
+        for (int k = 0; k < tc.nk; ++k) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, lim)) break;
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes + p.extra_tx);
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = ring + stage * kStageBytes;
           uint8_t* b_dst = a_dst + kABytes;
-          const int k0 = k * kBK;
+          const int k0 = (tc.kb + k) * kBK;
           if (!j.a_mn) {
             tma_load_2d_pair(a_dst, amap, bar, k0, m0);
           } else {
@@ -334,7 +346,8 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
       int acc = 0;
       uint32_t acc_phase = 0;
       const uint32_t ring_addr = smem_u32(ring);
-      // The K=16 MMAs of one stage into accumulator half h (column offset d_col).
+      // The K=16 MMAs of one stage into accumulator half h (column offset d_col);
+      // k counts the tile's own k-steps, so its first step overwrites the accumulator.
       auto issue = [&](int st, int k, const GemmJob& j, uint32_t idesc, int h, uint32_t d_col) {
         const uint32_t a_addr = ring_addr + st * kStageBytes;
         const uint32_t b_addr = a_addr + kABytes + h * kBBytes;
@@ -357,7 +370,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
         if constexpr (NH == 1) {
           if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, lim)) break;
           tc_fence_after();
-          for (int k = 0; k < j.k_steps; ++k) {
+          for (int k = 0; k < tc.nk; ++k) {
             if (!mbar_wait(&full[stage], phase, abort_flag, lim)) { ok = false; break; }
             tc_fence_after();
             issue(stage, k, j, idesc, 0, acc * kBN);
@@ -393,7 +406,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
             }
             held = 0;
           };
-          for (int k = 0; k < j.k_steps; ++k) {
+          for (int k = 0; k < tc.nk; ++k) {
             if (!mbar_wait(&full[stage], phase, abort_flag, lim)) { ok = false; break; }
             tc_fence_after();
             issue(stage, k, j, idesc, 0, 0);
@@ -675,23 +688,40 @@ void gemm_finalize_jobs(GemmParams* p) {
     j.tiles_m = (j.M + kPairM - 1) / kPairM;
     j.tiles_n = (j.N + tile_n - 1) / tile_n;
     j.k_steps = (j.K + kBK - 1) / kBK;
+    // a split needs a k-step for each half (an empty half would store an unwritten accumulator)
+    j.k_split = (j.k_split == 2 && j.k_steps >= 2) ? 2 : 1;
+    j.k_per = (j.k_steps + j.k_split - 1) / j.k_split;
     j.tile_begin = begin;
-    begin += j.tiles_m * j.tiles_n;
+    begin += job_tiles(j);
   }
   p->total_tiles = begin;
 }
 
-// Chooses the tile schedule for `P` pairs (see GemmParams::sched).
+// Cost of a launch in k-step units (one K=64 step of one N=256 MMA group).
+// Each tile also pays a fixed kTileOverhead for its accumulator hand-off and
+// pipeline turn; fitted to the backward launch of a 1024-row chunk (V=128256,
+// H=4096), whose 16-k-step dW tiles ran about 18% slower at 256 wide than at
+// 512 wide.
+constexpr double kTileOverhead = 8.0;
+
+namespace {
+// k-steps of one tile of job j (of one K half for a split job)
+long tile_ksteps(const GemmJob& j) { return j.k_split > 1 ? j.k_per : j.k_steps; }
+}  // namespace
+
+// Chooses the tile schedule for `P` pairs (see GemmParams::sched).  Tile costs
+// are k-steps x width plus the per-tile overhead.
 void balance_schedule(GemmParams* p, int P) {
   p->sched = 0;
   p->na = p->nb = p->rem = 0;
   if (p->njobs != 2) return;
   const GemmJob& j0 = p->jobs[0];
   const GemmJob& j1 = p->jobs[1];
-  const long T0 = (long)j0.tiles_m * j0.tiles_n, T1 = (long)j1.tiles_m * j1.tiles_n;
-  const long c0 = j0.k_steps, c1 = j1.k_steps > 0 ? j1.k_steps : 1;
+  const long T0 = job_tiles(j0), T1 = job_tiles(j1);
+  const double w = p->nh == 2 ? 2.0 : 1.0;
+  const double c0 = tile_ksteps(j0) * w + kTileOverhead, c1 = (tile_ksteps(j1) > 0 ? tile_ksteps(j1) : 1) * w + kTileOverhead;
   if (T0 > P || c0 < 4 * c1 || T1 == 0) return;  // equal-cost tiles: round-robin is balanced
-  const double ideal = (double)(T0 * c0 + T1 * c1) / P;
+  const double ideal = (T0 * c0 + T1 * c1) / P;
   long nb = (long)(ideal / c1);
   long na = (long)((ideal - c0) / c1);
   if (na < 0) na = 0;
@@ -711,44 +741,72 @@ void balance_schedule(GemmParams* p, int P) {
   p->rem = (int)(T1 - total());
 }
 
-// Estimated launch length, in N=256 MMA k-steps per pair, for pair tiles nh
-// MMAs wide on P pairs: the larger of the even share of all the work and the
-// longest single tile (a tile runs on one pair), or, for one problem of
-// equal-cost tiles, whole waves of tiles.
-// Cost of a launch in k-step units (one K=64 step of one N=256 MMA group): the
-// busiest pair's share.  Each tile also pays a fixed kTileOverhead for its
-// accumulator hand-off and pipeline turn; fitted to the backward launch of a
-// 1024-row chunk (V=128256, H=4096), whose 16-k-step dW tiles ran about 18%
-// slower at 256 wide than at 512 wide.
-constexpr double kTileOverhead = 8.0;
-
+// Estimated launch length on P pairs with pair tiles nh MMAs wide: the busiest
+// pair's load, in k-step units, under the schedule balance_schedule picks.
 double launch_estimate(GemmParams p, int nh, int P) {
   p.nh = nh;
   gemm_finalize_jobs(&p);
-  double work = 0.0, longest = 0.0;
-  for (int i = 0; i < p.njobs; ++i) {
-    const GemmJob& j = p.jobs[i];
-    const double tile = (double)j.k_steps * nh + kTileOverhead;
-    work += (double)j.tiles_m * j.tiles_n * tile;
-    if (j.tiles_m * j.tiles_n > 0 && tile > longest) longest = tile;
+  balance_schedule(&p, P);
+  const long T0 = job_tiles(p.jobs[0]);
+  const long T1 = p.njobs > 1 ? job_tiles(p.jobs[1]) : 0;
+  const double c0 = tile_ksteps(p.jobs[0]) * (double)nh + kTileOverhead;
+  const double c1 = p.njobs > 1 ? tile_ksteps(p.jobs[1]) * (double)nh + kTileOverhead : 0.0;
+  double worst = 0.0;
+  for (long q = 0; q < P; ++q) {
+    long n0, n1;
+    if (p.sched == 1) {
+      n0 = q < T0 ? 1 : 0;
+      n1 = (q < T0 ? p.na : p.nb) + (q < p.rem ? 1 : 0);
+    } else {
+      const long ntot = q < T0 + T1 ? (T0 + T1 - 1 - q) / P + 1 : 0;
+      n0 = q < T0 ? (T0 - 1 - q) / P + 1 : 0;
+      n1 = ntot - n0;
+    }
+    const double load = n0 * c0 + n1 * c1;
+    if (load > worst) worst = load;
   }
-  if (p.njobs == 1) {
-    const double waves = (double)((p.total_tiles + P - 1) / P);
-    return waves * longest;
-  }
-  const double share = work / P;
-  return share > longest ? share : longest;
+  return worst;
 }
 
 // 256 x 512 tiles move 25% fewer operand bytes per flop, halve the barrier
 // round trips and the tile count; measured on this kernel they run the same
 // k-step work about 10% faster when the launch stays balanced.  They need every
 // problem to be at least 512 wide.
+constexpr double kWideSpeed = 0.9;
+
 int pick_tile_width(const GemmParams& p, int P) {
   if (P <= 0) return 1;
   for (int i = 0; i < p.njobs; ++i)
     if (p.jobs[i].N < 2 * kBN) return 1;
-  return 0.9 * launch_estimate(p, 2, P) < launch_estimate(p, 1, P) ? 2 : 1;
+  return kWideSpeed * launch_estimate(p, 2, P) < launch_estimate(p, 1, P) ? 2 : 1;
+}
+
+// Measured on the fused backward launch (1024-row chunk and whole 8192-row
+// batch, V=128256, H=4096), the split was no faster: 5-10% slower at 1024 rows
+// and within 1% at 8192, although the schedule estimate promised 3-6%.  So it
+// runs only when a test or a measurement asks for it (debug knob 2).
+constexpr double kSplitGain = 0.98;
+
+int gemm_choose_k_split(GemmParams* p, int job, int P) {
+  const int knob = debug_knobs().gemm_split == 0 ? 1 : debug_knobs().gemm_split;
+  double best = 0.0;
+  int best_split = 1, best_nh = 1;
+  for (int split = 1; split <= 2; ++split) {
+    if ((knob == 1 && split == 2) || (knob == 2 && split == 1)) continue;
+    GemmParams q = *p;
+    q.jobs[job].k_split = split;
+    const int nh = debug_knobs().gemm_nh ? debug_knobs().gemm_nh : pick_tile_width(q, P);
+    const double e = launch_estimate(q, nh, P) * (nh == 2 ? kWideSpeed : 1.0);
+    if (split == 1 || knob == 2 || e < kSplitGain * best) {
+      best = e;
+      best_split = split;
+      best_nh = nh;
+    }
+  }
+  p->jobs[job].k_split = best_split;
+  p->nh = best_nh;
+  gemm_finalize_jobs(p);
+  return p->jobs[job].k_split;
 }
 
 namespace {
@@ -810,6 +868,8 @@ cudaError_t launch_gemm(const GemmParams& p0, DType dt, cudaStream_t stream) {
   int nh = 1;
   if (debug_knobs().gemm_nh) {
     nh = debug_knobs().gemm_nh;
+  } else if (p.nh == 1 || p.nh == 2) {
+    nh = p.nh;  // chosen by the caller (gemm_choose_k_split)
   } else {
     DevInfo di;
     if (dev_info(&di) == cudaSuccess) nh = pick_tile_width(p, di.sm_count / 2);
@@ -818,9 +878,12 @@ cudaError_t launch_gemm(const GemmParams& p0, DType dt, cudaStream_t stream) {
   gemm_finalize_jobs(&p);
   if (p.total_tiles <= 0) return cudaSuccess;
   // fp32 TMA outputs (chunked dW accumulation, the debug hook) move 32-column
-  // boxes: 4 epilogue warps with two boxes each drain them faster than 8 with one
+  // boxes: 4 epilogue warps with two boxes each drain them faster than 8 with one.
+  // A split job's fp32 output is small next to its K (two adds per output element
+  // over thousands of k-steps) and does not count.
   bool f32_tma = false;
-  for (int i = 0; i < p.njobs; ++i) f32_tma = f32_tma || (p.jobs[i].out_path != kOutDirect && p.jobs[i].out_f32);
+  for (int i = 0; i < p.njobs; ++i)
+    f32_tma = f32_tma || (p.jobs[i].out_path != kOutDirect && p.jobs[i].out_f32 && p.jobs[i].k_split < 2);
   if (dt == DType::BF16) {
     if (f32_tma) return nh == 2 ? launch_t<__nv_bfloat16, 2, 4>(p, stream) : launch_t<__nv_bfloat16, 1, 4>(p, stream);
     return nh == 2 ? launch_t<__nv_bfloat16, 2, 8>(p, stream) : launch_t<__nv_bfloat16, 1, 8>(p, stream);

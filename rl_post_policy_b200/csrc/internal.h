@@ -111,6 +111,10 @@ struct DebugKnobs {
   int gemm_nh = 0;       // GEMM tile width in N=256 MMAs (1 or 2; 0 = the host's choice)
   int loss_path = 0;     // loss kernel: 0 = the host's choice, 1 = small-batch kernel when eligible,
                          // 2 = the cooperative kernel
+  int rkl_path = 0;      // reverse KL with a gradient: 0 = the host's choice (the streaming kernel),
+                         // 1 = the streaming kernel, 2 = the register-resident kernel where it applies
+  int gemm_split = 0;    // K split of the backward launch's dX problem: 0 = the host's choice,
+                         // 1 = never, 2 = always (when it has at least two k-steps)
 };
 DebugKnobs& debug_knobs();
 

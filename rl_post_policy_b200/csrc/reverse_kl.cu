@@ -42,6 +42,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace pl {
 namespace {
@@ -226,6 +227,9 @@ struct RklArgs {
   int64_t slice;   // columns per CTA (multiple of 8)
   int cl;          // CTAs per cluster
   int vec;         // 16-byte vector path (s, t and grad share their address mod 16)
+  // register-resident gradient form only
+  unsigned long long wait_ns;  // bound of every wait
+  unsigned extra_tx;           // test-only: extra bytes each slot's load expects (0 in normal use)
 };
 
 __device__ __forceinline__ unsigned cluster_rank() {
@@ -535,6 +539,337 @@ __global__ void __launch_bounds__(kThreads, 2) reverse_kl_kernel(RklArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- register-resident gradient form
+// The forward + gradient call for 16-bit logits whose rows are 16-byte
+// aligned.  A row's slice is read from HBM once: 1-D bulk copies bring it into
+// shared-memory slots of 8 KB per tensor, pass 1 moves each slot into the
+// registers of the 512 compute threads (one 16-byte vector of each tensor per
+// thread and slot) while it accumulates the statistics, and releases the slot
+// at once, so a producer warp fetches the next row's slice while this row is
+// reduced, merged across the cluster and turned into its gradient.  Pass 2
+// reads nothing from memory: the gradient comes from the registers.  The
+// cluster merge exchanges the CTAs' statistics through distributed shared
+// memory with release/acquire mbarrier arrivals (every wait bounded), in rank
+// order as in reverse_kl_kernel.
+constexpr int kResThreads = 512;             // compute threads
+constexpr int kResWarps = kResThreads / 32;
+constexpr int kResBlock = kResThreads + 32;  // + one producer warp
+constexpr int kResSlots = 8;                 // slots per CTA slice
+constexpr int kResSlotBytes = 8192;          // per tensor and slot: 512 threads x 16 bytes
+
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kResThreads) : "memory"); }
+__device__ __forceinline__ uint4 ld_shared16(uint32_t saddr) {
+  uint4 u;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(saddr));
+  return u;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t cluster_addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
+}
+// Bounded wait on a barrier other CTAs of the cluster arrive on (acquire at cluster scope).
+__device__ __forceinline__ bool xwait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                      unsigned long long limit) {
+  if (sm100::mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = sm100::globaltimer();
+  while (!*abort) {
+    if (sm100::mbar_try_wait_cluster(bar, parity)) return true;
+    if (sm100::globaltimer() - t0 > limit) {
+      *abort = 1;
+      return false;
+    }
+  }
+  return false;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kResBlock, 1) reverse_kl_resident_kernel(RklArgs a) {
+  static_assert(sizeof(T) == 2, "16-bit logits");
+  constexpr int kP = Elt<T>::kPairs;
+  constexpr int kE = 2 * kP;                      // elements per 16-byte vector
+  constexpr int kSub = kResSlotBytes / (int)sizeof(T);
+  extern __shared__ __align__(128) unsigned char ring[];   // [slot][tensor][kResSlotBytes]
+  __shared__ uint64_t full[kResSlots], empty[kResSlots], xbar[2];
+  __shared__ Stats warp_stats[kResWarps];
+  __shared__ float xch[2][kMaxCluster][5];        // every CTA's statistics, by row parity
+  __shared__ unsigned long long s_count;
+  __shared__ double s_part;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned crank = cluster_rank(), cid = cluster_id(), ncl = cluster_count();
+  const int cl = a.cl;
+  if (tid == 0) {
+    s_count = 0;
+    s_part = 0.0;
+    s_abort = 0;
+    for (int j = 0; j < kResSlots; ++j) {
+      sm100::mbar_init(&full[j], 1);
+      sm100::mbar_init(&empty[j], kResWarps);   // one arrival per compute warp
+    }
+    sm100::mbar_init(&xbar[0], cl);
+    sm100::mbar_init(&xbar[1], cl);
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  cluster_sync();   // every CTA's barriers exist before any remote arrival
+
+  // ---- valid rows (every CTA counts the whole mask) ----
+  int64_t n_valid = a.N;
+  if (a.mask) {
+    if (tid < kResThreads) {
+      const uint8_t* m = a.mask;
+      const int64_t head = imin(a.N, (int64_t)((16 - (reinterpret_cast<uintptr_t>(m) & 15)) & 15));
+      const int64_t nv16 = (a.N - head) / 16;
+      unsigned long long c = 0;
+      for (int64_t i = tid; i < head; i += kResThreads) c += m[i] != 0;
+      const uint4* m16 = reinterpret_cast<const uint4*>(m + head);
+      for (int64_t i = tid; i < nv16; i += kResThreads) {
+        const uint4 u = __ldg(m16 + i);
+        c += nonzero_bytes(u.x) + nonzero_bytes(u.y) + nonzero_bytes(u.z) + nonzero_bytes(u.w);
+      }
+      for (int64_t i = head + nv16 * 16 + tid; i < a.N; i += kResThreads) c += m[i] != 0;
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) c += __shfl_down_sync(0xffffffffu, c, d);
+      if (lane == 0 && c) atomicAdd(&s_count, c);
+    }
+    __syncthreads();
+    n_valid = (int64_t)s_count;
+  }
+  const float log2_scale = -log2f((float)(n_valid > 1 ? n_valid : 1));
+
+  const int64_t v0 = imin(a.V, (int64_t)crank * a.slice);
+  const int64_t v1 = imin(a.V, v0 + a.slice);
+  const int n = (int)(v1 - v0);                   // multiple of 8 (the host checks V and slice)
+  const int nslot = (n + kSub - 1) / kSub;        // <= kResSlots (the host picks the cluster size)
+  volatile int* abort = &s_abort;
+
+  if (warp == kResWarps) {
+    // ---------------- producer: the slices of this cluster's valid rows, in row order ----------------
+    if (lane == 0) {
+      const unsigned long long pol = policy_evict_first();
+      uint32_t eph = 0;
+      for (int64_t r = cid; r < a.N && !*abort; r += ncl) {
+        if (a.mask && a.mask[r] == 0) continue;
+        const T* srow = static_cast<const T*>(a.s) + r * a.V + v0;
+        const T* trow = static_cast<const T*>(a.t) + r * a.V + v0;
+        for (int j = 0; j < nslot; ++j) {
+          // the consumers have moved this slot's previous row into registers
+          if (!sm100::mbar_wait(&empty[j], ((eph >> j) & 1u) ^ 1u, abort, a.wait_ns)) break;
+          eph ^= 1u << j;
+          const uint32_t bytes = (uint32_t)min(kSub, n - j * kSub) * (uint32_t)sizeof(T);
+          unsigned char* dst = ring + (size_t)j * 2 * kResSlotBytes;
+          sm100::mbar_arrive_expect_tx(&full[j], 2 * bytes + a.extra_tx);
+          sm100::bulk_load_1d(dst, srow + j * kSub, bytes, &full[j], pol);
+          sm100::bulk_load_1d(dst + kResSlotBytes, trow + j * kSub, bytes, &full[j], pol);
+        }
+      }
+      if (*abort) {
+        // leave time for copies already issued to land before shared memory is released
+        const unsigned long long t0 = sm100::globaltimer();
+        while (sm100::globaltimer() - t0 < 100000ull) __nanosleep(1000);
+      }
+    }
+  } else {
+    // ---------------- compute threads ----------------
+    uint32_t fph = 0, xph = 0;
+    int parity = 0;
+    uint4 sr[kResSlots], tr[kResSlots];
+    const uint32_t ring_u32 = sm100::smem_u32(ring);
+    const unsigned long long pl_first = policy_evict_first();
+    for (int64_t r = cid; r < a.N; r += ncl) {
+      T* grow = static_cast<T*>(a.grad) + r * a.V + v0;
+      if (a.mask && a.mask[r] == 0) {
+        // a masked row is not read; its gradient slice is zero
+#pragma unroll
+        for (int j = 0; j < kResSlots; ++j) {
+          const int nv = j < nslot ? min(kSub, n - j * kSub) / kE : 0;
+          if (tid < nv) st16_hint(reinterpret_cast<uint4*>(grow + j * kSub) + tid, make_uint4(0, 0, 0, 0), pl_first);
+        }
+        if (a.kl_rows && crank == 0 && tid == 0) a.kl_rows[r] = 0.0f;
+        continue;
+      }
+
+      // ---- pass 1: each slot into registers, online statistics ----
+      Acc acc;
+#pragma unroll
+      for (int j = 0; j < kResSlots; ++j) {
+        if (j < nslot) {
+          const int nv = min(kSub, n - j * kSub) / kE;
+          const bool ok = !*abort && sm100::mbar_wait(&full[j], (fph >> j) & 1u, abort, a.wait_ns);
+          fph ^= 1u << j;
+          if (ok && tid < nv) {
+            const uint32_t base = ring_u32 + (uint32_t)(j * 2 * kResSlotBytes) + (uint32_t)tid * 16u;
+            sr[j] = ld_shared16(base);
+            tr[j] = ld_shared16(base + kResSlotBytes);
+          }
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&empty[j]);   // the warp is done with the slot
+          if (ok && tid < nv) {
+            float2 ps[kP], pt[kP];
+            unpack<T>(sr[j], ps);
+            unpack<T>(tr[j], pt);
+            float bs = -INFINITY, bt = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < kP; ++k) {
+              bs = fmaxf(bs, fmaxf(ps[k].x, ps[k].y));
+              bt = fmaxf(bt, fmaxf(pt[k].x, pt[k].y));
+            }
+            acc.raise_max(bs, bt);
+            const float2 nmsl = make_float2(-acc.ms * kL2E, -acc.ms * kL2E);
+            const float2 nmtl = make_float2(-acc.mt * kL2E, -acc.mt * kL2E);
+#pragma unroll
+            for (int k = 0; k < kP; ++k) acc.add(ps[k], pt[k], nmsl, nmtl);
+          }
+        }
+      }
+
+      // ---- reduce: warp, then warps in order, then every CTA of the cluster in rank order ----
+      Stats st = acc.stats();
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) st = merge(st, shfl_down(st, d));
+      if (lane == 0) warp_stats[warp] = st;
+      consumers_sync();
+      if (warp == 0) {
+        st = lane < kResWarps ? warp_stats[lane] : Stats{-INFINITY, 0.f, 0.f, -INFINITY, 0.f};
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) st = merge(st, shfl_down(st, d));
+        // lane k < cl writes this CTA's statistics into slot [parity][crank] of CTA k
+        // of the cluster and arrives on its exchange barrier (release at cluster scope)
+        const float v[5] = {__shfl_sync(0xffffffffu, st.ms, 0), __shfl_sync(0xffffffffu, st.zs, 0),
+                            __shfl_sync(0xffffffffu, st.a, 0), __shfl_sync(0xffffffffu, st.mt, 0),
+                            __shfl_sync(0xffffffffu, st.zt, 0)};
+        if (lane < cl) {
+          const uint32_t dst = sm100::mapa_shared(sm100::smem_u32(&xch[parity][crank][0]), (uint32_t)lane);
+#pragma unroll
+          for (int q = 0; q < 5; ++q) st_cluster_f32(dst + 4u * q, v[q]);
+          sm100::mbar_arrive_cluster(sm100::mapa_shared(sm100::smem_u32(&xbar[parity]), (uint32_t)lane));
+        }
+      }
+      // every CTA's statistics for this row have arrived
+      xwait(&xbar[parity], (xph >> parity) & 1u, abort, a.wait_ns);
+      xph ^= 1u << parity;
+      Stats rs{xch[parity][0][0], xch[parity][0][1], xch[parity][0][2], xch[parity][0][3], xch[parity][0][4]};
+      for (int k = 1; k < cl; ++k)
+        rs = merge(rs, Stats{xch[parity][k][0], xch[parity][k][1], xch[parity][k][2], xch[parity][k][3],
+                             xch[parity][k][4]});
+      parity ^= 1;
+      const float ep = rs.a / rs.zs;                                      // E_p[s - t]
+      const float kl = ep - ((rs.ms - rs.mt) + logf(rs.zs / rs.zt));      // minus (lse_s - lse_t)
+      if (crank == 0 && tid == 0) {
+        s_part += (double)kl;
+        if (a.kl_rows) a.kl_rows[r] = kl;
+      }
+
+      // ---- pass 2: grad_v = scale * p_v * ((s_v - t_v) - E_p[s - t]) from the registers ----
+      const float off = -(rs.ms * kL2E + log2f(rs.zs)) + log2_scale;
+      const float2 l2e = make_float2(kL2E, kL2E), off2 = make_float2(off, off), nep = make_float2(-ep, -ep);
+#pragma unroll
+      for (int j = 0; j < kResSlots; ++j) {
+        const int nv = j < nslot ? min(kSub, n - j * kSub) / kE : 0;
+        if (tid < nv) {
+          float2 ps[kP], pt[kP], g[kP];
+          unpack<T>(sr[j], ps);
+          unpack<T>(tr[j], pt);
+#pragma unroll
+          for (int k = 0; k < kP; ++k) {
+            const float2 x = __ffma2_rn(ps[k], l2e, off2);
+            const float2 p = make_float2(ex2(x.x), ex2(x.y));
+            const float2 w = __fadd2_rn(__ffma2_rn(pt[k], make_float2(-1.f, -1.f), ps[k]), nep);
+            g[k] = __fmul2_rn(p, w);
+          }
+          st16_hint(reinterpret_cast<uint4*>(grow + j * kSub) + tid, pack<T>(g), pl_first);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  cluster_sync();   // no CTA leaves while a peer may still write into its exchange slots
+
+  // ---- loss: cluster partials, summed in cluster order by the last cluster ----
+  if (crank == 0 && warp == 0) {
+    double* partials = reinterpret_cast<double*>(a.ws + kWsHeader);
+    unsigned* done = reinterpret_cast<unsigned*>(a.ws + 8);
+    unsigned prev = 0;
+    if (lane == 0) {
+      partials[cid] = s_part;
+      __threadfence();
+      prev = atomicAdd(done, 1u);
+    }
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev == ncl - 1) {
+      __threadfence();
+      double sum = 0.0;
+      for (unsigned j = lane; j < ncl; j += 32) sum += *reinterpret_cast<volatile double*>(partials + j);
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) sum += __shfl_down_sync(0xffffffffu, sum, d);
+      if (lane == 0) {
+        *a.loss_out = (float)(sum / (double)(n_valid > 1 ? n_valid : 1));
+        if (a.n_valid_out) *a.n_valid_out = n_valid;
+        *done = 0u;
+      }
+    }
+  }
+  if (tid == 0 && *abort) atomicOr(reinterpret_cast<unsigned*>(a.ws), kDevErrTimeout);
+}
+
+template <typename T>
+size_t resident_smem(int nslot) { return (size_t)nslot * 2 * kResSlotBytes; }
+
+template <typename T>
+cudaError_t launch_resident_t(const RklArgs& a, unsigned nclusters, int nslot, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)a.cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(nclusters * (unsigned)a.cl);
+  cfg.blockDim = dim3(kResBlock);
+  cfg.dynamicSmemBytes = resident_smem<T>(nslot);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, reverse_kl_resident_kernel<T>, a);
+}
+
+// Resident clusters of the register-resident kernel at `cl` CTAs with `nslot` slots.
+template <typename T>
+int max_resident_clusters_t(int cl, int nslot) {
+  static std::mutex mu;
+  static int cache[16][4][kResSlots + 1] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return 0;
+  const int ci = cl == 1 ? 0 : cl == 2 ? 1 : cl == 4 ? 2 : 3;
+  std::lock_guard<std::mutex> lk(mu);
+  int& slot = cache[dev][ci][nslot];
+  if (slot == 0) {
+    const size_t smem = resident_smem<T>(nslot);
+    if (cudaFuncSetAttribute(reverse_kl_resident_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(kResSlots * 2 * kResSlotBytes)) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)cl * 64);
+    cfg.blockDim = dim3(kResBlock);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, reverse_kl_resident_kernel<T>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    slot = nc > 0 ? nc : -1;
+  }
+  return slot > 0 ? slot : 0;
+}
+
 template <typename T, bool GRAD>
 cudaError_t launch_t(const RklArgs& a, unsigned nclusters, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
@@ -633,6 +968,56 @@ extern "C" pl_status pl_reverse_kl(const void* student, const void* teacher, con
 
   DevInfo di;
   if (dev_info(&di) != cudaSuccess) return PL_ERR_CUDA;
+
+  // The register-resident form for the gradient of 16-bit logits whose rows
+  // start on 16-byte boundaries (the smallest cluster whose slices fit the
+  // shared-memory slots), on request: measured at the card's shape it was
+  // slower than the streaming kernel (517 against 336 us).
+  const int path = debug_knobs().rkl_path;
+  if (grad_out && dt != DType::F32 && V % 8 == 0 && ((ps | pt | pg) & 15) == 0 && path == 2) {
+    constexpr int64_t kSub = kResSlotBytes / 2;
+    int rc_cl = 0, nslot = 0, mc = 0;
+    const int forced_cl = debug_knobs().rkl_cluster;
+    for (int c = forced_cl ? forced_cl : 1; c <= kMaxCluster; c *= 2) {
+      const int64_t sl = ((V + c - 1) / c + 7) / 8 * 8;
+      const int ns = (int)((sl + kSub - 1) / kSub);
+      if (ns <= kResSlots) {
+        mc = dt == DType::BF16 ? max_resident_clusters_t<__nv_bfloat16>(c, ns)
+                               : max_resident_clusters_t<__half>(c, ns);
+        if (mc > 0) {
+          rc_cl = c;
+          nslot = ns;
+          break;
+        }
+      }
+      if (forced_cl) break;
+    }
+    if (rc_cl > 0) {
+      RklArgs a{};
+      a.s = student;
+      a.t = teacher;
+      a.mask = mask;
+      a.grad = grad_out;
+      a.loss_out = loss_out;
+      a.kl_rows = kl_rows_out;
+      a.n_valid_out = n_valid_out;
+      a.ws = static_cast<unsigned char*>(ws);
+      a.N = N;
+      a.V = V;
+      a.slice = ((V + rc_cl - 1) / rc_cl + 7) / 8 * 8;
+      a.cl = rc_cl;
+      a.vec = 1;
+      a.wait_ns = debug_knobs().wait_ns;
+      a.extra_tx = debug_knobs().extra_tx;
+      const int64_t want = N > 0 ? N : 1;
+      const unsigned ncl = (unsigned)std::min<int64_t>(std::min<int64_t>(want, mc), kMaxClusters);
+      launch_begin(2, s);
+      const cudaError_t e = dt == DType::BF16 ? launch_resident_t<__nv_bfloat16>(a, ncl, nslot, s)
+                                              : launch_resident_t<__half>(a, ncl, nslot, s);
+      launch_end(2, s);
+      return e == cudaSuccess ? PL_OK : PL_ERR_CUDA;
+    }
+  }
   int l2 = 0, dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
     return PL_ERR_CUDA;

@@ -32,6 +32,26 @@ def gemm_tile(request):
     pl.pl_debug_set_gemm_tile(0)
 
 
+@pytest.fixture(params=[1, 2], ids=["no_ksplit", "ksplit"])
+def dx_split(request):
+    """Runs a GPU test once with the backward launch's dX problem whole and once
+    with it split in two K halves (fp32 halves added into a zeroed buffer)."""
+    import rl_post_policy_b200 as pl
+    assert pl.pl_debug_set_gemm_split(request.param) == 0
+    yield request.param
+    pl.pl_debug_set_gemm_split(0)
+
+
+@pytest.fixture(params=[1, 2], ids=["rkl_streaming", "rkl_resident"])
+def rkl_path(request):
+    """Runs a GPU test once with the streaming reverse-KL kernel and once with the
+    register-resident gradient kernel wherever it applies."""
+    import rl_post_policy_b200 as pl
+    assert pl.pl_debug_set_rkl_path(request.param) == 0
+    yield request.param
+    pl.pl_debug_set_rkl_path(0)
+
+
 @pytest.fixture(params=[1, 2], ids=["small_kernel", "cooperative"])
 def loss_path(request):
     """Runs a GPU test once with each loss-only kernel: the small-batch kernel

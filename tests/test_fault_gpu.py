@@ -3,8 +3,9 @@ run out on purpose must come back as PL_ERR_DEVICE_TIMEOUT, release what they
 hold, and leave the context usable.
 
 The loss kernel's grid barrier is told to wait for one arrival more than there
-are blocks; the GEMM's pipeline stages are told to expect 16 bytes more than
-their TMA loads deliver.  Both waits are bounded to 50 ms for the test.
+are blocks; the GEMM's pipeline stages and the register-resident reverse-KL
+kernel's slots are told to expect 16 bytes more than their TMA loads deliver.
+The waits are bounded to 50 ms for the test.
 """
 import pytest
 import torch
@@ -60,3 +61,28 @@ def test_gemm_pipeline_timeout_is_reported(pl):
     assert pl.pl_device_status(None) == pl.PL_OK
     ref = A.double() @ B.double().t()
     assert torch.allclose(D.double(), ref, rtol=1e-4, atol=1e-3)
+
+
+def test_reverse_kl_slot_timeout_is_reported(pl):
+    # the register-resident reverse-KL kernel's slots expect 16 bytes more than their
+    # bulk copies deliver: the bounded waits run out, the cluster still finishes
+    # together, and the next normal call on the same workspace is correct
+    inp = synth.reverse_kl_inputs(2, 12, 5000, torch.bfloat16, synth.seed_for(51))
+    s, t, mk = inp["student"].cuda(), inp["teacher"].cuda(), inp["mask"].cuda()
+    N, V = 24, 5000
+    g = torch.empty(N, V, dtype=torch.bfloat16, device="cuda")
+    loss = torch.zeros(1, device="cuda")
+    wsb = pl.pl_reverse_kl_workspace_bytes(N, V)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    assert pl.pl_debug_set_rkl_path(2) == 0
+    pl.pl_debug_set_wait(50_000_000, 0, 16)
+    try:
+        pl.check(pl.pl_reverse_kl(s, t, mk, N, V, pl.PL_BF16, loss, g, None, None, ws, wsb))
+        assert pl.pl_device_status(ws) == pl.PL_ERR_DEVICE_TIMEOUT
+    finally:
+        pl.pl_debug_set_wait(0, 0, 0)
+        pl.pl_debug_set_rkl_path(0)
+    pl.check(pl.pl_reverse_kl(s, t, mk, N, V, pl.PL_BF16, loss, g, None, None, ws, wsb))
+    assert pl.pl_device_status(ws) == pl.PL_OK
+    want = oracle.reverse_kl(inp["student"], inp["teacher"], inp["mask"])
+    assert abs(loss.item() - want["loss"]) <= 1e-4 * abs(want["loss"])

@@ -16,7 +16,7 @@ import torch
 import oracle
 import synth
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("rkl_path")]
 
 
 def pl():
@@ -223,3 +223,24 @@ def test_aligned_rows(dtype, grad):
     want = oracle.reverse_kl(inp["student"], inp["teacher"], inp["mask"], want_grad=grad)
     got = run(inp["student"], inp["teacher"], inp["mask"], grad=grad)
     check(got, want, inp["mask"], dtype, 48, 3000)
+
+
+@pytest.mark.parametrize("V,cl", [(40008, 0), (16, 8), (8, 2)], ids=["five_slots_last_partial", "empty_slices",
+                                                                  "one_vector"])
+def test_resident_slices(V, cl):
+    # The register-resident kernel's edges: a slice of several 8 KB slots whose last
+    # slot is partial (V = 40008 takes two CTAs of 20008 columns), and clusters whose
+    # last CTAs own no columns at all; many rows per cluster with masked rows between.
+    m = pl()
+    inp = synth.reverse_kl_inputs(3, 70, V, torch.bfloat16, synth.seed_for(50, V))
+    mask = inp["mask"].reshape(-1).clone()
+    mask[:3] = 0
+    mask[50:90] = 0
+    mask = mask.reshape(3, 70)
+    want = oracle.reverse_kl(inp["student"], inp["teacher"], mask)
+    assert m.pl_debug_set_rkl_cluster(cl) == 0
+    try:
+        got = run(inp["student"], inp["teacher"], mask)
+    finally:
+        m.pl_debug_set_rkl_cluster(0)
+    check(got, want, mask, torch.bfloat16, 210, V)

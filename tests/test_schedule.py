@@ -1,20 +1,24 @@
 """Host-side checks of the persistent GEMM's tile schedule (no GPU needed).
 
 Every tile must run on exactly one CTA pair, and for the backward launch (a few
-long dX tiles with K = V next to many short dW tiles) the k-steps per pair must
-be balanced to within one long tile's share of the ideal.
+long dX tiles with K = V next to many short dW tiles) the load per pair -- each
+tile's k-steps plus the fixed hand-off cost of 8 k-steps the schedule counts --
+must be balanced to within one short tile of the ideal.  The backward launch's
+K split of its dX problem runs only when asked for.
 """
 import pytest
 
 import rl_post_policy_b200 as pl
 
+HANDOFF = 8  # k-steps the schedule adds per tile
 
-def loads(t0, t1, c0, c1, pairs):
+
+def loads(t0, t1, c0, c1, pairs, handoff=HANDOFF):
     rc, owner = pl.pl_debug_pair_tiles(t0, t1, c0, c1, pairs)
     assert rc == 0
     per = [0] * pairs
     for t, q in enumerate(owner):
-        per[q] += c0 if t < t0 else c1
+        per[q] += (c0 if t < t0 else c1) + handoff
     return per
 
 
@@ -31,19 +35,24 @@ def loads(t0, t1, c0, c1, pairs):
     (0, 7, 1, 1, 3),
 ])
 def test_every_tile_runs_once(t0, t1, c0, c1, pairs):
-    per = loads(t0, t1, c0, c1, pairs)
+    per = loads(t0, t1, c0, c1, pairs, handoff=0)
     assert sum(per) == t0 * c0 + t1 * c1
 
 
-def test_backward_schedule_is_balanced():
-    t0, t1, c0, c1, pairs = 64, 8016, 2004, 16, 74
+@pytest.mark.parametrize("t0,t1,c0,c1", [
+    (64, 8016, 2004, 16),    # 256-wide backward of a 1024-row chunk
+    (64, 4008, 2004, 32),    # 512-wide, dX split in two K halves (k-steps per N=256 MMA group)
+    (64, 4752, 2376, 32),    # the same at V=152064, H=4000
+])
+def test_backward_schedule_is_balanced(t0, t1, c0, c1):
+    pairs = 74
     per = loads(t0, t1, c0, c1, pairs)
-    ideal = (t0 * c0 + t1 * c1) / pairs
-    assert max(per) <= ideal + c1        # within one short tile of the ideal
-    # plain round-robin would leave the dX pairs ~8% over the ideal
+    ideal = (t0 * (c0 + HANDOFF) + t1 * (c1 + HANDOFF)) / pairs
+    assert max(per) <= ideal + c1 + HANDOFF        # within one short tile of the ideal
+    # plain round-robin would leave the dX pairs over the ideal
     rr = [0] * pairs
     for t in range(t0 + t1):
-        rr[t % pairs] += c0 if t < t0 else c1
+        rr[t % pairs] += (c0 if t < t0 else c1) + HANDOFF
     assert max(per) < max(rr)
 
 
@@ -69,14 +78,39 @@ def test_pick_tile_rejects_bad_input():
 
 
 def test_wide_backward_schedule_is_within_one_short_tile_of_its_longest_tile():
-    # at 512-wide tiles a dX tile (4008 units) exceeds the fair share (about 3466): the
-    # makespan cannot go below one dX tile, and the schedule stays within one dW tile of it
+    # without the K split, a 512-wide dX tile (4008 units) exceeds the fair share (about
+    # 3900 with the hand-off cost): the makespan cannot go below one dX tile, and the
+    # schedule stays within one dW tile of it
     t0, t1, c0, c1, pairs = 32, 4008, 4008, 32, 74
-    rc, owner = pl.pl_debug_pair_tiles(t0, t1, c0, c1, pairs)
-    assert rc == 0
-    per = [0] * pairs
-    for t, q in enumerate(owner):
-        per[q] += c0 if t < t0 else c1
-    assert max(per) <= c0 + c1
+    per = loads(t0, t1, c0, c1, pairs)
+    assert max(per) <= c0 + c1 + 2 * HANDOFF
     rest = per[t0:]
-    assert max(rest) - min(rest) <= c1
+    assert max(rest) - min(rest) <= c1 + HANDOFF
+
+
+@pytest.mark.parametrize("name,problems,want_nh", [
+    ("1024-row chunk", [(1024, 4096, 128256), (128256, 4096, 1024)], 2),
+    ("1024-row chunk, V=152064, H=4000", [(1024, 4000, 152064), (152064, 4000, 1024)], 2),
+    ("whole 8192-row batch", [(8192, 4096, 128256), (128256, 4096, 8192)], 2),
+    ("square", [(4096, 4096, 4096), (4096, 4096, 4096)], 2),
+    ("K of one step", [(1024, 1024, 64), (64, 1024, 1024)], 1),
+])
+def test_backward_k_split_is_off_unless_asked(name, problems, want_nh):
+    # measured no faster on the fused backward launch, the split runs only on request
+    assert pl.pl_debug_pick_split(problems, 74) == (1, want_nh), name
+
+
+def test_k_split_knob_forces_either_choice():
+    problems = [(1024, 4096, 128256), (128256, 4096, 1024)]
+    try:
+        assert pl.pl_debug_set_gemm_split(2) == 0
+        assert pl.pl_debug_pick_split(problems, 74) == (2, 2)
+        assert pl.pl_debug_pick_split([(4096, 4096, 4096), (4096, 4096, 4096)], 74)[0] == 2
+        # a single k-step has no halves
+        assert pl.pl_debug_pick_split([(1024, 1024, 64), (64, 1024, 1024)], 74)[0] == 1
+        assert pl.pl_debug_set_gemm_split(1) == 0
+        assert pl.pl_debug_pick_split(problems, 74)[0] == 1
+        assert pl.pl_debug_set_gemm_split(3) != 0
+    finally:
+        pl.pl_debug_set_gemm_split(0)
+    assert pl.pl_debug_pick_split([(1, 1, 1)], 74)[0] == -1
