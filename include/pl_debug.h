@@ -138,6 +138,25 @@ int pl_debug_pick_split(const int64_t* mnk, int pairs, int* nh_out);
  */
 int pl_debug_set_gemm_split(int mode);
 
+/*
+ * Fused path with several row chunks: 0 (the default) = chunk c's backward GEMM
+ * and chunk c+1's forward GEMM share one launch, whose CTA pairs claim tiles from
+ * a queue (dX tiles first, then the forward tiles interleaved with the dW
+ * tiles), with 8 epilogue warps; 1 = separate launches; 2 = shared launches with
+ * 4 epilogue warps.  Applies to later calls on this process.  Returns
+ * PL_ERR_ARG for another value.
+ */
+int pl_debug_set_gemm_merge(int mode);
+
+/*
+ * The GEMM's dynamic tile-queue order (host logic): jobs of tiles[0..njobs)
+ * tiles, numbered in job order; queue entry q runs tile out[q].  The tiles of
+ * jobs [0, q_f0) come first in order, then those of jobs [q_f0, q_w) spread
+ * evenly between those of job q_w (q_w < 0: every tile in order).  Returns 0,
+ * or -1 on bad input.
+ */
+int pl_debug_queue_tiles(int njobs, const int32_t* tiles, int q_f0, int q_w, int32_t* out);
+
 /* Number of kernels this library has launched in this process. */
 int64_t pl_debug_launch_count(void);
 

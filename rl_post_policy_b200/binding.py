@@ -98,6 +98,10 @@ _lib.pl_debug_set_gemm_tile.argtypes = [_I]
 _lib.pl_debug_set_gemm_tile.restype = _I
 _lib.pl_debug_set_rkl_cluster.argtypes = [_I]
 _lib.pl_debug_set_rkl_cluster.restype = _I
+_lib.pl_debug_set_gemm_merge.argtypes = [_I]
+_lib.pl_debug_set_gemm_merge.restype = _I
+_lib.pl_debug_queue_tiles.argtypes = [_I, _P, _I, _I, _P]
+_lib.pl_debug_queue_tiles.restype = _I
 _lib.pl_debug_set_rkl_path.argtypes = [_I]
 _lib.pl_debug_set_rkl_path.restype = _I
 _lib.pl_debug_pick_split.argtypes = [_P, _I, _P]
@@ -113,7 +117,7 @@ EXPORTED = ("pl_init", "pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_line
             "pl_version", "pl_debug_gemm", "pl_debug_gemm_out", "pl_debug_timing", "pl_debug_timing_read",
             "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_set_gemm_tile", "pl_debug_pair_tiles",
             "pl_debug_pick_tile", "pl_debug_set_loss_path", "pl_debug_pick_split", "pl_debug_set_gemm_split",
-            "pl_debug_set_rkl_path")
+            "pl_debug_set_rkl_path", "pl_debug_set_gemm_merge", "pl_debug_queue_tiles")
 
 
 class PLError(RuntimeError):
@@ -322,6 +326,21 @@ def pl_debug_set_rkl_path(path: int) -> int:
     """Test hook: reverse KL with a gradient -- 0 the default (the streaming kernel), 1 the
     streaming kernel, 2 the register-resident kernel where it applies."""
     return int(_lib.pl_debug_set_rkl_path(int(path)))
+
+
+def pl_debug_set_gemm_merge(mode: int) -> int:
+    """Test hook: several-chunk fused calls -- 0 merged backward/forward launches (default),
+    1 separate launches, 2 merged launches with 4 epilogue warps."""
+    return int(_lib.pl_debug_set_gemm_merge(int(mode)))
+
+
+def pl_debug_queue_tiles(tiles, q_f0: int, q_w: int):
+    """Test hook: the GEMM's dynamic tile-queue order for jobs of the given tile counts."""
+    n = int(sum(tiles))
+    arr = (ctypes.c_int32 * max(len(tiles), 1))(*[int(t) for t in tiles])
+    out = (ctypes.c_int32 * max(n, 1))()
+    rc = int(_lib.pl_debug_queue_tiles(len(tiles), arr, int(q_f0), int(q_w), out))
+    return rc, list(out)[:n]
 
 
 def pl_debug_set_gemm_split(mode: int) -> int:

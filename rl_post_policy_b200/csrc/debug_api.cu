@@ -84,6 +84,33 @@ extern "C" int pl_debug_pick_split(const int64_t* mnk, int pairs, int* nh_out) {
   return split;
 }
 
+extern "C" int pl_debug_set_gemm_merge(int mode) {
+  if (mode < 0 || mode > 2) return PL_ERR_ARG;
+  debug_knobs().gemm_merge = mode;
+  return PL_OK;
+}
+
+// pl_debug_queue_tiles: the dynamic tile queue's order for jobs of the given
+// tile counts (leading jobs [0, q_f0), then jobs [q_f0, q_w) interleaved with
+// job q_w; q_w < 0: job order).  out[q] receives the global tile id of entry q.
+extern "C" int pl_debug_queue_tiles(int njobs, const int32_t* tiles, int q_f0, int q_w, int32_t* out) {
+  if (njobs < 1 || njobs > kMaxJobs || !tiles || !out) return -1;
+  if (q_w >= njobs || (q_w >= 0 && (q_f0 < 0 || q_f0 > q_w))) return -1;
+  GemmParams p{};
+  p.njobs = njobs;
+  int begin = 0;
+  for (int i = 0; i < njobs; ++i) {
+    if (tiles[i] < 0) return -1;
+    p.jobs[i].tile_begin = begin;
+    begin += tiles[i];
+  }
+  p.total_tiles = begin;
+  p.q_f0 = q_f0;
+  p.q_w = q_w;
+  for (int q = 0; q < begin; ++q) out[q] = queue_tile(p, q);
+  return 0;
+}
+
 extern "C" int pl_debug_set_gemm_split(int mode) {
   if (mode < 0 || mode > 2) return PL_ERR_ARG;
   debug_knobs().gemm_split = mode;

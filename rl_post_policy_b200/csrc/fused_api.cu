@@ -28,7 +28,7 @@ namespace {
 int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
-  int64_t N = 0, C = 1024, Cbuf = 1, nchunks = 0, ld = 0;
+  int64_t N = 0, C = 1024, Cbuf = 1, nchunks = 0, ld = 0, logits_bytes = 0;
   int ntv = 0, nparts = 0, part_stride = 1;  // 256-column vocabulary tiles; LSE partials per row
   FusedOffsets off{};
 };
@@ -65,7 +65,10 @@ Plan make_plan(int64_t bs, int64_t T, int64_t H, int64_t V, uint32_t mode, bool 
   p.off.zt_ref = region(4 * p.Cbuf);
   p.off.part = region(8 * p.Cbuf * (int64_t)p.nparts);
   p.off.part_ref = region(8 * p.Cbuf * (int64_t)p.nparts);
-  p.off.logits = region(2 * p.Cbuf * p.ld);
+  // two halves when several chunks run with a backward: chunk c's backward and
+  // chunk c+1's forward share a launch (see run_pipeline)
+  p.logits_bytes = align_up(2 * p.Cbuf * p.ld, 1024);
+  p.off.logits = region(p.logits_bytes * (p.nchunks > 1 ? 2 : 1));
   p.off.dw_acc = region((need_dW && p.nchunks > 1) ? 4 * V * H : 0);
   p.off.dx_acc = region(4 * p.Cbuf * (H > 0 ? H : 0));
   p.off.db_acc = region((need_dbias && p.nchunks > 1) ? 4 * V : 0);
@@ -147,158 +150,229 @@ pl_status run_pipeline(const Pipe& q) {
 
   const unsigned char* Xb = static_cast<const unsigned char*>(X);
   const unsigned char* Xrb = static_cast<const unsigned char*>(Xref);
-  int last_blocks = 0;
-  for (int64_t c = 0; c < plan.nchunks; ++c) {
-    const int64_t r0 = c * plan.C;
-    const int64_t rows = (N - r0) < plan.C ? (N - r0) : plan.C;
+  const bool has_gemm_bwd = need_bwd && (dX || dW);
+  // Several chunks with a backward GEMM: chunk c's backward and chunk c+1's
+  // forward share one launch (their tiles do not depend on each other), so the
+  // memory-heavy dW tiles with their fp32 accumulator adds run beside the
+  // compute-heavy forward tiles, and each launch's tail is paid once.  The two
+  // chunks' logits live in alternate halves of the logits region.
+  const bool merge = has_gemm_bwd && plan.nchunks > 1 && debug_knobs().gemm_merge != 1;
+  auto logits_of = [&](int64_t c) -> unsigned char* {
+    return ws + plan.off.logits + (merge ? (c & 1) * plan.logits_bytes : 0);
+  };
+  auto rows_of = [&](int64_t c) -> int64_t { return (N - c * plan.C) < plan.C ? (N - c * plan.C) : plan.C; };
 
-    // ---- forward GEMM(s): reference then policy logits tiles ----
-    GemmParams fp{};
-    fp.err = reinterpret_cast<unsigned*>(ws);
-    fp.wait_ns = kWaitLimitNs;
-    int nj = 0;
+  // Chunk c's forward jobs (reference, then policy) appended to g; maps from *nm.
+  auto add_fwd = [&](GemmParams& g, int64_t c, int& nm) -> bool {
+    const int64_t r0 = c * plan.C, rows = rows_of(c);
     if (has_kl) {
-      if (!make_tmap_2d(&fp.maps[0], Xrb + r0 * H * esz, dt, H, rows, H * esz, kBK, kBM) ||
-          !make_tmap_2d(&fp.maps[1], Wref, dt, H, V, H * esz, kBK, kBNh))
-        return PL_ERR_CUDA;
-      GemmJob& j = fp.jobs[nj++];
-      j.a_map = 0; j.b_map = 1; j.a_mn = 0; j.b_mn = 0;
+      const int ma = nm++, mb = nm++;
+      if (!make_tmap_2d(&g.maps[ma], Xrb + r0 * H * esz, dt, H, rows, H * esz, kBK, kBM) ||
+          !make_tmap_2d(&g.maps[mb], Wref, dt, H, V, H * esz, kBK, kBNh))
+        return false;
+      GemmJob& j = g.jobs[g.njobs++];
+      j.a_map = ma; j.b_map = mb; j.a_mn = 0; j.b_mn = 0;
       j.M = (int)rows; j.N = (int)V; j.K = (int)H; j.n_inner = 0; j.epi = kEpiLse;
       j.bias = nullptr; j.targets = targets + r0;
       j.part = reinterpret_cast<float2*>(ws + plan.off.part_ref); j.part_ld = plan.nparts;
       j.zt = reinterpret_cast<float*>(ws + plan.off.zt_ref); j.logits = nullptr;
       j.logit_scale = q.inv_temp;
     }
-    if (!make_tmap_2d(&fp.maps[2], Xb + r0 * H * esz, dt, H, rows, H * esz, kBK, kBM) ||
-        !make_tmap_2d(&fp.maps[3], W, dt, H, V, H * esz, kBK, kBNh))
-      return PL_ERR_CUDA;
-    {
-      GemmJob& j = fp.jobs[nj++];
-      j.a_map = 2; j.b_map = 3; j.a_mn = 0; j.b_mn = 0;
-      j.M = (int)rows; j.N = (int)V; j.K = (int)H; j.n_inner = 0; j.epi = kEpiLse;
-      j.bias = bias; j.targets = targets + r0;
-      j.part = reinterpret_cast<float2*>(ws + plan.off.part); j.part_ld = plan.nparts;
-      j.zt = reinterpret_cast<float*>(ws + plan.off.zt);
-      j.logits = need_bwd ? ws + plan.off.logits : nullptr; j.logits_ld = plan.ld;
-      j.logit_scale = q.inv_temp;
-      if (j.logits) {
-        // the chunk's [rows, V] logits, written by TMA stores from the epilogue
-        if (!make_tmap_2d(&fp.maps[4], ws + plan.off.logits, dt, V, rows, plan.ld * esz, kOutBoxN16, kOutBoxM))
-          return PL_ERR_CUDA;
-        j.out_path = kOutTmaStore; j.out_map = 4;
-      }
+    const int ma = nm++, mb = nm++;
+    if (!make_tmap_2d(&g.maps[ma], Xb + r0 * H * esz, dt, H, rows, H * esz, kBK, kBM) ||
+        !make_tmap_2d(&g.maps[mb], W, dt, H, V, H * esz, kBK, kBNh))
+      return false;
+    GemmJob& j = g.jobs[g.njobs++];
+    j.a_map = ma; j.b_map = mb; j.a_mn = 0; j.b_mn = 0;
+    j.M = (int)rows; j.N = (int)V; j.K = (int)H; j.n_inner = 0; j.epi = kEpiLse;
+    j.bias = bias; j.targets = targets + r0;
+    j.part = reinterpret_cast<float2*>(ws + plan.off.part); j.part_ld = plan.nparts;
+    j.zt = reinterpret_cast<float*>(ws + plan.off.zt);
+    j.logits = need_bwd ? logits_of(c) : nullptr; j.logits_ld = plan.ld;
+    j.logit_scale = q.inv_temp;
+    if (j.logits) {
+      // the chunk's [rows, V] logits, written by TMA stores from the epilogue
+      const int mo = nm++;
+      if (!make_tmap_2d(&g.maps[mo], j.logits, dt, V, rows, plan.ld * esz, kOutBoxN16, kOutBoxM)) return false;
+      j.out_path = kOutTmaStore; j.out_map = mo;
     }
-    fp.njobs = nj;
-    gemm_finalize_jobs(&fp);
-    if (!ok(launch_gemm(fp, dt, s))) return PL_ERR_CUDA;
+    return true;
+  };
 
-    // ---- combine: lse, logp, loss partials, g ----
+  // Chunk c's dX job (rows of this chunk = dz W), appended to g.
+  auto add_dx = [&](GemmParams& g, int64_t c, int& nm) -> bool {
+    const int64_t r0 = c * plan.C, rows = rows_of(c);
+    const int ma = nm++, mb = nm++;
+    if (!make_tmap_2d(&g.maps[ma], logits_of(c), dt, V, rows, plan.ld * esz, kBK, kBM) ||
+        !make_tmap_2d(&g.maps[mb], W, dt, H, V, H * esz, 64, kBK))
+      return false;
+    GemmJob& j = g.jobs[g.njobs++];
+    j.a_map = ma; j.b_map = mb; j.a_mn = 0; j.b_mn = 1;
+    j.M = (int)rows; j.N = (int)H; j.K = (int)V; j.n_inner = 0; j.epi = kEpiStore;
+    j.out = static_cast<unsigned char*>(dX) + r0 * H * esz; j.out_f32 = 0; j.acc_in = nullptr;
+    j.out_ld = H; j.scale = reinterpret_cast<const float*>(ws + plan.off.inv_scale) + c;
+    // whole 128-byte lines through the TMA unit when dX is 16-byte aligned
+    if (aligned(dX, 16)) {
+      const int mo = nm++;
+      if (!make_tmap_2d(&g.maps[mo], j.out, dt, H, rows, H * esz, kOutBoxN16, kOutBoxM)) return false;
+      j.out_path = kOutTmaStore; j.out_map = mo;
+    }
+    return true;
+  };
+
+  // Chunk c's dW contribution (dz^T X_chunk), appended to g.  Several chunks:
+  // the first stores its fp32 contribution, every later one adds its own
+  // through the TMA unit (the memory system does the add, so the epilogue never
+  // waits on a load), and the sum is rounded to the model dtype once, after the
+  // last chunk.
+  auto add_dw = [&](GemmParams& g, int64_t c, int& nm) -> bool {
+    const int64_t r0 = c * plan.C, rows = rows_of(c);
+    const int ma = nm++, mb = nm++, mo = nm++;
+    if (!make_tmap_2d(&g.maps[ma], logits_of(c), dt, V, rows, plan.ld * esz, 64, kBK) ||
+        !make_tmap_2d(&g.maps[mb], Xb + r0 * H * esz, dt, H, rows, H * esz, 64, kBK))
+      return false;
+    GemmJob& j = g.jobs[g.njobs++];
+    j.a_map = ma; j.b_map = mb; j.a_mn = 1; j.b_mn = 1;
+    j.M = (int)V; j.N = (int)H; j.K = (int)rows; j.n_inner = 1; j.epi = kEpiStore;
+    j.out_ld = H; j.scale = reinterpret_cast<const float*>(ws + plan.off.inv_scale) + c;
+    float* acc = reinterpret_cast<float*>(ws + plan.off.dw_acc);
+    j.acc_in = nullptr;
+    if (plan.nchunks == 1) {
+      j.out = dW; j.out_f32 = 0; j.out_path = kOutDirect;
+      if (aligned(dW, 16)) {
+        if (!make_tmap_2d(&g.maps[mo], dW, dt, H, V, H * esz, kOutBoxN16, kOutBoxM)) return false;
+        j.out_path = kOutTmaStore; j.out_map = mo;
+      }
+    } else {
+      if (!make_tmap_2d(&g.maps[mo], acc, DType::F32, H, V, H * 4, kOutBoxN, kOutBoxM)) return false;
+      j.out = acc; j.out_f32 = 1; j.out_map = mo;
+      j.out_path = c == 0 ? kOutTmaStore : kOutTmaReduce;
+    }
+    return true;
+  };
+
+  int last_blocks = 0;
+  auto combine = [&](int64_t c) -> bool {
+    const int64_t rows = rows_of(c);
     CombineArgs ca{};
     ca.ws = ws; ca.off = plan.off; ca.targets = targets; ca.old_lp = old_lp; ca.adv = adv; ca.mask = mask;
     ca.logp_out = logp_out; ca.ref_logp_out = ref_logp_out;
-    ca.row0 = r0; ca.rows = rows; ca.bs = bs; ca.T = T; ca.V = V; ca.nparts = plan.nparts;
+    ca.row0 = c * plan.C; ca.rows = rows; ca.bs = bs; ca.T = T; ca.V = V; ca.nparts = plan.nparts;
     ca.chunk = (int)c; ca.part_stride = plan.part_stride;
     ca.lo = 1.0f - eps_lo; ca.hi = 1.0f + eps_hi; ca.beta = beta;
     ca.grpo = (mode & PL_REDUCTION_MASK) == PL_GRPO; ca.adv_lp_dtype = (mode & PL_ADV_LP_DTYPE) != 0;
     ca.bf16 = dt == DType::BF16;
     ca.grad_logp = q.grad_logp;
     ca.g_scale = q.inv_temp;
-    if (q.ext_g) {
-      if (!ok(launch_combine_ext(ca, s))) return PL_ERR_CUDA;
-    } else if (!ok(launch_combine(ca, has_kl, two_sided, s))) {
-      return PL_ERR_CUDA;
-    }
     last_blocks = (int)((rows + 7) / 8);
-
-    if (!need_bwd) continue;
-
-    // ---- dlogits in place (+ dbias) ----
+    return ok(q.ext_g ? launch_combine_ext(ca, s) : launch_combine(ca, has_kl, two_sided, s));
+  };
+  auto dlogits = [&](int64_t c) -> bool {
     DlogitsArgs da{};
-    da.ws = ws; da.off = plan.off; da.targets = targets; da.logits = ws + plan.off.logits; da.ld = plan.ld;
-    da.row0 = r0; da.rows = rows; da.V = V; da.chunk = (int)c;
+    da.ws = ws; da.off = plan.off; da.targets = targets; da.logits = logits_of(c); da.ld = plan.ld;
+    da.row0 = c * plan.C; da.rows = rows_of(c); da.V = V; da.chunk = (int)c;
     da.dbias_mode = dbias ? acc_mode(c, plan.nchunks) : kAccNone;
     da.dbias_acc = reinterpret_cast<float*>(ws + plan.off.db_acc); da.dbias = dbias;
     da.db_part = reinterpret_cast<float*>(ws + plan.off.db_part);
     da.db_cnt = reinterpret_cast<unsigned*>(ws + plan.off.db_cnt);
-    if (!ok(launch_dlogits(da, dt, s))) return PL_ERR_CUDA;
-
-    if (!dX && !dW) continue;
-
-    // ---- backward GEMMs: dX rows of this chunk, dW contribution ----
-    GemmParams bp{};
-    bp.err = reinterpret_cast<unsigned*>(ws);
-    bp.wait_ns = kWaitLimitNs;
-    nj = 0;
-    const float* inv_scale = reinterpret_cast<const float*>(ws + plan.off.inv_scale) + c;
-    if (dX) {
-      if (!make_tmap_2d(&bp.maps[0], ws + plan.off.logits, dt, V, rows, plan.ld * esz, kBK, kBM) ||
-          !make_tmap_2d(&bp.maps[1], W, dt, H, V, H * esz, 64, kBK))
-        return PL_ERR_CUDA;
-      GemmJob& j = bp.jobs[nj++];
-      j.a_map = 0; j.b_map = 1; j.a_mn = 0; j.b_mn = 1;
-      j.M = (int)rows; j.N = (int)H; j.K = (int)V; j.n_inner = 0; j.epi = kEpiStore;
-      j.out = static_cast<unsigned char*>(dX) + r0 * H * esz; j.out_f32 = 0; j.acc_in = nullptr;
-      j.out_ld = H; j.scale = inv_scale;
-      // whole 128-byte lines through the TMA unit when dX is 16-byte aligned
-      if (aligned(dX, 16)) {
-        if (!make_tmap_2d(&bp.maps[5], j.out, dt, H, rows, H * esz, kOutBoxN16, kOutBoxM)) return PL_ERR_CUDA;
-        j.out_path = kOutTmaStore; j.out_map = 5;
-      }
-    }
-    if (dW) {
-      if (!make_tmap_2d(&bp.maps[2], ws + plan.off.logits, dt, V, rows, plan.ld * esz, 64, kBK) ||
-          !make_tmap_2d(&bp.maps[3], Xb + r0 * H * esz, dt, H, rows, H * esz, 64, kBK))
-        return PL_ERR_CUDA;
-      GemmJob& j = bp.jobs[nj++];
-      j.a_map = 2; j.b_map = 3; j.a_mn = 1; j.b_mn = 1;
-      j.M = (int)V; j.N = (int)H; j.K = (int)rows; j.n_inner = 1; j.epi = kEpiStore;
-      j.out_ld = H; j.scale = inv_scale;
-      // Several chunks: the first stores its fp32 contribution, every later one
-      // adds its own through the TMA unit (the memory system does the add, so
-      // the epilogue never waits on a load), and the sum is rounded to the
-      // model dtype once, after the last chunk.
-      float* acc = reinterpret_cast<float*>(ws + plan.off.dw_acc);
-      j.acc_in = nullptr;
-      if (plan.nchunks == 1) {
-        j.out = dW; j.out_f32 = 0; j.out_path = kOutDirect;
-        if (aligned(dW, 16)) {
-          if (!make_tmap_2d(&bp.maps[4], dW, dt, H, V, H * esz, kOutBoxN16, kOutBoxM)) return PL_ERR_CUDA;
-          j.out_path = kOutTmaStore; j.out_map = 4;
-        }
-      } else {
-        if (!make_tmap_2d(&bp.maps[4], acc, DType::F32, H, V, H * 4, kOutBoxN, kOutBoxM)) return PL_ERR_CUDA;
-        j.out = acc; j.out_f32 = 1; j.out_map = 4;
-        j.out_path = c == 0 ? kOutTmaStore : kOutTmaReduce;
-      }
-    }
-    bp.njobs = nj;
+    return ok(launch_dlogits(da, dt, s));
+  };
+  auto fresh = [&]() {
+    GemmParams g{};
+    g.err = reinterpret_cast<unsigned*>(ws);
+    g.wait_ns = kWaitLimitNs;
+    g.q_w = -1;
+    return g;
+  };
+  // dX has K = V: a test or measurement may ask for each dX tile to be computed
+  // as two tiles over the halves of the vocabulary, both adding their fp32
+  // result into a zeroed buffer through the TMA unit (two addends onto zero: the
+  // sum does not depend on their order), which one pass then rounds into dX.
+  float* dx_acc = reinterpret_cast<float*>(ws + plan.off.dx_acc);
+  auto launch_backward_alone = [&](GemmParams& bp, int64_t c) -> bool {
+    const int64_t r0 = c * plan.C, rows = rows_of(c);
     gemm_finalize_jobs(&bp);
-    // dX has K = V: its few long tiles would finish last next to the many short
-    // dW tiles.  When the schedule estimate says so, each dX tile is computed as
-    // two tiles over the halves of the vocabulary, both adding their fp32 result
-    // into a zeroed buffer through the TMA unit (two addends onto zero: the sum
-    // does not depend on their order), which one pass then rounds into dX.
     int dx_split = 1;
-    float* dx_acc = reinterpret_cast<float*>(ws + plan.off.dx_acc);
     if (dX) {
       DevInfo di;
-      if (dev_info(&di) != cudaSuccess) return PL_ERR_CUDA;
+      if (dev_info(&di) != cudaSuccess) return false;
       dx_split = gemm_choose_k_split(&bp, 0, di.sm_count / 2);
     }
     if (dx_split == 2) {
       GemmJob& j = bp.jobs[0];
-      if (!make_tmap_2d(&bp.maps[5], dx_acc, DType::F32, H, rows, H * 4, kOutBoxN, kOutBoxM)) return PL_ERR_CUDA;
-      j.out = dx_acc; j.out_f32 = 1; j.out_path = kOutTmaReduce; j.out_map = 5; j.out_ld = H;
-      if (!ok(cudaMemsetAsync(dx_acc, 0, (size_t)rows * H * 4, s))) return PL_ERR_CUDA;
+      const int mo = kMaxMaps - 1;
+      if (!make_tmap_2d(&bp.maps[mo], dx_acc, DType::F32, H, rows, H * 4, kOutBoxN, kOutBoxM)) return false;
+      j.out = dx_acc; j.out_f32 = 1; j.out_path = kOutTmaReduce; j.out_map = mo; j.out_ld = H;
+      if (!ok(cudaMemsetAsync(dx_acc, 0, (size_t)rows * H * 4, s))) return false;
     }
-    if (!ok(launch_gemm(bp, dt, s))) return PL_ERR_CUDA;
+    if (!ok(launch_gemm(bp, dt, s))) return false;
     if (dx_split == 2 &&
         !ok(launch_convert(dx_acc, static_cast<unsigned char*>(dX) + r0 * H * esz, rows * H, dt, s)))
-      return PL_ERR_CUDA;
-    if (dW && plan.nchunks > 1 && c + 1 == plan.nchunks &&
-        !ok(launch_convert(reinterpret_cast<const float*>(ws + plan.off.dw_acc), dW, V * H, dt, s)))
-      return PL_ERR_CUDA;
+      return false;
+    return true;
+  };
+
+  if (!merge) {
+    for (int64_t c = 0; c < plan.nchunks; ++c) {
+      // ---- forward GEMM(s): reference then policy logits tiles ----
+      GemmParams fp = fresh();
+      int nm = 0;
+      if (!add_fwd(fp, c, nm)) return PL_ERR_CUDA;
+      gemm_finalize_jobs(&fp);
+      if (!ok(launch_gemm(fp, dt, s))) return PL_ERR_CUDA;
+      // ---- combine: lse, logp, loss partials, g ----
+      if (!combine(c)) return PL_ERR_CUDA;
+      if (!need_bwd) continue;
+      // ---- dlogits in place (+ dbias) ----
+      if (!dlogits(c)) return PL_ERR_CUDA;
+      if (!dX && !dW) continue;
+      // ---- backward GEMMs: dX rows of this chunk, dW contribution ----
+      GemmParams bp = fresh();
+      nm = 0;
+      if ((dX && !add_dx(bp, c, nm)) || (dW && !add_dw(bp, c, nm))) return PL_ERR_CUDA;
+      if (!launch_backward_alone(bp, c)) return PL_ERR_CUDA;
+    }
+  } else {
+    // chunk 0's forward alone, then [backward c + forward c+1] launches
+    {
+      GemmParams fp = fresh();
+      int nm = 0;
+      if (!add_fwd(fp, 0, nm)) return PL_ERR_CUDA;
+      gemm_finalize_jobs(&fp);
+      if (!ok(launch_gemm(fp, dt, s))) return PL_ERR_CUDA;
+      if (!combine(0) || !dlogits(0)) return PL_ERR_CUDA;
+    }
+    for (int64_t c = 0; c < plan.nchunks; ++c) {
+      GemmParams g = fresh();
+      int nm = 0;
+      if (c + 1 < plan.nchunks) {
+        // queue order: dX tiles (long, K = V) first, then the next chunk's
+        // forward tiles interleaved evenly with this chunk's dW tiles
+        if (dX && !add_dx(g, c, nm)) return PL_ERR_CUDA;
+        g.q_f0 = g.njobs;
+        if (!add_fwd(g, c + 1, nm)) return PL_ERR_CUDA;
+        if (dW) {
+          g.q_w = g.njobs;
+          if (!add_dw(g, c, nm)) return PL_ERR_CUDA;
+        }
+        g.dyn = 1;
+        g.ctr = reinterpret_cast<unsigned*>(ws + kWsGemmQueue);
+        g.ctr_done = g.ctr + 1;
+        bool wide = true;
+        for (int i = 0; i < g.njobs; ++i) wide = wide && g.jobs[i].N >= 2 * kBN;
+        g.nh = wide ? 2 : 1;
+        gemm_finalize_jobs(&g);
+        if (!ok(launch_gemm(g, dt, s))) return PL_ERR_CUDA;
+        if (!combine(c + 1) || !dlogits(c + 1)) return PL_ERR_CUDA;
+      } else {
+        if ((dX && !add_dx(g, c, nm)) || (dW && !add_dw(g, c, nm))) return PL_ERR_CUDA;
+        if (!launch_backward_alone(g, c)) return PL_ERR_CUDA;
+      }
+    }
   }
+  if (dW && plan.nchunks > 1 &&
+      !ok(launch_convert(reinterpret_cast<const float*>(ws + plan.off.dw_acc), dW, V * H, dt, s)))
+    return PL_ERR_CUDA;
 
   if (q.ext_g) return PL_OK;
   if (!ok(launch_finalize(ws, plan.off, (int)plan.nchunks, plan.part_stride, last_blocks, loss, n_valid_out, s)))

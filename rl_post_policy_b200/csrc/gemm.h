@@ -82,11 +82,24 @@ struct GemmJob {
   const float* scale;      // device scalar multiplier, or null for 1
 };
 
+constexpr int kMaxJobs = 4;
+constexpr int kMaxMaps = 12;
+
 struct __align__(64) GemmParams {
-  CUtensorMap maps[6];
-  GemmJob jobs[2];
+  CUtensorMap maps[kMaxMaps];
+  GemmJob jobs[kMaxJobs];
   int njobs;
   int total_tiles;
+  // Dynamic tile queue (dyn = 1): the pairs claim tiles from a global counter
+  // (*ctr, zero before the launch; the last CTA to finish sets it and *ctr_done
+  // back to zero) in queue order: the tiles of jobs [0, q_f0) first, then the
+  // tiles of jobs [q_f0, q_w) interleaved evenly with those of job q_w (q_w < 0:
+  // no interleaving, every tile in job order).  Used for launches whose jobs
+  // differ in tile cost and in memory traffic: long tiles first, and
+  // memory-heavy tiles spread over the launch next to compute-heavy ones.
+  int dyn, q_f0, q_w;
+  unsigned* ctr;
+  unsigned* ctr_done;
   // Tile schedule (set by launch_gemm).  0: pair p takes tiles p, p+P, p+2P ...
   // 1: two jobs of very different tile cost -- pair p < T0 takes job-0 tile p,
   //    then every pair takes a contiguous run of job-1 tiles, `na` (p < T0) or
@@ -133,5 +146,7 @@ int gemm_choose_k_split(GemmParams* p, int job, int P);
 // sched/na/nb/rem for P pairs; pair_tile gives the i-th tile of a pair or -1.
 void balance_schedule(GemmParams* p, int P);
 __host__ __device__ int pair_tile(const GemmParams& p, int pair, int npairs, int i);
+// Global tile id of the q-th entry of the dynamic queue (see GemmParams::dyn).
+__host__ __device__ int queue_tile(const GemmParams& p, int q);
 
 }  // namespace pl

@@ -56,6 +56,7 @@ using namespace sm100;
 constexpr uint32_t kABytes = kBM * kBK * 2;             // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t kBBytes = kBNh * kBK * 2;            // 16 KB: this CTA's 128 rows of B per MMA
 constexpr uint32_t kTmemCols = 512;
+constexpr int kQSlots = 4;   // dynamic queue: tile ids in flight between the roles
 // Epilogue staging for the TMA output paths: 8 boxes of 4 KB (32 rows x 128
 // bytes), one per epilogue warp (8 warps) or two (4 warps).
 constexpr uint32_t kOutBoxBytes = kOutBoxM * kOutBoxN * 4;
@@ -110,7 +111,10 @@ struct TileCoord {
 // split job lists all tiles of its first K half, then all of the second.
 __device__ __forceinline__ TileCoord tile_coord(const GemmParams& p, int tile) {
   TileCoord c;
-  c.job = (p.njobs > 1 && tile >= p.jobs[1].tile_begin) ? 1 : 0;
+  c.job = 0;
+#pragma unroll
+  for (int q = 1; q < kMaxJobs; ++q)
+    if (q < p.njobs && tile >= p.jobs[q].tile_begin) c.job = q;
   const GemmJob& j = p.jobs[c.job];
   int local = tile - j.tile_begin;
   c.kb = 0;
@@ -152,6 +156,19 @@ __host__ __device__ int pair_tile(const GemmParams& p, int pair, int npairs, int
   const int hi = pair > T0 ? pair - T0 : 0;
   const int rm = pair < p.rem ? pair : p.rem;
   return T0 + lo * p.na + hi * p.nb + rm + k;
+}
+
+__host__ __device__ int queue_tile(const GemmParams& p, int q) {
+  if (p.q_w < 0) return q;
+  const int t_lead = p.jobs[p.q_f0].tile_begin;
+  if (q < t_lead) return q;
+  const long long qq = q - t_lead;
+  const long long tw_begin = p.jobs[p.q_w].tile_begin;
+  const long long tf = tw_begin - t_lead;
+  const long long r = (long long)p.total_tiles - t_lead;
+  const long long f0 = qq * tf / r, f1 = (qq + 1) * tf / r;
+  if (f1 > f0) return (int)(t_lead + f0);   // the f0-th tile of jobs [q_f0, q_w)
+  return (int)(tw_begin + (qq - f0));       // the (qq - f0)-th tile of job q_w
 }
 
 namespace {
@@ -236,6 +253,9 @@ __device__ __forceinline__ void add_bias32(const T* bias, float (&v)[32], int nv
 template <typename T, int NH, int EW>
 __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   static_assert(EW == 4 || EW == 8, "4 or 8 epilogue warps");
+  // readers of a dynamic-queue slot: the peer's producer, the MMA issuer and
+  // every epilogue warp of both CTAs
+  constexpr int kQReaders = 2 + 2 * EW;
   using Cfg = TileCfg<NH>;
   constexpr int kStages = Cfg::kStages;
   constexpr uint32_t kStageBytes = Cfg::kStageBytes;
@@ -248,7 +268,13 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  // dynamic queue (GemmParams::dyn): a ring of claimed tile ids, published by the
+  // leader's producer into both CTAs, each slot released by every role that reads it
+  uint64_t* qfull = done + 1;
+  uint64_t* qempty = qfull + kQSlots;
+  int* qring_raw = reinterpret_cast<int*>(qempty + kQSlots);
+  volatile int* qring = qring_raw;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qring_raw + kQSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -268,6 +294,10 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
       mbar_init(&tempty[b], 2 * EW * 32);  // both CTAs' epilogue threads release the leader's accumulator
     }
     mbar_init(done, 1);
+    for (int q = 0; q < kQSlots; ++q) {
+      mbar_init(&qfull[q], 1);                // the leader producer's arrival
+      mbar_init(&qempty[q], kQReaders);       // (leader only) every reader of the slot
+    }
     *abort_flag = 0;
     fence_barrier_init();
     for (int q = 0; q < p.njobs; ++q) {
@@ -287,13 +317,51 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
   const uint32_t tmem_base = *tmem_slot;
   const unsigned long long lim = p.wait_ns;
 
+  // ---- dynamic queue: entry `it` of this pair's tile sequence ----
+  // Readers wait for the leader producer's publication (acquire at cluster
+  // scope), take the id, and release the slot on the leader's barrier.
+  // Returns the tile (or -1: no more), or -2 when a wait ran out.
+  auto q_read = [&](int it) -> int {
+    const int slot = it % kQSlots;
+    const uint32_t par = (uint32_t)(it / kQSlots) & 1u;
+    if (!mbar_wait_cluster(&qfull[slot], par, abort_flag, lim)) return -2;
+    return qring[slot];
+  };
+  auto q_release = [&](int it) {
+    mbar_arrive_cluster(mapa_shared(smem_u32(&qempty[it % kQSlots]), 0));
+  };
+  // The leader producer: claim the next queue entry and publish its tile id in
+  // both CTAs once every reader has released the slot's previous entry.
+  auto q_claim = [&](int it) -> int {
+    const int slot = it % kQSlots;
+    const uint32_t par = (uint32_t)(it / kQSlots) & 1u;
+    const unsigned q = atomicAdd(p.ctr, 1u);
+    const int tile = q < (unsigned)p.total_tiles ? queue_tile(p, (int)q) : -1;
+    if (!mbar_wait_cluster(&qempty[slot], par ^ 1u, abort_flag, lim)) return -2;
+    qring[slot] = tile;
+    st_cluster_s32(mapa_shared(smem_u32(&qring_raw[slot]), 1), tile);
+    mbar_arrive(&qfull[slot]);
+    mbar_arrive_cluster(mapa_shared(smem_u32(&qfull[slot]), 1));
+    return tile;
+  };
+
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs; completions counted by the leader) ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       for (int it = 0; !*abort_flag; ++it) {
-        const int tile = pair_tile(p, pair, npairs, it);
+        int tile;
+        if (p.dyn) {
+          if (leader) {
+            tile = q_claim(it);
+          } else {
+            tile = q_read(it);
+            if (tile != -2) q_release(it);
+          }
+        } else {
+          tile = pair_tile(p, pair, npairs, it);
+        }
         if (tile < 0) break;
         const TileCoord tc = tile_coord(p, tile);
         const GemmJob& j = p.jobs[tc.job];
@@ -361,7 +429,13 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
         }
       };
       for (int it = 0; !*abort_flag; ++it) {
-        const int tile = pair_tile(p, pair, npairs, it);
+        int tile;
+        if (p.dyn) {
+          tile = q_read(it);
+          if (tile != -2) q_release(it);
+        } else {
+          tile = pair_tile(p, pair, npairs, it);
+        }
         if (tile < 0) break;
         const TileCoord tc = tile_coord(p, tile);
         const GemmJob& j = p.jobs[tc.job];
@@ -468,14 +542,18 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
     int acc = 0;
     uint32_t acc_phase = 0;
     constexpr float kLog2e = 1.4426950408889634f;
-    // the jobs' device scale factors, read once per launch rather than per tile
-    const float job_scale0 = p.jobs[0].scale ? __ldg(p.jobs[0].scale) : 1.0f;
-    const float job_scale1 = (p.njobs > 1 && p.jobs[1].scale) ? __ldg(p.jobs[1].scale) : 1.0f;
     // this warp's two staging boxes for the TMA output paths
     const uint32_t box0 = smem_u32(out_stage) + (uint32_t)((warp - 2) * kBoxes) * kOutBoxBytes;
     int sbuf = 0;
     for (int it = 0;; ++it) {
-      const int tile = pair_tile(p, pair, npairs, it);
+      int tile;
+      if (p.dyn) {
+        tile = q_read(it);
+        __syncwarp();
+        if (lane == 0 && tile != -2) q_release(it);
+      } else {
+        tile = pair_tile(p, pair, npairs, it);
+      }
       if (tile < 0) break;
       const TileCoord tc = tile_coord(p, tile);
       const GemmJob& j = p.jobs[tc.job];
@@ -598,7 +676,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
           // bank once per 8 lanes.  Lane 0 then issues the box's store (or fp32
           // add), which the TMA unit writes as whole 128-byte lines.  Rows and
           // columns past the output's extent are dropped by the TMA unit.
-          const float sc = tc.job ? job_scale1 : job_scale0;
+          const float sc = j.scale ? __ldg(j.scale) : 1.0f;
           const CUtensorMap* omap = &p.maps[j.out_map];
           const int y = m0 + quarter * 32;
           const int step = j.out_f32 ? 1 : 2;  // 32-column TMEM slices per box
@@ -638,7 +716,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
             if (kBoxes > 1) sbuf ^= 1;
           }
         } else {
-          const float sc = tc.job ? job_scale1 : job_scale0;
+          const float sc = j.scale ? __ldg(j.scale) : 1.0f;
   #pragma unroll 1
           for (int c = c_lo; c < c_hi; ++c) {
             float v[32];
@@ -676,6 +754,16 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, kDevErrTimeout);
+  if (p.dyn && threadIdx.x == 0) {
+    // the last CTA to finish returns the queue counter to zero for the next launch
+    // (every claim of this CTA's pair precedes its arrival here)
+    __threadfence();
+    if (atomicAdd(p.ctr_done, 1u) == gridDim.x - 1) {
+      *reinterpret_cast<volatile unsigned*>(p.ctr) = 0u;
+      *reinterpret_cast<volatile unsigned*>(p.ctr_done) = 0u;
+      __threadfence();
+    }
+  }
 }
 
 }  // namespace
@@ -881,9 +969,14 @@ cudaError_t launch_gemm(const GemmParams& p0, DType dt, cudaStream_t stream) {
   // boxes: 4 epilogue warps with two boxes each drain them faster than 8 with one.
   // A split job's fp32 output is small next to its K (two adds per output element
   // over thousands of k-steps) and does not count.
-  bool f32_tma = false;
-  for (int i = 0; i < p.njobs; ++i)
+  // A launch that also holds logits tiles (a chunk's backward merged with the
+  // next chunk's forward) keeps 8 warps for their logsumexp epilogue.
+  bool f32_tma = false, lse = false;
+  for (int i = 0; i < p.njobs; ++i) {
     f32_tma = f32_tma || (p.jobs[i].out_path != kOutDirect && p.jobs[i].out_f32 && p.jobs[i].k_split < 2);
+    lse = lse || p.jobs[i].epi == kEpiLse;
+  }
+  if (lse && debug_knobs().gemm_merge != 2) f32_tma = false;
   if (dt == DType::BF16) {
     if (f32_tma) return nh == 2 ? launch_t<__nv_bfloat16, 2, 4>(p, stream) : launch_t<__nv_bfloat16, 1, 4>(p, stream);
     return nh == 2 ? launch_t<__nv_bfloat16, 2, 8>(p, stream) : launch_t<__nv_bfloat16, 1, 8>(p, stream);

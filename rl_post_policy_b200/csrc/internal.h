@@ -24,7 +24,10 @@ constexpr unsigned kDevErrTarget = 2u;
 //   +4  u32 grid-barrier arrival counter
 //   +8  u32 finished-block counter
 //   +16 u64 global valid-token count
+//   +32 u32 GEMM tile-queue counter, +36 u32 its finished-CTA counter (fused path;
+//       both return to zero at the end of every launch that uses them)
 constexpr size_t kWsHeader = 256;
+constexpr size_t kWsGemmQueue = 32;
 
 // Bound on every device-side wait, in nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -113,6 +116,9 @@ struct DebugKnobs {
                          // 2 = the cooperative kernel
   int rkl_path = 0;      // reverse KL with a gradient: 0 = the host's choice (the streaming kernel),
                          // 1 = the streaming kernel, 2 = the register-resident kernel where it applies
+  int gemm_merge = 0;    // fused path with several chunks: 0 = chunk c's backward and chunk c+1's
+                         // forward share a launch (8 epilogue warps), 1 = separate launches,
+                         // 2 = shared launches with 4 epilogue warps
   int gemm_split = 0;    // K split of the backward launch's dX problem: 0 = the host's choice,
                          // 1 = never, 2 = always (when it has at least two k-steps)
 };

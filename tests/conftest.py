@@ -32,14 +32,19 @@ def gemm_tile(request):
     pl.pl_debug_set_gemm_tile(0)
 
 
-@pytest.fixture(params=[1, 2], ids=["no_ksplit", "ksplit"])
-def dx_split(request):
-    """Runs a GPU test once with the backward launch's dX problem whole and once
-    with it split in two K halves (fp32 halves added into a zeroed buffer)."""
+@pytest.fixture(params=[(1, 0), (2, 1), (1, 2)], ids=["merged", "separate_ksplit", "merged_ew4"])
+def gemm_variant(request):
+    """Runs a GPU test with each way the fused path may launch its GEMMs: several
+    chunks' backward and next forward merged into one dynamically scheduled launch
+    (the default), separate launches with the backward's dX problem split in two K
+    halves, and merged launches with 4 epilogue warps."""
     import rl_post_policy_b200 as pl
-    assert pl.pl_debug_set_gemm_split(request.param) == 0
+    split, merge = request.param
+    assert pl.pl_debug_set_gemm_split(split) == 0
+    assert pl.pl_debug_set_gemm_merge(merge) == 0
     yield request.param
     pl.pl_debug_set_gemm_split(0)
+    pl.pl_debug_set_gemm_merge(0)
 
 
 @pytest.fixture(params=[1, 2], ids=["rkl_streaming", "rkl_resident"])

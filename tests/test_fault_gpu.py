@@ -86,3 +86,41 @@ def test_reverse_kl_slot_timeout_is_reported(pl):
     assert pl.pl_device_status(ws) == pl.PL_OK
     want = oracle.reverse_kl(inp["student"], inp["teacher"], inp["mask"])
     assert abs(loss.item() - want["loss"]) <= 1e-4 * abs(want["loss"])
+
+
+def test_merged_chunk_launch_timeout_is_reported(pl):
+    # several chunks: the merged backward + forward launch (dynamic tile queue)
+    # times out like any other, and its queue counters are back at zero for the
+    # next call on the same workspace
+    import numpy as np
+    bs, T, H, V = 2, 192, 128, 1000
+    inp = synth.fused_inputs(bs, T, H, V, torch.bfloat16, 6161, bias=False, need_ref=True)
+    _, lp, _ = oracle.lm_head_logprob(inp["X"], inp["W"], None, inp["targets"])
+    inp["old_lp"] = (torch.from_numpy(lp) + inp["old_noise"].double()).float()
+    g = {k: inp[k].cuda() for k in ("X", "W", "Xref", "Wref", "targets", "old_lp", "adv", "mask")}
+    mode = pl.PL_BF16 | pl.PL_GRPO | pl.PL_CHUNK_ROWS(128)
+    wsb = pl.pl_fused_linear_grpo_workspace_bytes(bs, T, H, V, mode, 1, 0)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    loss = torch.zeros(1, device="cuda")
+    dX = torch.empty(bs * T, H, dtype=torch.bfloat16, device="cuda")
+    dW = torch.empty(V, H, dtype=torch.bfloat16, device="cuda")
+
+    def call():
+        return pl.pl_fused_linear_grpo(g["X"], g["W"], None, g["targets"], g["Xref"], g["Wref"], g["old_lp"],
+                                       g["adv"], g["mask"], bs, T, H, V, 0.2, 0.28, 0.04, mode, loss, dX, dW,
+                                       None, None, None, None, ws, wsb)
+
+    pl.pl_debug_set_wait(50_000_000, 0, 16)
+    pl.check(call())
+    assert pl.pl_device_status(ws) == pl.PL_ERR_DEVICE_TIMEOUT
+    pl.pl_debug_set_wait(0, 0, 0)
+    # a workspace that saw a device error is zeroed again before reuse
+    ws.zero_()
+    pl.check(call())
+    assert pl.pl_device_status(ws) == pl.PL_OK
+    want = oracle.fused_grpo(inp["X"], inp["W"], None, inp["targets"], inp["Xref"], inp["Wref"],
+                             inp["old_lp"].reshape(bs, T), inp["adv"], inp["mask"], eps_lo=0.2, eps_hi=0.28,
+                             beta=0.04, reduction=oracle.GRPO)
+    assert abs(loss.item() - want["loss"]) <= 1e-3 * abs(want["loss"])
+    rel = np.linalg.norm(dW.cpu().double().numpy() - want["dW"]) / np.linalg.norm(want["dW"])
+    assert rel <= 1e-2

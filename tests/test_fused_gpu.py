@@ -13,7 +13,7 @@ import torch
 import oracle
 import synth
 
-pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gemm_tile", "dx_split")]
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gemm_tile", "gemm_variant")]
 
 EPS_LO, EPS_HI = 0.2, 0.28
 

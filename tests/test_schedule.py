@@ -114,3 +114,39 @@ def test_k_split_knob_forces_either_choice():
     finally:
         pl.pl_debug_set_gemm_split(0)
     assert pl.pl_debug_pick_split([(1, 1, 1)], 74)[0] == -1
+
+
+@pytest.mark.parametrize("tiles,q_f0,q_w", [
+    ([32, 1004, 1004, 4008], 1, 3),   # merged launch: dX, reference and policy forward, dW
+    ([64, 1004, 4008], 1, 2),         # the same at beta = 0 (no reference forward)
+    ([1004, 1004, 4008], 0, 2),       # no dX
+    ([32, 1004, 1004], 1, -1),        # no dW: job order
+    ([3, 0, 5, 9], 1, 3),
+])
+def test_dynamic_queue_order(tiles, q_f0, q_w):
+    rc, order = pl.pl_debug_queue_tiles(tiles, q_f0, q_w)
+    assert rc == 0
+    total = sum(tiles)
+    assert sorted(order) == list(range(total))           # every tile exactly once
+    lead = sum(tiles[:q_f0])
+    assert order[:lead] == list(range(lead))              # the long tiles first, in order
+    if q_w < 0:
+        assert order == list(range(total))
+        return
+    f_begin, w_begin = lead, sum(tiles[:q_w])
+    rest = order[lead:]
+    fw = [t for t in rest if t < w_begin]
+    dw = [t for t in rest if t >= w_begin]
+    assert fw == sorted(fw) and dw == sorted(dw)          # each kind in its own order
+    # spread evenly: every prefix of the rest holds the forward tiles in proportion
+    nf, n = len(fw), len(rest)
+    seen = 0
+    for i, t in enumerate(rest):
+        seen += t < w_begin
+        assert abs(seen - (i + 1) * nf / n) <= 1.0
+
+
+def test_dynamic_queue_rejects_bad_input():
+    assert pl.pl_debug_queue_tiles([], 0, -1)[0] == -1
+    assert pl.pl_debug_queue_tiles([1, 2, 3, 4, 5], 0, -1)[0] == -1
+    assert pl.pl_debug_queue_tiles([1, 2], 2, 1)[0] == -1

@@ -9,7 +9,7 @@ import torch
 import oracle
 import synth
 
-pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gemm_tile", "dx_split")]
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gemm_tile", "gemm_variant")]
 
 
 def run(inp, dtype, grad_logp=None, chunk=None, want=("dX", "dW", "dbias"), targets=None):
