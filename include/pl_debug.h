@@ -149,6 +149,26 @@ int pl_debug_set_gemm_split(int mode);
 int pl_debug_set_gemm_merge(int mode);
 
 /*
+ * 512-wide GEMM launches on the round-robin schedule (the forward launches):
+ * 0 (the default) = when the last partial wave holds R <= pairs / 2 tiles, those
+ * tiles run as 2R tiles 256 wide, so the wave ends after half a tile's time;
+ * 1 = never.  pl_debug_tail_halves returns R for `tiles` equal tiles on `pairs`
+ * pairs (0: no split).  Returns PL_ERR_ARG for another mode.
+ */
+int pl_debug_set_gemm_tail(int mode);
+int pl_debug_tail_halves(int tiles, int pairs);
+
+/*
+ * Fused path with several row chunks, how dW is finished: 1 = the last chunk
+ * adds into the fp32 accumulator like the others and a separate kernel rounds
+ * it; 2 = the last chunk's dW epilogue adds the fp32 accumulator of the earlier
+ * chunks and stores the model dtype; 0 restores the default (1, measured
+ * faster).  Applies to later calls on this process.  Returns PL_ERR_ARG for
+ * another value.
+ */
+int pl_debug_set_dw_finish(int mode);
+
+/*
  * The GEMM's dynamic tile-queue order (host logic): jobs of tiles[0..njobs)
  * tiles, numbered in job order; queue entry q runs tile out[q].  The tiles of
  * jobs [0, q_f0) come first in order, then those of jobs [q_f0, q_w) spread

@@ -98,6 +98,12 @@ _lib.pl_debug_set_gemm_tile.argtypes = [_I]
 _lib.pl_debug_set_gemm_tile.restype = _I
 _lib.pl_debug_set_rkl_cluster.argtypes = [_I]
 _lib.pl_debug_set_rkl_cluster.restype = _I
+_lib.pl_debug_set_gemm_tail.argtypes = [_I]
+_lib.pl_debug_set_gemm_tail.restype = _I
+_lib.pl_debug_tail_halves.argtypes = [_I, _I]
+_lib.pl_debug_tail_halves.restype = _I
+_lib.pl_debug_set_dw_finish.argtypes = [_I]
+_lib.pl_debug_set_dw_finish.restype = _I
 _lib.pl_debug_set_gemm_merge.argtypes = [_I]
 _lib.pl_debug_set_gemm_merge.restype = _I
 _lib.pl_debug_queue_tiles.argtypes = [_I, _P, _I, _I, _P]
@@ -117,7 +123,8 @@ EXPORTED = ("pl_init", "pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_line
             "pl_version", "pl_debug_gemm", "pl_debug_gemm_out", "pl_debug_timing", "pl_debug_timing_read",
             "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_set_gemm_tile", "pl_debug_pair_tiles",
             "pl_debug_pick_tile", "pl_debug_set_loss_path", "pl_debug_pick_split", "pl_debug_set_gemm_split",
-            "pl_debug_set_rkl_path", "pl_debug_set_gemm_merge", "pl_debug_queue_tiles")
+            "pl_debug_set_rkl_path", "pl_debug_set_gemm_merge", "pl_debug_queue_tiles",
+            "pl_debug_set_dw_finish", "pl_debug_set_gemm_tail", "pl_debug_tail_halves")
 
 
 class PLError(RuntimeError):
@@ -326,6 +333,23 @@ def pl_debug_set_rkl_path(path: int) -> int:
     """Test hook: reverse KL with a gradient -- 0 the default (the streaming kernel), 1 the
     streaming kernel, 2 the register-resident kernel where it applies."""
     return int(_lib.pl_debug_set_rkl_path(int(path)))
+
+
+def pl_debug_set_gemm_tail(mode: int) -> int:
+    """Test hook: 512-wide round-robin launches -- 0 the last partial wave in 256-wide halves
+    where that helps (default), 1 never."""
+    return int(_lib.pl_debug_set_gemm_tail(int(mode)))
+
+
+def pl_debug_tail_halves(tiles: int, pairs: int) -> int:
+    """Test hook: tiles of the last partial wave that run in halves (0: none)."""
+    return int(_lib.pl_debug_tail_halves(int(tiles), int(pairs)))
+
+
+def pl_debug_set_dw_finish(mode: int) -> int:
+    """Test hook: several-chunk dW -- 1 fp32 add then a separate rounding kernel (the default, 0),
+    2 the last chunk's epilogue adds the accumulator and stores the model dtype."""
+    return int(_lib.pl_debug_set_dw_finish(int(mode)))
 
 
 def pl_debug_set_gemm_merge(mode: int) -> int:

@@ -84,6 +84,20 @@ extern "C" int pl_debug_pick_split(const int64_t* mnk, int pairs, int* nh_out) {
   return split;
 }
 
+extern "C" int pl_debug_set_gemm_tail(int mode) {
+  if (mode < 0 || mode > 1) return PL_ERR_ARG;
+  debug_knobs().gemm_tail = mode;
+  return PL_OK;
+}
+
+extern "C" int pl_debug_tail_halves(int tiles, int pairs) { return tail_halves(tiles, pairs); }
+
+extern "C" int pl_debug_set_dw_finish(int mode) {
+  if (mode < 0 || mode > 2) return PL_ERR_ARG;
+  debug_knobs().dw_finish = mode;
+  return PL_OK;
+}
+
 extern "C" int pl_debug_set_gemm_merge(int mode) {
   if (mode < 0 || mode > 2) return PL_ERR_ARG;
   debug_knobs().gemm_merge = mode;

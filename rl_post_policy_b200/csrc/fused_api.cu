@@ -161,6 +161,12 @@ pl_status run_pipeline(const Pipe& q) {
     return ws + plan.off.logits + (merge ? (c & 1) * plan.logits_bytes : 0);
   };
   auto rows_of = [&](int64_t c) -> int64_t { return (N - c * plan.C) < plan.C ? (N - c * plan.C) : plan.C; };
+  // Several chunks: the last chunk adds into the fp32 accumulator like the others
+  // and a streaming kernel rounds it (at the copy bandwidth).  On request, the
+  // last chunk's dW epilogue instead adds the accumulator and stores the model
+  // dtype in one pass: measured, its per-thread accumulator loads slowed that
+  // launch by about what the rounding kernel costs, or more.
+  const bool fuse_finish = debug_knobs().dw_finish == 2;
 
   // Chunk c's forward jobs (reference, then policy) appended to g; maps from *nm.
   auto add_fwd = [&](GemmParams& g, int64_t c, int& nm) -> bool {
@@ -239,6 +245,14 @@ pl_status run_pipeline(const Pipe& q) {
     j.acc_in = nullptr;
     if (plan.nchunks == 1) {
       j.out = dW; j.out_f32 = 0; j.out_path = kOutDirect;
+      if (aligned(dW, 16)) {
+        if (!make_tmap_2d(&g.maps[mo], dW, dt, H, V, H * esz, kOutBoxN16, kOutBoxM)) return false;
+        j.out_path = kOutTmaStore; j.out_map = mo;
+      }
+    } else if (c + 1 == plan.nchunks && fuse_finish) {
+      // the last chunk: its epilogue adds the accumulator of the earlier chunks and
+      // rounds the sum to the model dtype in one pass (no separate rounding kernel)
+      j.out = dW; j.out_f32 = 0; j.acc_in = acc; j.out_path = kOutDirect;
       if (aligned(dW, 16)) {
         if (!make_tmap_2d(&g.maps[mo], dW, dt, H, V, H * esz, kOutBoxN16, kOutBoxM)) return false;
         j.out_path = kOutTmaStore; j.out_map = mo;
@@ -370,7 +384,7 @@ pl_status run_pipeline(const Pipe& q) {
       }
     }
   }
-  if (dW && plan.nchunks > 1 &&
+  if (dW && plan.nchunks > 1 && !fuse_finish &&
       !ok(launch_convert(reinterpret_cast<const float*>(ws + plan.off.dw_acc), dW, V * H, dt, s)))
     return PL_ERR_CUDA;
 

@@ -59,6 +59,11 @@ struct GemmJob {
   // long tiles would otherwise finish last.
   int k_split;
   int k_per;               // k-steps per split (set by gemm_finalize_jobs)
+  // 512-wide launches: the job's last `tail` tiles each run as two 256-wide
+  // tiles (columns [0, 256) and [256, 512) of the pair tile), listed after its
+  // other tiles, so that a round-robin launch's last partial wave is spread over
+  // twice as many pairs (set by launch_gemm; 0 = none).
+  int tail;
   int n_inner;             // 1: consecutive tiles walk N first (share the A rows)
   int tile_begin;          // first global tile index of this job
   int epi;
@@ -75,9 +80,10 @@ struct GemmJob {
   // kEpiStore
   void* out;
   int out_f32;
-  int out_path;            // OutPath; kOutTma* need acc_in = null and out_map
+  int out_path;            // OutPath; kOutTma* need out_map
   int out_map;             // tensor-map index of `out` for the kOutTma* paths
-  const float* acc_in;     // [M, out_ld] fp32 added before the store, or null
+  const float* acc_in;     // [M, out_ld] fp32 added before the store, or null (16-bit outputs
+                           // of kOutDirect and kOutTmaStore)
   int64_t out_ld;
   const float* scale;      // device scalar multiplier, or null for 1
 };
@@ -126,8 +132,20 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, DType dt, uint64_t inner, 
 // tiles nh * kBN wide.  launch_gemm picks nh (unless p->nh is set) and calls it again.
 void gemm_finalize_jobs(GemmParams* p);
 
-// Tiles of a job (output tiles times its K split).
-inline int job_tiles(const GemmJob& j) { return j.tiles_m * j.tiles_n * (j.k_split > 1 ? j.k_split : 1); }
+// Tiles of a job (output tiles times its K split, plus one for each tail tile run in halves).
+inline int job_tiles(const GemmJob& j) {
+  return j.tiles_m * j.tiles_n * (j.k_split > 1 ? j.k_split : 1) + (j.tail > 0 ? j.tail : 0);
+}
+
+// Tiles of a round-robin launch of T equal 512-wide tiles on P pairs to run in
+// halves: the last partial wave's R = T mod P tiles when R <= P / 2 (their 2R
+// halves then take half a tile's time on 2R pairs instead of a whole one on R),
+// else none.
+inline int tail_halves(int T, int P) {
+  if (P <= 1 || T <= P) return 0;
+  const int r = T % P;
+  return (r > 0 && 2 * r <= P) ? r : 0;
+}
 
 cudaError_t launch_gemm(const GemmParams& p, DType dt, cudaStream_t stream);
 

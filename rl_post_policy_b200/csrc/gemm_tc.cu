@@ -105,6 +105,7 @@ template <> struct AbFormat<__nv_bfloat16> { static constexpr uint32_t v = 1; };
 struct TileCoord {
   int job, mb, nb;
   int kb, nk;  // first k-step and number of k-steps of this tile (all of K unless the job is split)
+  int half;    // -1: the whole pair tile; 0 or 1: only its columns [256 * half, 256 * half + 256)
 };
 
 // Tile `tile` of the launch: its job, row block, column block and K range.  A
@@ -119,6 +120,15 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmParams& p, int tile) {
   int local = tile - j.tile_begin;
   c.kb = 0;
   c.nk = j.k_steps;
+  c.half = -1;
+  if (j.tail > 0) {
+    const int base = j.tiles_m * j.tiles_n - j.tail;
+    if (local >= base) {
+      const int hh = local - base;
+      local = base + (hh >> 1);
+      c.half = hh & 1;
+    }
+  }
   if (j.k_split > 1) {
     const int per = j.tiles_m * j.tiles_n;
     const int ks = local / per;
@@ -221,6 +231,25 @@ __device__ __forceinline__ void add_row32_f32(const float* src, float (&v)[32], 
 #pragma unroll
     for (int j = 0; j < 32; ++j)
       if (j < nvalid) v[j] += src[j];
+  }
+}
+
+// v[q] = v[q] * sc + src[q] over the first nvalid of 32 columns (v[q] * sc past
+// them); src is read once, with streaming loads.
+__device__ __forceinline__ void scale_add_row32(const float* src, float (&v)[32], float sc, int nvalid) {
+  if (nvalid >= 32 && ((reinterpret_cast<uintptr_t>(src) & 15) == 0)) {
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 a = __ldcs(s4 + q);
+      v[4 * q] = v[4 * q] * sc + a.x;
+      v[4 * q + 1] = v[4 * q + 1] * sc + a.y;
+      v[4 * q + 2] = v[4 * q + 2] * sc + a.z;
+      v[4 * q + 3] = v[4 * q + 3] * sc + a.w;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 32; ++q) v[q] = q < nvalid ? v[q] * sc + __ldcs(src + q) : v[q] * sc;
   }
 }
 
@@ -369,9 +398,12 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
         const int nt0 = tc.nb * Cfg::kTileN + (int)rank * kBNh;
         const CUtensorMap* amap = &p.maps[j.a_map];
         const CUtensorMap* bmap = &p.maps[j.b_map];
+        // a half tile loads one B half (its columns) into the stage's first B slot
+        const int nb_loads = tc.half < 0 ? NH : 1;
+        const uint32_t stage_tx = 2 * (kABytes + (uint32_t)nb_loads * kBBytes) + p.extra_tx;
         for (int k = 0; k < tc.nk; ++k) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, lim)) break;
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes + p.extra_tx);
+          if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx);
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = ring + stage * kStageBytes;
           uint8_t* b_dst = a_dst + kABytes;
@@ -384,8 +416,9 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
           }
 #pragma unroll
           for (int h = 0; h < NH; ++h) {
+            if (h >= nb_loads) break;
             // MMA h needs columns [h*kBN, (h+1)*kBN) of the tile; this CTA holds kBNh of them
-            const int n0 = nt0 + h * kBN;
+            const int n0 = nt0 + (tc.half < 0 ? h : tc.half) * kBN;
             uint8_t* bh = b_dst + h * kBBytes;
             if (!j.b_mn) {
               tma_load_2d_pair(bh, bmap, bar, k0, n0);
@@ -460,6 +493,25 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
             acc = 0;
             acc_phase ^= 1;
           }
+        } else if (tc.half >= 0) {
+          // A half tile: its one 256-column MMA per stage goes into accumulator
+          // half 0 (the epilogue drains only that half and releases half 1 at
+          // once, which keeps both halves' barrier phases in step with the tiles).
+          if (!mbar_wait(&tempty[0], acc_phase ^ 1, abort_flag, lim)) break;
+          tc_fence_after();
+          for (int k = 0; k < tc.nk; ++k) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, lim)) { ok = false; break; }
+            tc_fence_after();
+            issue(stage, k, j, idesc, 0, 0);
+            mma_commit_pair(&empty[stage], 0x3);
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+          if (!ok) break;
+          mma_commit_pair(&tfull[0], 0x3);
+          acc_phase ^= 1;
         } else {
           // One 512-column accumulator, drained by the epilogue in two halves
           // (tempty[0], tempty[1]).  Half 0 of this tile starts once the
@@ -566,9 +618,11 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
       tc_fence_after();
 #pragma unroll 1
       for (int h = 0; h < NH; ++h) {
-        // 256-column group h of the tile: TMEM columns [col_base, col_base + 256)
-        const int n0 = tc.nb * Cfg::kTileN + h * kBN;
-        const int grp = tc.nb * NH + h;     // index of this 256-column group along N
+        // 256-column group h of the tile: TMEM columns [col_base, col_base + 256);
+        // a half tile has one group, its columns in accumulator half 0
+        const int colh = tc.half < 0 ? h : tc.half;
+        const int n0 = (tc.half >= 0 && h > 0) ? j.N : tc.nb * Cfg::kTileN + colh * kBN;
+        const int grp = tc.nb * NH + colh;  // index of this 256-column group along N
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (NH == 1 ? acc : h) * kBN;
         if (n0 >= j.N) {
           // past the end of N: zeros only, nothing to store
@@ -688,6 +742,20 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
             if (j.out_f32) {
   #pragma unroll
               for (int q = 0; q < 32; ++q) w[q] = __float_as_uint(v[q] * sc);
+            } else if (j.acc_in) {
+              // the fp32 accumulator of the earlier chunks added to this tile, then
+              // rounded once to the model dtype (the last chunk of a multi-chunk dW)
+              const float* arow = j.acc_in + (int64_t)(row_ok ? row : 0) * j.out_ld;
+              const int colA = n0 + c * 32;
+              float sa = row_ok ? 1.0f : 0.0f;  // rows past M: no load, dropped by the TMA store
+              if (row_ok) scale_add_row32(arow + colA, v, sc, min(32, j.N - colA));
+              else sa = sc;
+  #pragma unroll
+              for (int q = 0; q < 16; ++q) w[q] = pack2<T>(v[2 * q] * sa, v[2 * q + 1] * sa);
+              tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
+              if (row_ok) scale_add_row32(arow + colA + 32, v, sc, min(32, j.N - colA - 32));
+  #pragma unroll
+              for (int q = 0; q < 16; ++q) w[16 + q] = pack2<T>(v[2 * q] * sa, v[2 * q + 1] * sa);
             } else {
   #pragma unroll
               for (int q = 0; q < 16; ++q) w[q] = pack2<T>(v[2 * q] * sc, v[2 * q + 1] * sc);
@@ -940,6 +1008,15 @@ cudaError_t launch_t(const GemmParams& p, cudaStream_t stream) {
   cfg.gridDim = dim3(2 * pairs);
   GemmParams q = p;
   balance_schedule(&q, pairs);
+  if (NH == 2 && q.sched == 0 && !q.dyn && debug_knobs().gemm_tail != 1) {
+    // a round-robin launch's last partial wave in 256-wide halves
+    GemmJob& last = q.jobs[q.njobs - 1];
+    const int tail = tail_halves(q.total_tiles, pairs);
+    if (tail > 0 && last.k_split < 2 && last.tiles_m * last.tiles_n >= tail) {
+      last.tail = tail;
+      gemm_finalize_jobs(&q);
+    }
+  }
   launch_begin(0, stream);
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<T, NH, EW>, q);
   launch_end(0, stream);

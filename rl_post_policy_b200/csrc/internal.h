@@ -119,6 +119,11 @@ struct DebugKnobs {
   int gemm_merge = 0;    // fused path with several chunks: 0 = chunk c's backward and chunk c+1's
                          // forward share a launch (8 epilogue warps), 1 = separate launches,
                          // 2 = shared launches with 4 epilogue warps
+  int gemm_tail = 0;     // 512-wide round-robin launches: 0 = the last partial wave's tiles run as
+                         // 256-wide halves where that shortens the launch, 1 = never
+  int dw_finish = 0;     // several chunks: 0 = the host's choice (1), 1 = fp32 add, then a separate
+                         // rounding kernel, 2 = the last chunk's dW epilogue adds the fp32
+                         // accumulator and stores the model dtype
   int gemm_split = 0;    // K split of the backward launch's dX problem: 0 = the host's choice,
                          // 1 = never, 2 = always (when it has at least two k-steps)
 };

@@ -32,19 +32,24 @@ def gemm_tile(request):
     pl.pl_debug_set_gemm_tile(0)
 
 
-@pytest.fixture(params=[(1, 0), (2, 1), (1, 2)], ids=["merged", "separate_ksplit", "merged_ew4"])
+@pytest.fixture(params=[(1, 0, 0), (2, 1, 2), (1, 2, 0)], ids=["merged", "separate_ksplit_fused_finish",
+                                                                 "merged_ew4"])
 def gemm_variant(request):
     """Runs a GPU test with each way the fused path may launch its GEMMs: several
-    chunks' backward and next forward merged into one dynamically scheduled launch
-    (the default), separate launches with the backward's dX problem split in two K
-    halves, and merged launches with 4 epilogue warps."""
+    chunks' backward and next forward merged into one dynamically scheduled launch,
+    with a separate pass rounding the fp32 dW accumulator (the default); separate
+    launches with the backward's dX problem split in two K halves and the last
+    chunk's dW epilogue finishing the fp32 accumulation; and merged launches with
+    4 epilogue warps."""
     import rl_post_policy_b200 as pl
-    split, merge = request.param
+    split, merge, finish = request.param
     assert pl.pl_debug_set_gemm_split(split) == 0
     assert pl.pl_debug_set_gemm_merge(merge) == 0
+    assert pl.pl_debug_set_dw_finish(finish) == 0
     yield request.param
     pl.pl_debug_set_gemm_split(0)
     pl.pl_debug_set_gemm_merge(0)
+    pl.pl_debug_set_dw_finish(0)
 
 
 @pytest.fixture(params=[1, 2], ids=["rkl_streaming", "rkl_resident"])

@@ -279,3 +279,21 @@ def test_repeat_calls_are_bit_identical():
     assert a["loss"] == b["loss"]
     for k in ("logp", "ref_logp", "dX", "dW", "dbias"):
         assert np.array_equal(a[k], b[k]), k
+
+
+@pytest.mark.parametrize("beta", [0.04, 0.0], ids=["beta0.04", "beta0"])
+def test_forward_last_wave_in_half_tiles(beta):
+    # 256 rows x V = 40900 (80 vocabulary tiles of 512, the last one ragged) per model:
+    # 160 forward tiles (80 at beta = 0) on 74 pairs leave a last wave of 12 (6) tiles,
+    # which run as 256-wide halves with the tile512 fixture; the logsumexp partials
+    # and the stored logits of those halves must be those of whole tiles
+    m = pl()
+    inp = build_inputs(2, 128, 128, 40900, torch.bfloat16, 5252, bias=True, len_lo=0, len_hi=128)
+    try:
+        for no_tail in (0, 1):
+            assert m.pl_debug_set_gemm_tail(no_tail) == 0
+            for red in (0, 1):
+                got = run_fused(inp, torch.bfloat16, red, beta)
+                check(inp, got, red, beta)
+    finally:
+        m.pl_debug_set_gemm_tail(0)

@@ -109,3 +109,18 @@ def test_tma_output_paths(a_mn, b_mn, shape):
     D = fresh(R)
     m.check(m.pl_debug_gemm_out(Ad, a_mn, lda, Bd, b_mn, ldb, D, ldd, 2, M, N, K, mode), "add")
     check(D, R.double() + ref, R.double().abs())
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (1, 1)])
+@pytest.mark.parametrize("N", [40960, 40900], ids=["N_tile_exact", "N_ragged"])
+def test_last_wave_in_half_tiles(a_mn, b_mn, N):
+    # 80 tiles of 256 x 512 on the 74 pairs of a B200: the last 6 run as 12 tiles
+    # 256 wide (with the tile512 fixture), including the partial last column tile
+    m = __import__("rl_post_policy_b200")
+    assert m.pl_debug_tail_halves(80, 74) == 6
+    try:
+        for no_tail in (0, 1):
+            assert m.pl_debug_set_gemm_tail(no_tail) == 0
+            run(256, N, 192, a_mn, b_mn, torch.bfloat16, seed=N + a_mn)
+    finally:
+        m.pl_debug_set_gemm_tail(0)

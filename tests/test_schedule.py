@@ -150,3 +150,21 @@ def test_dynamic_queue_rejects_bad_input():
     assert pl.pl_debug_queue_tiles([], 0, -1)[0] == -1
     assert pl.pl_debug_queue_tiles([1, 2, 3, 4, 5], 0, -1)[0] == -1
     assert pl.pl_debug_queue_tiles([1, 2], 2, 1)[0] == -1
+
+
+@pytest.mark.parametrize("tiles,pairs,want", [
+    (2008, 74, 10),    # the batch-1 forward at 512 wide: 27 waves and 10 tiles
+    (16064, 74, 6),    # a whole 8192-row batch
+    (2018, 74, 20),
+    (2049, 74, 0),     # 51 tiles in the last wave: halves would not end it sooner
+    (148, 74, 0),      # whole waves
+    (50, 74, 0),       # a single partial wave
+    (10, 1, 0),
+])
+def test_tail_halves(tiles, pairs, want):
+    r = pl.pl_debug_tail_halves(tiles, pairs)
+    assert r == want
+    if r:
+        # full waves, then 2r halves on 2r pairs: the launch ends half a tile after the full waves
+        full = tiles - r
+        assert full % pairs == 0 and 2 * r <= pairs
