@@ -261,6 +261,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// The bias of up to 64 consecutive columns (the first nvalid) added to v.
+template <typename T>
+__device__ __forceinline__ void add_bias64(const T* bias, float (&v)[64], int nvalid) {
+  if (nvalid >= 64 && ((reinterpret_cast<uintptr_t>(bias) & 15) == 0)) {
+    const uint4* b4 = reinterpret_cast<const uint4*>(bias);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint4 u = __ldg(b4 + q);
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[8 * q + k] += cvt_in(e[k]);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 64; ++k)
+      if (k < nvalid) v[k] += cvt_in(bias[k]);
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ void add_bias32(const T* bias, float (&v)[32], int nvalid) {
   if (nvalid >= 32 && ((reinterpret_cast<uintptr_t>(bias) & 15) == 0)) {
@@ -639,62 +658,89 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
   #pragma unroll 1
           for (int c = c_lo; c < c_hi; c += 2) {
             uint32_t w[32];
+            // the box's 64 columns in one tensor-memory load
+            float v[64];
+            tmem_ld_32x32b_x64(taddr + c * 32, v);
+            const int col0 = n0 + c * 32;
+            const int nv0 = min(32, j.N - col0), nv1 = min(32, j.N - col0 - 32);
+            if (nv0 > 0) {
+              if (bias) add_bias64<T>(bias + col0, v, nv0 + (nv1 > 0 ? nv1 : 0));
+              if (j.logit_scale != 1.0f) {
   #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              float v[32];
-              tmem_ld_32x32b_x32(taddr + (c + h) * 32, v);
-              const int col0 = n0 + (c + h) * 32;
-              const int nvalid = min(32, j.N - col0);
-              if (nvalid > 0) {
-                if (bias) add_bias32<T>(bias + col0, v, nvalid);
-                if (j.logit_scale != 1.0f) {
-  #pragma unroll
-                  for (int q = 0; q < 32; ++q) v[q] *= j.logit_scale;
-                }
-                if (nvalid == 32) {
-                  // full chunk: no per-column predicates; two columns per packed instruction
-                  float cmax = v[0];
-  #pragma unroll
-                  for (int q = 1; q < 32; ++q) cmax = fmaxf(cmax, v[q]);
-                  const float m_new = fmaxf(m_run, cmax);
-                  const float2 nmb = make_float2(-m_new * kLog2e, -m_new * kLog2e);
-                  const float2 l2e = make_float2(kLog2e, kLog2e);
-                  float2 s2 = make_float2(0.0f, 0.0f);
-  #pragma unroll
-                  for (int q = 0; q < 32; q += 2) {
-                    const float2 x = __ffma2_rn(make_float2(v[q], v[q + 1]), l2e, nmb);
-                    s2 = __fadd2_rn(s2, make_float2(ex2_approx(x.x), ex2_approx(x.y)));
-                  }
-                  s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, nmb.x)) + (s2.x + s2.y);
-                  m_run = m_new;
-                } else {
-                  float cmax = -INFINITY;
-  #pragma unroll
-                  for (int q = 0; q < 32; ++q)
-                    if (q < nvalid) cmax = fmaxf(cmax, v[q]);
-                  const float m_new = fmaxf(m_run, cmax);
-                  const float mb = m_new * kLog2e;
-                  float s = 0.0f;
-  #pragma unroll
-                  for (int q = 0; q < 32; ++q)
-                    if (q < nvalid) s += ex2_approx(fmaf(v[q], kLog2e, -mb));
-                  s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, -mb)) + s;
-                  m_run = m_new;
-                }
-                const int64_t rel = tgt_rel - (c + h) * 32;
-                if (rel >= 0 && rel < 32) {
-  #pragma unroll
-                  for (int q = 0; q < 32; ++q)
-                    if (q == (int)rel) ztv = v[q];
-                  got = true;
-                }
-                if (logits && !tma_logits && row_ok)
-                  store_row32<T>(logits + (int64_t)row * j.logits_ld + col0, v, nvalid);
+                for (int q = 0; q < 64; ++q) v[q] *= j.logit_scale;
               }
-              if (tma_logits) {
+            }
+            if (nv1 == 32) {
+              // 64 full columns: the maximum by a tree and the sum of exponentials in
+              // four independent packed accumulators (short dependency chains), with
+              // one rescale of the running sum
+              float t[16];
   #pragma unroll
-                for (int q = 0; q < 16; ++q) w[16 * h + q] = pack2<T>(v[2 * q], v[2 * q + 1]);
+              for (int i = 0; i < 16; ++i)
+                t[i] = fmaxf(fmaxf(v[2 * i], v[2 * i + 1]), fmaxf(v[32 + 2 * i], v[33 + 2 * i]));
+  #pragma unroll
+              for (int i = 0; i < 8; ++i) t[i] = fmaxf(t[i], t[i + 8]);
+  #pragma unroll
+              for (int i = 0; i < 4; ++i) t[i] = fmaxf(t[i], t[i + 4]);
+              const float m_new = fmaxf(m_run, fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])));
+              const float2 nmb = make_float2(-m_new * kLog2e, -m_new * kLog2e);
+              const float2 l2e = make_float2(kLog2e, kLog2e);
+              float2 sacc[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                                make_float2(0.0f, 0.0f)};
+  #pragma unroll
+              for (int q = 0; q < 64; q += 2) {
+                const float2 x = __ffma2_rn(make_float2(v[q], v[q + 1]), l2e, nmb);
+                sacc[(q >> 1) & 3] = __fadd2_rn(sacc[(q >> 1) & 3], make_float2(ex2_approx(x.x), ex2_approx(x.y)));
               }
+              const float2 s01 = __fadd2_rn(sacc[0], sacc[1]), s23 = __fadd2_rn(sacc[2], sacc[3]);
+              const float2 s4 = __fadd2_rn(s01, s23);
+              s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, nmb.x)) + (s4.x + s4.y);
+              m_run = m_new;
+            } else {
+              // a ragged end of N: each 32-column slice with its own column predicates
+  #pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int nvalid = h ? nv1 : nv0;
+                if (nvalid <= 0) continue;
+                float cmax = -INFINITY;
+  #pragma unroll
+                for (int q = 0; q < 32; ++q)
+                  if (q < nvalid) cmax = fmaxf(cmax, v[32 * h + q]);
+                const float m_new = fmaxf(m_run, cmax);
+                const float mb = m_new * kLog2e;
+                float s = 0.0f;
+  #pragma unroll
+                for (int q = 0; q < 32; ++q)
+                  if (q < nvalid) s += ex2_approx(fmaf(v[32 * h + q], kLog2e, -mb));
+                s_run = s_run * ex2_approx(fmaf(m_run, kLog2e, -mb)) + s;
+                m_run = m_new;
+              }
+            }
+            // the target logit, if this box holds the row's target column
+            const int64_t rel = tgt_rel - c * 32;
+            if (rel >= 0 && rel < 64 && rel < (int64_t)(nv0 + (nv1 > 0 ? nv1 : 0))) {
+  #pragma unroll
+              for (int q = 0; q < 64; ++q)
+                if (q == (int)rel) ztv = v[q];
+              got = true;
+            }
+            if (logits && !tma_logits && row_ok) {
+              if (nv0 > 0) {
+                float u[32];
+  #pragma unroll
+                for (int q = 0; q < 32; ++q) u[q] = v[q];
+                store_row32<T>(logits + (int64_t)row * j.logits_ld + col0, u, nv0);
+              }
+              if (nv1 > 0) {
+                float u[32];
+  #pragma unroll
+                for (int q = 0; q < 32; ++q) u[q] = v[32 + q];
+                store_row32<T>(logits + (int64_t)row * j.logits_ld + col0 + 32, u, nv1);
+              }
+            }
+            if (tma_logits) {
+  #pragma unroll
+              for (int q = 0; q < 32; ++q) w[q] = pack2<T>(v[2 * q], v[2 * q + 1]);
             }
             if (tma_logits && n0 + c * 32 < j.N && y < j.M) {
               // the box's previous contents have been read out by the TMA unit
