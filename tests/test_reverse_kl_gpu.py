@@ -115,6 +115,30 @@ def test_many_rows_per_cluster_with_masked_runs(cl, dtype):
     check(got, want, mask, dtype, bs * seq, V)
 
 
+@pytest.mark.parametrize("cl", [1, 2, 4])
+def test_rows_dealt_by_kind_across_row_blocks(cl):
+    # Valid rows are dealt to the clusters by their rank among valid rows and
+    # masked rows by theirs, in blocks of 512 rows: here the masked rows all
+    # come first (a plain round-robin would give every cluster the same share
+    # of them), the run of valid rows crosses two block boundaries, and the
+    # last block is partial; without a mask every row is valid.
+    m = pl()
+    bs, seq, V = 3, 500, 1544
+    inp = synth.reverse_kl_inputs(bs, seq, V, torch.bfloat16, synth.seed_for(48, cl))
+    mask = torch.ones(bs * seq, dtype=torch.uint8)
+    mask[:700] = 0
+    mask[1100] = 0
+    mask = mask.reshape(bs, seq)
+    assert m.pl_debug_set_rkl_cluster(cl) == 0
+    try:
+        for mk in (mask, None):
+            want = oracle.reverse_kl(inp["student"], inp["teacher"], mk)
+            got = run(inp["student"], inp["teacher"], mk)
+            check(got, want, mk, torch.bfloat16, bs * seq, V)
+    finally:
+        m.pl_debug_set_rkl_cluster(0)
+
+
 def test_close_teacher_small_kl():
     # teacher = student + N(0, 0.05): kl ~ 1e-3, the cancellation-prone regime
     inp = synth.reverse_kl_inputs(4, 16, 32000, torch.bfloat16, synth.seed_for(42), teacher_std=0.05)
