@@ -257,6 +257,22 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
       }
     }
   }
+  // phase B's first two vectors of each thread toward L2 while the grid gathers
+  // at the barrier (measured 0.7% faster at 2^27 tokens)
+  if (VEC) {
+    const T* lpp = reinterpret_cast<const T*>(a.lp);
+    const T* odp = reinterpret_cast<const T*>(a.old);
+    const T* rfp = reinterpret_cast<const T*>(a.ref);
+#pragma unroll
+    for (int d = 0; d < 2; ++d) {
+      const int64_t tp = t0 + ((int64_t)tid + (int64_t)d * kThreads) * VW;
+      if (tp + VW <= t1) {
+        prefetch_l2(lpp + tp);
+        prefetch_l2(odp + tp);
+        if (HAS_KL) prefetch_l2(rfp + tp);
+      }
+    }
+  }
   flush(run_row, run_cnt);
   // block total of valid tokens -> one global atomic
 #pragma unroll
