@@ -169,6 +169,19 @@ int pl_debug_tail_halves(int tiles, int pairs);
 int pl_debug_set_dw_finish(int mode);
 
 /*
+ * Fused path with several bf16 row chunks run in shared launches, how many
+ * rows one dW contribution covers: 1 = each chunk's dW contribution is its own
+ * GEMM job (K = the chunk's rows); 2 = chunks 2i and 2i+1 contribute through one
+ * job whose K runs over both chunks' rows (the earlier chunk's dlogits wait one
+ * launch in the workspace, which then holds three chunks' logits); 0 restores
+ * the default (2).  The dlogits of a pair then share the scale 2^0, so one
+ * epilogue scale undoes both.  Applies to later calls on this process (the
+ * workspace size of pl_fused_linear_grpo_workspace_bytes allows for either).
+ * Returns PL_ERR_ARG for another value.
+ */
+int pl_debug_set_dw_pair(int mode);
+
+/*
  * The GEMM's dynamic tile-queue order (host logic): jobs of tiles[0..njobs)
  * tiles, numbered in job order; queue entry q runs tile out[q].  The tiles of
  * jobs [0, q_f0) come first in order, then those of jobs [q_f0, q_w) spread

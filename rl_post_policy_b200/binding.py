@@ -104,6 +104,8 @@ _lib.pl_debug_tail_halves.argtypes = [_I, _I]
 _lib.pl_debug_tail_halves.restype = _I
 _lib.pl_debug_set_dw_finish.argtypes = [_I]
 _lib.pl_debug_set_dw_finish.restype = _I
+_lib.pl_debug_set_dw_pair.argtypes = [_I]
+_lib.pl_debug_set_dw_pair.restype = _I
 _lib.pl_debug_set_gemm_merge.argtypes = [_I]
 _lib.pl_debug_set_gemm_merge.restype = _I
 _lib.pl_debug_queue_tiles.argtypes = [_I, _P, _I, _I, _P]
@@ -124,7 +126,7 @@ EXPORTED = ("pl_init", "pl_loss", "pl_loss_ex", "pl_loss_static", "pl_fused_line
             "pl_debug_launch_count", "pl_debug_set_wait", "pl_debug_set_rkl_cluster", "pl_debug_set_gemm_tile", "pl_debug_pair_tiles",
             "pl_debug_pick_tile", "pl_debug_set_loss_path", "pl_debug_pick_split", "pl_debug_set_gemm_split",
             "pl_debug_set_rkl_path", "pl_debug_set_gemm_merge", "pl_debug_queue_tiles",
-            "pl_debug_set_dw_finish", "pl_debug_set_gemm_tail", "pl_debug_tail_halves")
+            "pl_debug_set_dw_finish", "pl_debug_set_gemm_tail", "pl_debug_tail_halves", "pl_debug_set_dw_pair")
 
 
 class PLError(RuntimeError):
@@ -344,6 +346,12 @@ def pl_debug_set_gemm_tail(mode: int) -> int:
 def pl_debug_tail_halves(tiles: int, pairs: int) -> int:
     """Test hook: tiles of the last partial wave that run in halves (0: none)."""
     return int(_lib.pl_debug_tail_halves(int(tiles), int(pairs)))
+
+
+def pl_debug_set_dw_pair(mode: int) -> int:
+    """Test hook: several bf16 chunks -- 1 one dW job per chunk, 2 one per pair of chunks
+    (K over both chunks' rows; the default, 0)."""
+    return int(_lib.pl_debug_set_dw_pair(int(mode)))
 
 
 def pl_debug_set_dw_finish(mode: int) -> int:

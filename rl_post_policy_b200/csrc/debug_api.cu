@@ -98,6 +98,12 @@ extern "C" int pl_debug_set_dw_finish(int mode) {
   return PL_OK;
 }
 
+extern "C" int pl_debug_set_dw_pair(int mode) {
+  if (mode < 0 || mode > 2) return PL_ERR_ARG;
+  debug_knobs().dw_pair = mode;
+  return PL_OK;
+}
+
 extern "C" int pl_debug_set_gemm_merge(int mode) {
   if (mode < 0 || mode > 2) return PL_ERR_ARG;
   debug_knobs().gemm_merge = mode;

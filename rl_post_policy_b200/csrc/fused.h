@@ -73,6 +73,8 @@ struct DlogitsArgs {
   int64_t ld;
   int64_t row0, rows, V;
   int chunk;
+  int unit_scale;     // 1: dz is stored unscaled (2^0), whatever max|g| is (bf16 chunks whose
+                      // dW contributions share one GEMM job and so one epilogue scale)
   int dbias_mode;
   float* dbias_acc;
   void* dbias;

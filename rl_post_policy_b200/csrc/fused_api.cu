@@ -29,6 +29,8 @@ int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
   int64_t N = 0, C = 1024, Cbuf = 1, nchunks = 0, ld = 0, logits_bytes = 0;
+  int nslots = 1;    // chunk-sized slots of the logits region
+  bool pair = false; // bf16, dW wanted, several chunks: chunks 2i and 2i+1 share one dW job
   int ntv = 0, nparts = 0, part_stride = 1;  // 256-column vocabulary tiles; LSE partials per row
   FusedOffsets off{};
 };
@@ -65,10 +67,14 @@ Plan make_plan(int64_t bs, int64_t T, int64_t H, int64_t V, uint32_t mode, bool 
   p.off.zt_ref = region(4 * p.Cbuf);
   p.off.part = region(8 * p.Cbuf * (int64_t)p.nparts);
   p.off.part_ref = region(8 * p.Cbuf * (int64_t)p.nparts);
-  // two halves when several chunks run with a backward: chunk c's backward and
-  // chunk c+1's forward share a launch (see run_pipeline)
+  // Several chunks: chunk c's backward and chunk c+1's forward share a launch, so
+  // two chunks' logits are live at once (see run_pipeline); with paired dW jobs
+  // (bf16 with a weight gradient) chunk 2i's dlogits also wait for chunk 2i+1's,
+  // and from three chunks on a third slot takes chunk 2i+2's forward meanwhile.
+  p.pair = need_dW && p.nchunks > 1 && ((mode & PL_DTYPE_MASK) == PL_BF16);
+  p.nslots = p.nchunks > 1 ? ((p.pair && p.nchunks > 2) ? 3 : 2) : 1;
   p.logits_bytes = align_up(2 * p.Cbuf * p.ld, 1024);
-  p.off.logits = region(p.logits_bytes * (p.nchunks > 1 ? 2 : 1));
+  p.off.logits = region(p.logits_bytes * p.nslots);
   p.off.dw_acc = region((need_dW && p.nchunks > 1) ? 4 * V * H : 0);
   p.off.dx_acc = region(4 * p.Cbuf * (H > 0 ? H : 0));
   p.off.db_acc = region((need_dbias && p.nchunks > 1) ? 4 * V : 0);
@@ -157,9 +163,17 @@ pl_status run_pipeline(const Pipe& q) {
   // compute-heavy forward tiles, and each launch's tail is paid once.  The two
   // chunks' logits live in alternate halves of the logits region.
   const bool merge = has_gemm_bwd && plan.nchunks > 1 && debug_knobs().gemm_merge != 1;
+  // bf16 chunks 2i and 2i+1 contribute to dW through one job whose K runs over both
+  // chunks' rows (half the fp32 accumulator traffic and twice the k-steps per dW
+  // tile); their dlogits then share the scale 2^0
+  const bool pair = merge && dW && plan.pair && debug_knobs().dw_pair != 1;
+  const int nslots = merge ? (pair ? plan.nslots : 2) : 1;
   auto logits_of = [&](int64_t c) -> unsigned char* {
-    return ws + plan.off.logits + (merge ? (c & 1) * plan.logits_bytes : 0);
+    return ws + plan.off.logits + (c % nslots) * plan.logits_bytes;
   };
+  // dW contributions: one per chunk, or one per pair of chunks (the last chunk of
+  // an odd count alone)
+  const int64_t ncontrib = pair ? (plan.nchunks + 1) / 2 : plan.nchunks;
   auto rows_of = [&](int64_t c) -> int64_t { return (N - c * plan.C) < plan.C ? (N - c * plan.C) : plan.C; };
   // Several chunks: the last chunk adds into the fp32 accumulator like the others
   // and a streaming kernel rounds it (at the copy bandwidth).  On request, the
@@ -226,31 +240,44 @@ pl_status run_pipeline(const Pipe& q) {
     return true;
   };
 
-  // Chunk c's dW contribution (dz^T X_chunk), appended to g.  Several chunks:
-  // the first stores its fp32 contribution, every later one adds its own
-  // through the TMA unit (the memory system does the add, so the epilogue never
-  // waits on a load), and the sum is rounded to the model dtype once, after the
-  // last chunk.
-  auto add_dw = [&](GemmParams& g, int64_t c, int& nm) -> bool {
-    const int64_t r0 = c * plan.C, rows = rows_of(c);
+  // The dW contribution of chunks c0..c1 (c1 = c0, or c0 + 1 for a pair: K runs over
+  // both chunks' rows, in two segments), appended to g.  Several contributions:
+  // the first stores its fp32 result, every later one adds its own through the TMA
+  // unit (the memory system does the add, so the epilogue never waits on a load),
+  // and the sum is rounded to the model dtype once, after the last.
+  auto add_dw = [&](GemmParams& g, int64_t c0, int64_t c1, int& nm) -> bool {
+    const int64_t r0 = c0 * plan.C, rows0 = rows_of(c0);
+    const int64_t rows = rows0 + (c1 > c0 ? rows_of(c1) : 0);
+    const int64_t ci = pair ? c0 / 2 : c0;  // index of this contribution
     const int ma = nm++, mb = nm++, mo = nm++;
-    if (!make_tmap_2d(&g.maps[ma], logits_of(c), dt, V, rows, plan.ld * esz, 64, kBK) ||
-        !make_tmap_2d(&g.maps[mb], Xb + r0 * H * esz, dt, H, rows, H * esz, 64, kBK))
+    if (!make_tmap_2d(&g.maps[ma], logits_of(c0), dt, V, rows0, plan.ld * esz, 64, kBK) ||
+        !make_tmap_2d(&g.maps[mb], Xb + r0 * H * esz, dt, H, rows0, H * esz, 64, kBK))
       return false;
     GemmJob& j = g.jobs[g.njobs++];
     j.a_map = ma; j.b_map = mb; j.a_mn = 1; j.b_mn = 1;
+    if (c1 > c0) {
+      // chunk c1's rows as the second K segment (chunk c0 is a full chunk: C rows, a whole
+      // number of k-steps)
+      const int ma2 = nm++, mb2 = nm++;
+      const int64_t r1 = c1 * plan.C;
+      if (!make_tmap_2d(&g.maps[ma2], logits_of(c1), dt, V, rows_of(c1), plan.ld * esz, 64, kBK) ||
+          !make_tmap_2d(&g.maps[mb2], Xb + r1 * H * esz, dt, H, rows_of(c1), H * esz, 64, kBK))
+        return false;
+      j.k_seg = (int)(rows0 / kBK); j.a_map2 = ma2; j.b_map2 = mb2;
+    }
     j.M = (int)V; j.N = (int)H; j.K = (int)rows; j.n_inner = 1; j.epi = kEpiStore;
-    j.out_ld = H; j.scale = reinterpret_cast<const float*>(ws + plan.off.inv_scale) + c;
+    // a pair's dlogits share the scale 2^0 (unit_scale), so chunk c0's factor serves both
+    j.out_ld = H; j.scale = reinterpret_cast<const float*>(ws + plan.off.inv_scale) + c0;
     float* acc = reinterpret_cast<float*>(ws + plan.off.dw_acc);
     j.acc_in = nullptr;
-    if (plan.nchunks == 1) {
+    if (ncontrib == 1) {
       j.out = dW; j.out_f32 = 0; j.out_path = kOutDirect;
       if (aligned(dW, 16)) {
         if (!make_tmap_2d(&g.maps[mo], dW, dt, H, V, H * esz, kOutBoxN16, kOutBoxM)) return false;
         j.out_path = kOutTmaStore; j.out_map = mo;
       }
-    } else if (c + 1 == plan.nchunks && fuse_finish) {
-      // the last chunk: its epilogue adds the accumulator of the earlier chunks and
+    } else if (ci + 1 == ncontrib && fuse_finish) {
+      // the last contribution: its epilogue adds the accumulator of the earlier ones and
       // rounds the sum to the model dtype in one pass (no separate rounding kernel)
       j.out = dW; j.out_f32 = 0; j.acc_in = acc; j.out_path = kOutDirect;
       if (aligned(dW, 16)) {
@@ -260,7 +287,7 @@ pl_status run_pipeline(const Pipe& q) {
     } else {
       if (!make_tmap_2d(&g.maps[mo], acc, DType::F32, H, V, H * 4, kOutBoxN, kOutBoxM)) return false;
       j.out = acc; j.out_f32 = 1; j.out_map = mo;
-      j.out_path = c == 0 ? kOutTmaStore : kOutTmaReduce;
+      j.out_path = ci == 0 ? kOutTmaStore : kOutTmaReduce;
     }
     return true;
   };
@@ -285,6 +312,7 @@ pl_status run_pipeline(const Pipe& q) {
     DlogitsArgs da{};
     da.ws = ws; da.off = plan.off; da.targets = targets; da.logits = logits_of(c); da.ld = plan.ld;
     da.row0 = c * plan.C; da.rows = rows_of(c); da.V = V; da.chunk = (int)c;
+    da.unit_scale = pair ? 1 : 0;
     da.dbias_mode = dbias ? acc_mode(c, plan.nchunks) : kAccNone;
     da.dbias_acc = reinterpret_cast<float*>(ws + plan.off.db_acc); da.dbias = dbias;
     da.db_part = reinterpret_cast<float*>(ws + plan.off.db_part);
@@ -343,7 +371,7 @@ pl_status run_pipeline(const Pipe& q) {
       // ---- backward GEMMs: dX rows of this chunk, dW contribution ----
       GemmParams bp = fresh();
       nm = 0;
-      if ((dX && !add_dx(bp, c, nm)) || (dW && !add_dw(bp, c, nm))) return PL_ERR_CUDA;
+      if ((dX && !add_dx(bp, c, nm)) || (dW && !add_dw(bp, c, c, nm))) return PL_ERR_CUDA;
       if (!launch_backward_alone(bp, c)) return PL_ERR_CUDA;
     }
   } else {
@@ -359,15 +387,23 @@ pl_status run_pipeline(const Pipe& q) {
     for (int64_t c = 0; c < plan.nchunks; ++c) {
       GemmParams g = fresh();
       int nm = 0;
+      // the dW contribution this launch carries: chunk c's own, or with pairs that of
+      // chunks c-1 and c (c odd), or chunk c's alone (the last of an odd count)
+      int64_t w0 = -1, w1 = -1;
+      if (dW) {
+        if (!pair) w0 = w1 = c;
+        else if (c & 1) { w0 = c - 1; w1 = c; }
+        else if (c + 1 == plan.nchunks) w0 = w1 = c;
+      }
       if (c + 1 < plan.nchunks) {
         // queue order: dX tiles (long, K = V) first, then the next chunk's
-        // forward tiles interleaved evenly with this chunk's dW tiles
+        // forward tiles interleaved evenly with the dW tiles
         if (dX && !add_dx(g, c, nm)) return PL_ERR_CUDA;
         g.q_f0 = g.njobs;
         if (!add_fwd(g, c + 1, nm)) return PL_ERR_CUDA;
-        if (dW) {
+        if (w0 >= 0) {
           g.q_w = g.njobs;
-          if (!add_dw(g, c, nm)) return PL_ERR_CUDA;
+          if (!add_dw(g, w0, w1, nm)) return PL_ERR_CUDA;
         }
         g.dyn = 1;
         g.ctr = reinterpret_cast<unsigned*>(ws + kWsGemmQueue);
@@ -379,12 +415,12 @@ pl_status run_pipeline(const Pipe& q) {
         if (!ok(launch_gemm(g, dt, s))) return PL_ERR_CUDA;
         if (!combine(c + 1) || !dlogits(c + 1)) return PL_ERR_CUDA;
       } else {
-        if ((dX && !add_dx(g, c, nm)) || (dW && !add_dw(g, c, nm))) return PL_ERR_CUDA;
+        if ((dX && !add_dx(g, c, nm)) || (w0 >= 0 && !add_dw(g, w0, w1, nm))) return PL_ERR_CUDA;
         if (!launch_backward_alone(g, c)) return PL_ERR_CUDA;
       }
     }
   }
-  if (dW && plan.nchunks > 1 && !fuse_finish &&
+  if (dW && ncontrib > 1 && !fuse_finish &&
       !ok(launch_convert(reinterpret_cast<const float*>(ws + plan.off.dw_acc), dW, V * H, dt, s)))
     return PL_ERR_CUDA;
 

@@ -9,7 +9,8 @@
 //                      the KL term, g = dLoss/dlogp and the chunk's loss partials.
 //   dlogits_kernel  -- in place over the chunk's logits workspace:
 //                      dz = g * (onehot(target) - exp(z - lse)) * 2^e, stored in the
-//                      model dtype, and the column sums of dz (the bias gradient),
+//                      model dtype (2^e keeps fp16 dz in range; bf16 chunks paired
+//                      into one dW job take e = 0), and the column sums of dz (the bias gradient),
 //                      stored / accumulated in fp32 / converted like dW.
 //   finalize_kernel -- fixed-order sum of every chunk's loss partials.
 //   convert_kernel  -- the fp32 dW accumulator of a multi-chunk call, rounded
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(256, 3) dlogits_kernel(const __grid_constant__
   // power-of-two scale 2^e keeping max|dz| * 2^e <= 2^14 (fp16 range), exact to undo
   const float gm = __uint_as_float(reinterpret_cast<const unsigned*>(ws + a.off.gmax)[a.chunk]);
   int e = 0;
-  if (gm > 0.0f) {
+  if (gm > 0.0f && !a.unit_scale) {
     e = 14 - (int)ceilf(log2f(gm));
     e = max(-100, min(100, e));
   }

@@ -65,6 +65,12 @@ struct GemmJob {
   // twice as many pairs (set by launch_gemm; 0 = none).
   int tail;
   int n_inner;             // 1: consecutive tiles walk N first (share the A rows)
+  // Two K segments: k-steps [0, k_seg) read A and B through a_map / b_map, and
+  // k-steps [k_seg, k_steps) through a_map2 / b_map2, counting K from 0 again
+  // (two row chunks of the fused path contributing to dW through one job: their
+  // dlogits sit in different workspace slots).  k_seg = 0: one segment.
+  int k_seg;
+  int a_map2, b_map2;
   int tile_begin;          // first global tile index of this job
   int epi;
   // kEpiLse
@@ -89,7 +95,7 @@ struct GemmJob {
 };
 
 constexpr int kMaxJobs = 4;
-constexpr int kMaxMaps = 12;
+constexpr int kMaxMaps = 14;
 
 struct __align__(64) GemmParams {
   CUtensorMap maps[kMaxMaps];

@@ -351,6 +351,10 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
     for (int q = 0; q < p.njobs; ++q) {
       prefetch_tmap(&p.maps[p.jobs[q].a_map]);
       prefetch_tmap(&p.maps[p.jobs[q].b_map]);
+      if (p.jobs[q].k_seg > 0) {
+        prefetch_tmap(&p.maps[p.jobs[q].a_map2]);
+        prefetch_tmap(&p.maps[p.jobs[q].b_map2]);
+      }
       if (p.jobs[q].out_path != kOutDirect) prefetch_tmap(&p.maps[p.jobs[q].out_map]);
     }
   }
@@ -415,8 +419,6 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
         const GemmJob& j = p.jobs[tc.job];
         const int m0 = tc.mb * kPairM + (int)rank * kBM;
         const int nt0 = tc.nb * Cfg::kTileN + (int)rank * kBNh;
-        const CUtensorMap* amap = &p.maps[j.a_map];
-        const CUtensorMap* bmap = &p.maps[j.b_map];
         // a half tile loads one B half (its columns) into the stage's first B slot
         const int nb_loads = tc.half < 0 ? NH : 1;
         const uint32_t stage_tx = 2 * (kABytes + (uint32_t)nb_loads * kBBytes) + p.extra_tx;
@@ -426,7 +428,12 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = ring + stage * kStageBytes;
           uint8_t* b_dst = a_dst + kABytes;
-          const int k0 = (tc.kb + k) * kBK;
+          // the job's second K segment (if any) through its own maps, K from 0
+          const int kg = tc.kb + k;
+          const bool seg2 = j.k_seg > 0 && kg >= j.k_seg;
+          const CUtensorMap* amap = &p.maps[seg2 ? j.a_map2 : j.a_map];
+          const CUtensorMap* bmap = &p.maps[seg2 ? j.b_map2 : j.b_map];
+          const int k0 = (seg2 ? kg - j.k_seg : kg) * kBK;
           if (!j.a_mn) {
             tma_load_2d_pair(a_dst, amap, bar, k0, m0);
           } else {

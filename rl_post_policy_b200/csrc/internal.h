@@ -126,6 +126,8 @@ struct DebugKnobs {
                          // accumulator and stores the model dtype
   int gemm_split = 0;    // K split of the backward launch's dX problem: 0 = the host's choice,
                          // 1 = never, 2 = always (when it has at least two k-steps)
+  int dw_pair = 0;       // several bf16 chunks with shared launches: 0 = the host's choice (2),
+                         // 1 = one dW contribution per chunk, 2 = one per pair of chunks (K = 2 C)
 };
 DebugKnobs& debug_knobs();
 

@@ -136,6 +136,32 @@ def test_ragged_multi_tile(dtype, chunk, beta):
         check(inp, got, red, beta)
 
 
+@pytest.mark.parametrize("nchunks", [2, 3, 4, 5])
+def test_paired_weight_gradient(nchunks):
+    # bf16 with several chunks: chunks 2i and 2i+1 contribute to dW through one GEMM
+    # job whose K runs over both chunks' rows (two tensor-map segments), with the
+    # dlogits of every chunk unscaled; the last chunk of an odd count contributes
+    # alone, and two chunks make a single contribution stored straight in bf16.
+    # The last chunk is ragged.  Both ways, and one dW job per chunk, match the
+    # oracle, and dX and the log-probs do not depend on the pairing beyond
+    # rounding (a launch's epilogue warp count, and with it the grouping of the
+    # logsumexp partials, can differ between the two ways under some variants).
+    m = pl()
+    T = 128 * nchunks - 37
+    inp = build_inputs(1, T, 192, 900, torch.bfloat16, 5150 + nchunks, bias=True, len_lo=T - 40, len_hi=T)
+    got = {}
+    try:
+        for mode in (2, 1):
+            assert m.pl_debug_set_dw_pair(mode) == 0
+            got[mode] = run_fused(inp, torch.bfloat16, 1, 0.04, chunk=128)
+            check(inp, got[mode], 1, 0.04)
+    finally:
+        m.pl_debug_set_dw_pair(0)
+    assert np.max(np.abs(got[2]["logp"] - got[1]["logp"])) <= 1e-5
+    assert rel_fro(got[2]["dX"], got[1]["dX"]) <= 1e-3
+    assert m.pl_debug_set_dw_pair(3) != 0
+
+
 def test_two_sided_clip():
     inp = build_inputs(2, 64, 128, 640, torch.bfloat16, 99, bias=False)
     got = run_fused(inp, torch.bfloat16, 1, 0.04, two_sided=True)
