@@ -72,6 +72,22 @@ __device__ __forceinline__ void load16_pairs(const float* p, float2 (&v)[2]) {
   v[1] = make_float2(u.z, u.w);
 }
 
+__device__ __forceinline__ uint4 ld16_raw(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+__device__ __forceinline__ void unpack16_pairs(const uint4& u, const __nv_bfloat16*, float2 (&v)[4]) {
+  const unsigned w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) v[k] = make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u));
+}
+__device__ __forceinline__ void unpack16_pairs(const uint4& u, const __half*, float2 (&v)[4]) {
+  const unsigned w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) v[k] = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+}
+__device__ __forceinline__ void unpack16_pairs(const uint4& u, const float*, float2 (&v)[2]) {
+  v[0] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
+  v[1] = make_float2(__uint_as_float(u.z), __uint_as_float(u.w));
+}
+
 __device__ __forceinline__ void store16_pairs(__nv_bfloat16* p, const float2 (&g)[4]) {
   uint4 u;
   unsigned* w = reinterpret_cast<unsigned*>(&u);
@@ -341,6 +357,15 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
         if (HAS_GRAD) gr[u] = from_f<T>(valid ? dterm * scale : 0.0f);
       }
     };
+    uint4 cu_l = make_uint4(0u, 0u, 0u, 0u), cu_o = cu_l, cu_r = cu_l;
+    if constexpr (VEC) {
+      const int64_t tf = t0 + (int64_t)tid * VW;
+      if (tf + VW <= t1) {
+        cu_l = ld16_raw(lp + tf);
+        cu_o = ld16_raw(od + tf);
+        if (HAS_KL) cu_r = ld16_raw(rf + tf);
+      }
+    }
     for (int64_t t = t0 + (int64_t)tid * VW; t < t1; t += (int64_t)kThreads * VW) {
       if constexpr (VEC) {
         if (t + VW > t1) {
@@ -348,19 +373,28 @@ __global__ void __launch_bounds__(kThreads, 2) loss_kernel(LossArgs a) {
           continue;
         }
         constexpr int NP = VW / 2;
-        {
-          // bring this thread's next vector toward the SM while this one is computed
-          const int64_t tn = t + (int64_t)kThreads * VW;
-          if (tn + VW <= t1) {
-            prefetch_l2(lp + tn);
-            prefetch_l2(od + tn);
-            if (HAS_KL) prefetch_l2(rf + tn);
+        // this thread's next vector: its loads in flight while this one is computed,
+        // and the one after it toward L2
+        const int64_t tn = t + (int64_t)kThreads * VW;
+        uint4 nx_l = cu_l, nx_o = cu_o, nx_r = cu_r;
+        if (tn + VW <= t1) {
+          nx_l = ld16_raw(lp + tn);
+          nx_o = ld16_raw(od + tn);
+          if (HAS_KL) nx_r = ld16_raw(rf + tn);
+          const int64_t tnn = tn + (int64_t)kThreads * VW;
+          if (tnn + VW <= t1) {
+            prefetch_l2(lp + tnn);
+            prefetch_l2(od + tnn);
+            if (HAS_KL) prefetch_l2(rf + tnn);
           }
         }
         float2 pl[NP], po[NP], pr[NP], pg[NP];
-        load16_pairs(lp + t, pl);
-        load16_pairs(od + t, po);
-        if (HAS_KL) load16_pairs(rf + t, pr);
+        unpack16_pairs(cu_l, lp, pl);
+        unpack16_pairs(cu_o, od, po);
+        if (HAS_KL) unpack16_pairs(cu_r, rf, pr);
+        cu_l = nx_l;
+        cu_o = nx_o;
+        cu_r = nx_r;
         unsigned bits;
         if (bits_in_smem) {
           bits = s_maskbits[(t - t0) / VW];
