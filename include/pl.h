@@ -181,10 +181,14 @@ pl_status pl_loss_static(const void* policy_lp, const void* old_lp, const void* 
  * persistent tcgen05 GEMM computes the reference and policy logits tile by tile;
  * its epilogue keeps a per-(row, 256-column tile) running max / sum of exponentials
  * and the target logit, and stores the policy logits into a bounded workspace of
- * chunk x V elements (full-batch logits are never materialised).  The logits are
- * then turned into dz in place and a second persistent GEMM computes dX and dW;
- * dW and dbias are accumulated in fp32 across chunks (the first chunk stores, later
- * chunks add, the last converts to the model dtype).
+ * chunk x V elements per slot (full-batch logits are never materialised; two
+ * slots with several chunks, three with several bf16 chunks and a weight
+ * gradient).  The logits are then turned into dz in place and a second
+ * persistent GEMM computes dX and dW (with several chunks, chunk c's backward
+ * GEMM shares a launch with chunk c+1's forward); dW and dbias are accumulated in
+ * fp32 across chunks (the first contribution stores, later ones add, a last pass
+ * converts to the model dtype; bf16 chunks 2i and 2i+1 make one dW contribution
+ * whose K covers both chunks' rows).
  *
  *   X [N,H], W [V,H], bias [V] or NULL : model dtype (PL_F16 or PL_BF16).
  *   targets [N] int64                  : sampled token ids; a row whose id is outside
