@@ -5,10 +5,12 @@ Loss-only kernel: bs, seq, dtype, reduction, beta, clip form, clip bounds,
 advantage dtype, arbitrary (non-prefix) masks and misaligned pointers.  Fused
 linear path: batch and sequence sizes, hidden sizes down to one 16-byte row,
 vocabularies smaller than one tile and ragged ones, bias, beta, reduction and
-chunking.  Tolerances as in the dedicated tests; tokens within rounding of a
-clip bound may take either side of the min() and are left out of the
-element-wise loss-gradient comparison (loss-only) or moved off the bound in the
-input recipe (fused).
+chunking.  Reverse KL: rows (across several 512-row blocks of the row
+dealing), vocabulary sizes, dtypes, mask densities including none and all,
+cluster sizes and the forward-only form.  Tolerances as in the dedicated
+tests; tokens within rounding of a clip bound may take either side of the
+min() and are left out of the element-wise loss-gradient comparison
+(loss-only) or moved off the bound in the input recipe (fused).
 """
 import numpy as np
 import pytest
@@ -165,3 +167,52 @@ def test_fused_path_random_shapes(bs, T, H, V, dtype, bias, beta, red, chunk, se
     for k, t in (("dX", dX), ("dW", dW), ("dbias", db)):
         if t is not None:
             assert rel(t, want[k]) <= 1e-2, k
+
+
+@settings(**dict(SETTINGS, max_examples=40))
+@given(N=st.integers(1, 1400), V=st.integers(1, 2500),
+       dtype=st.sampled_from([torch.bfloat16, torch.float16, torch.float32]),
+       keep=st.sampled_from([0.0, 0.05, 0.5, 0.9, 1.0, None]), cl=st.sampled_from([0, 1, 2, 4, 8]),
+       grad=st.booleans(), seed=st.integers(0, 2 ** 20))
+def test_reverse_kl_random_shapes(N, V, dtype, keep, cl, grad, seed):
+    # valid rows are dealt to the clusters by their rank among the valid rows, in
+    # blocks of 512 rows, and masked rows after them: any count, density and order
+    import rl_post_policy_b200 as pl
+    dev = torch.device("cuda")
+    inp = synth.reverse_kl_inputs(1, N, V, dtype, seed)
+    s, t = inp["student"].reshape(N, V), inp["teacher"].reshape(N, V)
+    if keep is None:
+        mask = None
+    else:
+        g = torch.Generator().manual_seed(seed + 7)
+        mask = (torch.rand(N, generator=g) < keep).to(torch.uint8)
+    want = oracle.reverse_kl(s, t, mask, want_grad=grad)
+    assert pl.pl_debug_set_rkl_cluster(cl) == 0
+    try:
+        S, T = s.to(dev), t.to(dev)
+        G = torch.full_like(S, float("nan")) if grad else None
+        M = mask.to(dev) if mask is not None else None
+        loss = torch.full((1,), float("nan"), device=dev)
+        kl = torch.full((N,), float("nan"), device=dev)
+        nv = torch.full((1,), -1, dtype=torch.int64, device=dev)
+        wsb = pl.pl_reverse_kl_workspace_bytes(N, V)
+        ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+        pl.check(pl.pl_reverse_kl(S, T, M, N, V, pl.dtype_mode(dtype), loss, G, kl, nv, ws, wsb))
+        torch.cuda.synchronize()
+        assert pl.pl_device_status(ws) == 0
+    finally:
+        pl.pl_debug_set_rkl_cluster(0)
+    valid = np.ones(N, bool) if mask is None else mask.numpy() != 0
+    assert int(nv.item()) == int(valid.sum())
+    wl = float(want["loss"])
+    assert abs(loss.item() - wl) <= 1e-4 * abs(wl) + 1e-7, (loss.item(), wl)
+    wk = np.asarray(want["kl_rows"]).reshape(-1)
+    gk = kl.cpu().double().numpy()
+    assert np.all(np.abs(gk[valid] - wk[valid]) <= 1e-5 + 1e-4 * np.abs(wk[valid]))
+    assert np.all(gk[~valid] == 0.0)
+    if grad:
+        gg = G.float().cpu().double().numpy()
+        wg = np.asarray(want["grad"]).reshape(N, V)
+        err = np.linalg.norm(gg - wg) / max(np.linalg.norm(wg), 1e-300)
+        assert err <= (1e-4 if dtype == torch.float32 else 1e-2), err
+        assert np.all(gg[~valid] == 0.0)
