@@ -160,8 +160,8 @@ pl_status run_pipeline(const Pipe& q) {
   // Several chunks with a backward GEMM: chunk c's backward and chunk c+1's
   // forward share one launch (their tiles do not depend on each other), so the
   // memory-heavy dW tiles with their fp32 accumulator adds run beside the
-  // compute-heavy forward tiles, and each launch's tail is paid once.  The two
-  // chunks' logits live in alternate halves of the logits region.
+  // compute-heavy forward tiles, and each launch's tail is paid once.  The chunks'
+  // logits take turns in the logits region's slots (chunk c in slot c mod slots).
   const bool merge = has_gemm_bwd && plan.nchunks > 1 && debug_knobs().gemm_merge != 1;
   // bf16 chunks 2i and 2i+1 contribute to dW through one job whose K runs over both
   // chunks' rows (half the fp32 accumulator traffic and twice the k-steps per dW
