@@ -84,6 +84,29 @@ def test_workspace_sizes_grow_with_batch():
     assert pl.pl_loss_workspace_bytes(16, 1024) >= 256 + 16 * 8
 
 
+def test_fused_workspace_logits_slots():
+    # The fused path's logits region holds one chunk-sized slot for one chunk, two
+    # with several (a chunk's backward shares a launch with the next chunk's
+    # forward), and three with several bf16 chunks and a weight gradient from three
+    # chunks on (chunks 2i and 2i+1 make one dW contribution, so chunk 2i's dlogits
+    # wait one launch).  A slot is C x ceil(V/64)*64 16-bit values.
+    H, V, C = 256, 1000, 128
+    slot = C * 1024 * 2
+
+    def ws(bs, dtype, dW):
+        mode = dtype | pl.PL_CHUNK_ROWS(C)
+        return pl.pl_fused_linear_grpo_workspace_bytes(bs, C, H, V, mode, dW, 0)
+
+    for dtype in (pl.PL_BF16, pl.PL_F16):
+        # one chunk -> two chunks: one more slot, plus the fp32 dW accumulator with dW
+        assert ws(2, dtype, 0) - ws(1, dtype, 0) >= slot
+    # three chunks: bf16 with dW has a third slot, fp16 and bf16 without dW do not
+    assert ws(3, pl.PL_BF16, 1) - ws(3, pl.PL_F16, 1) == slot
+    assert ws(3, pl.PL_BF16, 0) == ws(3, pl.PL_F16, 0)
+    # two chunks: the pair needs no third slot
+    assert ws(2, pl.PL_BF16, 1) == ws(2, pl.PL_F16, 1)
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
 def test_valid_call_without_device_reports_cuda_error():
     assert _loss() in (pl.PL_ERR_CUDA, pl.PL_ERR_ARCH)
