@@ -650,6 +650,14 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
         const int n0 = (tc.half >= 0 && h > 0) ? j.N : tc.nb * Cfg::kTileN + colh * kBN;
         const int grp = tc.nb * NH + colh;  // index of this 256-column group along N
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (NH == 1 ? acc : h) * kBN;
+        // hands the group's accumulator columns back to the issuer (once per group)
+        bool released = false;
+        auto release = [&]() {
+          if (released) return;
+          released = true;
+          tc_fence_before();
+          mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&tempty[NH == 1 ? acc : h]), 0));
+        };
         if (n0 >= j.N) {
           // past the end of N: zeros only, nothing to store
         } else if (j.epi == kEpiLse) {
@@ -787,37 +795,9 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
           const CUtensorMap* omap = &p.maps[j.out_map];
           const int y = m0 + quarter * 32;
           const int step = j.out_f32 ? 1 : 2;  // 32-column TMEM slices per box
-  #pragma unroll 1
-          for (int c = c_lo; c < c_hi; c += step) {
-            uint32_t w[32];
-            float v[32];
-            tmem_ld_32x32b_x32(taddr + c * 32, v);
-            if (j.out_f32) {
-  #pragma unroll
-              for (int q = 0; q < 32; ++q) w[q] = __float_as_uint(v[q] * sc);
-            } else if (j.acc_in) {
-              // the fp32 accumulator of the earlier chunks added to this tile, then
-              // rounded once to the model dtype (the last chunk of a multi-chunk dW)
-              const float* arow = j.acc_in + (int64_t)(row_ok ? row : 0) * j.out_ld;
-              const int colA = n0 + c * 32;
-              float sa = row_ok ? 1.0f : 0.0f;  // rows past M: no load, dropped by the TMA store
-              if (row_ok) scale_add_row32(arow + colA, v, sc, min(32, j.N - colA));
-              else sa = sc;
-  #pragma unroll
-              for (int q = 0; q < 16; ++q) w[q] = pack2<T>(v[2 * q] * sa, v[2 * q + 1] * sa);
-              tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
-              if (row_ok) scale_add_row32(arow + colA + 32, v, sc, min(32, j.N - colA - 32));
-  #pragma unroll
-              for (int q = 0; q < 16; ++q) w[16 + q] = pack2<T>(v[2 * q] * sa, v[2 * q + 1] * sa);
-            } else {
-  #pragma unroll
-              for (int q = 0; q < 16; ++q) w[q] = pack2<T>(v[2 * q] * sc, v[2 * q + 1] * sc);
-              tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
-  #pragma unroll
-              for (int q = 0; q < 16; ++q) w[16 + q] = pack2<T>(v[2 * q] * sc, v[2 * q + 1] * sc);
-            }
-            const int col0 = n0 + c * 32;
-            if (col0 >= j.N || y >= j.M) continue;
+          // one staged box of packed words: columns [col0, col0 + 128 bytes)
+          auto store_box = [&](const uint32_t (&w)[32], int col0) {
+            if (col0 >= j.N || y >= j.M) return;
             // the box's previous contents have been read out by the TMA unit
             if (lane == 0) bulk_wait_group_read<kBoxes - 1>();
             __syncwarp();
@@ -835,6 +815,56 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
               bulk_commit_group();
             }
             if (kBoxes > 1) sbuf ^= 1;
+          };
+          if (kCG == 2 && !j.acc_in && !j.out_f32) {
+            // 8 warps, a 16-bit output: this warp's 128 columns of the group come into
+            // registers first (scaled and packed, 16 columns per tensor-memory load) and
+            // the accumulator half goes back to the issuer before any of them is staged,
+            // so the next tile's MMAs into it overlap the stores (the issuer waited for
+            // the staging of each half before)
+            uint32_t w[2][32];
+  #pragma unroll
+            for (int b = 0; b < 8; ++b) {
+              float v[16];
+              tmem_ld_32x32b_x16(taddr + (uint32_t)(c_lo * 32 + b * 16), v);
+  #pragma unroll
+              for (int q = 0; q < 8; ++q) w[b >> 2][(b & 3) * 8 + q] = pack2<T>(v[2 * q] * sc, v[2 * q + 1] * sc);
+            }
+            release();
+  #pragma unroll
+            for (int b = 0; b < 2; ++b) store_box(w[b], n0 + (c_lo + 2 * b) * 32);
+          } else {
+  #pragma unroll 1
+            for (int c = c_lo; c < c_hi; c += step) {
+              uint32_t w[32];
+              float v[32];
+              tmem_ld_32x32b_x32(taddr + c * 32, v);
+              if (j.out_f32) {
+  #pragma unroll
+                for (int q = 0; q < 32; ++q) w[q] = __float_as_uint(v[q] * sc);
+              } else if (j.acc_in) {
+                // the fp32 accumulator of the earlier chunks added to this tile, then
+                // rounded once to the model dtype (the last chunk of a multi-chunk dW)
+                const float* arow = j.acc_in + (int64_t)(row_ok ? row : 0) * j.out_ld;
+                const int colA = n0 + c * 32;
+                float sa = row_ok ? 1.0f : 0.0f;  // rows past M: no load, dropped by the TMA store
+                if (row_ok) scale_add_row32(arow + colA, v, sc, min(32, j.N - colA));
+                else sa = sc;
+  #pragma unroll
+                for (int q = 0; q < 16; ++q) w[q] = pack2<T>(v[2 * q] * sa, v[2 * q + 1] * sa);
+                tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
+                if (row_ok) scale_add_row32(arow + colA + 32, v, sc, min(32, j.N - colA - 32));
+  #pragma unroll
+                for (int q = 0; q < 16; ++q) w[16 + q] = pack2<T>(v[2 * q] * sa, v[2 * q + 1] * sa);
+              } else {
+  #pragma unroll
+                for (int q = 0; q < 16; ++q) w[q] = pack2<T>(v[2 * q] * sc, v[2 * q + 1] * sc);
+                tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v);
+  #pragma unroll
+                for (int q = 0; q < 16; ++q) w[16 + q] = pack2<T>(v[2 * q] * sc, v[2 * q + 1] * sc);
+              }
+              store_box(w, n0 + c * 32);
+            }
           }
         } else {
           const float sc = j.scale ? __ldg(j.scale) : 1.0f;
@@ -853,8 +883,7 @@ __global__ void __launch_bounds__(gemm_threads(EW), 1) gemm_kernel(const __grid_
             else store_row32<T>(reinterpret_cast<T*>(j.out) + off, v, nvalid);
           }
         }
-        tc_fence_before();
-        mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&tempty[NH == 1 ? acc : h]), 0));
+        release();
       }  // groups
       if (NH == 1) {
         if (++acc == 2) {
